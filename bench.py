@@ -1,0 +1,360 @@
+#!/usr/bin/env python
+"""LatentMoE layer-forward benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--T T]
+    python bench.py --impl reference ...
+
+One step = one whole layer forward (router, top-k, dispatch, down-projection,
+routed experts, combine, RMSNorm, shared experts, up-projection) over the
+workload's batch, inputs resident in HBM.  Prints one JSON line (rank 0).
+
+N > 1 (launched with torch.distributed.run) runs N independent replicas, one
+per GPU, each on its own batch: the layer's rows are independent and there is
+no exchange step, so there is no data-path collective (weak scaling).  The
+NCCL process group is used only for the barrier and the max over ranks of the
+timed region.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+layer has) on the host cores, each step a bounded sample of token rows.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % of tensor-core or HBM roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--workload", default="acc_d2048")
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--gemm", type=int, default=0, help="0 tensor cores, 1 CUDA cores")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            j = json.load(fh)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), float(j.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- algorithmic model
+def layer_flops(w, T):
+    """2dE + 4dl + 6klf + 12 d f_s per token (router, projections, routed, shared)."""
+    return T * (2 * w.d * w.E + 4 * w.d * w.l + 6 * w.k * w.l * w.f + 12 * w.d * w.f_s)
+
+
+def layer_bytes(w, T, touched):
+    B = w.item_bytes
+    weights = touched * 3 * w.l * w.f * B + 6 * w.d * w.f_s * B + 2 * w.d * w.l * B + 4 * w.d * w.E
+    io = T * w.d * B * 2 + T * w.k * (4 + B) + T * w.l * B
+    return weights + io
+
+
+def stage_model(w, T, touched):
+    """Per-kernel algorithmic (flops, bytes): operands read once, results written once."""
+    B, S = w.item_bytes, T * w.k
+    return {
+        "router": (2 * T * w.d * w.E, T * w.d * B + 4 * w.d * w.E + 4 * T * w.E),
+        "topk": (0, 4 * T * w.E + T * w.k * (8 + B)),
+        "scan": (0, 0),
+        "dispatch": (0, T * w.k * 16),
+        "down_proj": (2 * T * w.d * w.l, T * w.d * B + w.l * w.d * B + S * w.l * B),
+        "gate_up": (2 * S * 2 * w.f * w.l, touched * 2 * w.f * w.l * B + S * w.l * B + S * w.f * B),
+        "down_combine": (2 * S * w.l * w.f, touched * w.l * w.f * B + S * w.f * B + S * w.l * 4),
+        "combine_norm": (0, S * w.l * 4 + 2 * T * w.l * B),
+        "shared_gate_up": (2 * T * w.d * 4 * w.f_s, T * w.d * B + 4 * w.f_s * w.d * B + T * 2 * w.f_s * B),
+        "final": (2 * T * w.d * (2 * w.f_s + w.l),
+                  T * (2 * w.f_s + w.l) * B + w.d * (2 * w.f_s + w.l) * B + T * w.d * B),
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_id), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def time_oracle(w, x, W, seconds, max_rows=None):
+    """Time the fp64 oracle on a bounded, seeded sample of token rows."""
+    import numpy as np
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    T = x.shape[0]
+    rng = np.random.default_rng(7)
+    n0 = min(cores, T)
+    t0 = time.perf_counter()
+    oracle.forward(x, W, w.k, rows=rng.choice(T, n0, replace=False), eps=w.eps)
+    dt0 = time.perf_counter() - t0
+    n = int(max(n0, min(T if max_rows is None else max_rows, n0 * seconds / max(dt0, 1e-6))))
+    rows = rng.choice(T, n, replace=False)
+    t1 = time.perf_counter()
+    oracle.forward(x, W, w.k, rows=rows, eps=w.eps)
+    dt = time.perf_counter() - t1
+    return n / dt, n, dt, cores
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import lmoe_inputs as li
+    w = li.WORKLOADS[args.workload]
+    T = args.T or w.T
+    x, W = li.tokens(w, T), li.weights(w)
+    # one step = the oracle on a bounded sample of rows, sized to ~4 s
+    _, n, _, cores = time_oracle(w, x, W, 4.0)
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(11)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = rng.choice(T, n, replace=False)
+        t0 = time.perf_counter()
+        oracle.forward(x, W, w.k, rows=rows, eps=w.eps)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_step = sum(times) / len(times)
+    value = n / per_step
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "T": T, "d": w.d, "l": w.l, "f": w.f, "E": w.E, "k": w.k,
+                       "f_shared": w.f_s, "sample_rows_per_step": n},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{n} seeded token rows of {T} per step (fp64 C oracle, threads over rows)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- own arm
+def run_own(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import lmoe_inputs as li
+    import latent_space_routed_b200 as lm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = li.WORKLOADS[args.workload]
+    T = args.T or w.T
+    W = li.weights(w)
+    x_cpu = li.tokens(w, T, seed=w.seed + 1000 * rank)
+    layer = lm.LatentMoE(lm.config_for(w, gemm=args.gemm), {k: v.to(dev) for k, v in W.items()})
+    x = x_cpu.to(dev)
+    out = layer.empty_outputs(T)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    # warm-up (also yields the realised touched-expert count)
+    for _ in range(max(args.warmup, 3)):
+        layer.forward_into(x, out)
+    torch.cuda.synchronize()
+    layer.check_device(T)
+    counts = layer.region(T, "counts", torch.int32, (w.E,)).cpu().numpy()
+    touched = int((counts > 0).sum())
+
+    ns = lm.LMOE_NUM_STAGES + 1
+    ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(ns)] for _ in range(args.steps)]
+    for evs in ev_stage:   # materialise the events on this device before taking their handles
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    arrays = [(ctypes.c_void_p * ns)(*[e.cuda_event for e in evs]) for evs in ev_stage]
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    gpu_id = 0
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = local_rank
+    clocks = Clocks(gpu_id)
+    time.sleep(0.5)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))                      # evict L2 between timed steps (untimed)
+        lm.lmoe_set_stage_events(layer.handle, arrays[i], ns)
+        ev_a[i].record(stream)
+        layer.forward_into(x, out)
+        ev_b[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    lm.lmoe_set_stage_events(layer.handle, None, 0)
+    layer.check_device(T)
+
+    step_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    stage_ms = {}
+    for si, name in enumerate(lm.STAGE_NAMES):
+        stage_ms[name] = sum(ev_stage[i][si].elapsed_time(ev_stage[i][si + 1]) for i in range(args.steps)) / args.steps
+
+    # end to end through the public API: pinned host x in, host outputs back, copies inside the timing
+    x_host = x_cpu.pin_memory()
+    out_host = layer.empty_outputs(T, device="cpu", pin=True)
+    for _ in range(2):
+        layer.forward_host(x_host, out_host)
+    torch.cuda.synchronize()
+    e_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        e_a[i].record(stream)
+        layer.forward_host(x_host, out_host)
+        e_b[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_a, e_b))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    B = w.item_bytes
+    h2d = T * w.d * B
+    d2h = T * w.d * B + T * w.k * 4 + T * w.k * B + T * w.l * B
+
+    if rank != 0:
+        layer.close()
+        return
+
+    hbm, tf_burst, tf_sus, peak_src = peaks()
+    ms = total_ms / args.steps
+    value = world * T / (ms / 1e3)
+    model = stage_model(w, T, touched)
+    dom = max(stage_ms, key=lambda k: stage_ms[k])
+    fl, by = model[dom]
+    t_s = stage_ms[dom] / 1e3
+    if fl / (tf_burst * 1e12) >= by / (hbm * 1e9):
+        roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": tf_burst, "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stage_ms[dom]}
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst bf16 / copy bandwidth)"
+    Lf, Lb = layer_flops(w, T), layer_bytes(w, T, touched)
+    t_roof = max(Lf / (tf_burst * 1e12), Lb / (hbm * 1e9))
+    layer_roof = {"flops": Lf, "bytes": Lb, "roofline_ms": t_roof * 1e3, "frac": t_roof / (ms / 1e3),
+                  "bound": "tensor" if Lf / (tf_burst * 1e12) >= Lb / (hbm * 1e9) else "hbm",
+                  "achieved_tflops": Lf / (ms / 1e3) / 1e12, "achieved_gbs": Lb / (ms / 1e3) / 1e9,
+                  "frac_of_sustained_tensor": (Lf / (tf_sus * 1e12)) / (ms / 1e3) if tf_sus else None}
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v, n, dt, cores = time_oracle(w, x_cpu, W, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n} seeded token rows of the {T}-token batch in {dt:.1f} s (fp64 C oracle)"}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+            "data": "synthetic (seeded N(0,1) tokens, N(0,1/fan_in) weights)",
+            "config": {"workload": w.name, "T": T, "d": w.d, "l": w.l, "f": w.f, "E": w.E, "k": w.k,
+                       "f_shared": w.f_s, "touched_experts": touched,
+                       "gemm": "tcgen05" if (args.gemm == 0 and w.dtype == "bf16") else "cuda-cores",
+                       "l2": "flushed between timed steps (256 MiB write, untimed)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": roof, "layer_roofline": layer_roof,
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * T / (e2e_ms / args.steps / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": layer.launch_count(T) * args.steps, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    layer.close()
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import datetime
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_own(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * lmoe.h -- C ABI of the B200 (sm_100a) LatentMoE layer forward library.
+ *
+ * The library computes, for every token row x of width d (rows independent):
+ *
+ *   r   = sigmoid(W_r x)                       router scores at model width
+ *   T_k = TopK(r + b, k)                       the bias changes selection only
+ *   p_i = r_i / sum_{j in T_k} r_j             mixture weights from raw scores
+ *   z   = W_down x                             latent width l = d / alpha
+ *   u   = sum_{i in T_k} p_i D_i act(G_i z, U_i z)   routed experts l -> f -> l
+ *   y   = S_1(x) + S_2(x) + W_up RMSNorm(u)    two shared experts at width d
+ *
+ * as defined by the "Stable LatentMoE" problem (TensorTonic, Kimi K3 set:
+ * equations for r, T_k(x), p_i, u and y; Requirements and Constraints), with
+ * the routed/shared split of the cooking-agi page "LatentMoE: must experts be
+ * as wide as the backbone?" (section "Which part becomes narrower?") and the
+ * variant arithmetic of the PyPI latent_moe README (section "Latent-MoE").
+ * act is SwiGLU, silu(g) * v, or the capped SiTU-GLU gate
+ * cg tanh(g/cg) sigmoid(g) * cu tanh(v/cu).
+ *
+ * Conventions for every entry point:
+ *  - Every call returns an lmoe_status; nothing throws, nothing aborts.
+ *    On failure lmoe_last_error() returns a message for the calling thread.
+ *  - "device" pointers are CUDA global-memory addresses on the device that is
+ *    current when lmoe_create was called; "host" pointers are CPU memory.
+ *  - Matrices are dense row-major, "out x in" (W @ x): the layouts below.
+ *  - Streams are passed as void* holding a cudaStream_t (NULL = legacy
+ *    default stream).  Calls that take a stream only enqueue work on it and
+ *    return without synchronising, unless stated otherwise.
+ *  - Floating tensors use the configuration's dtype (fp32 or bf16, "the token
+ *    dtype"), except W_r and b, which are always fp32.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LMOE_API __attribute__((visibility("default")))
+#else
+#define LMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LMOE_OK = 0,
+    LMOE_ERR_INVALID_ARG = 1,     /* a pointer, size or configuration value is invalid */
+    LMOE_ERR_UNSUPPORTED = 2,     /* valid, but outside what the kernels handle (alignment) */
+    LMOE_ERR_OOM = 3,             /* cudaMalloc for handle-owned memory failed */
+    LMOE_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+    LMOE_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait gave up (see lmoe_check_device) */
+    LMOE_ERR_WORKSPACE = 6        /* the workspace passed in is too small */
+} lmoe_status;
+
+typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;
+typedef enum { LMOE_ACT_SWIGLU = 0, LMOE_ACT_SITU = 1 } lmoe_act;
+
+/* Layer configuration.
+ *  d         model width                  l      latent width (l <= d)
+ *  f         routed expert intermediate   E      routed experts
+ *  k         selected experts, 1 <= k <= E ("Selected count is positive and
+ *            no larger than the routed expert count", Stable LatentMoE,
+ *            Constraints)
+ *  f_shared  shared expert intermediate   n_shared  must be 2 ("Exactly two
+ *            shared experts are supplied", Stable LatentMoE, Constraints)
+ *  eps       RMSNorm epsilon, inside the square root; the norm has unit gain
+ *  dtype     lmoe_dtype of tokens, outputs and all weights except W_r and b
+ *  act       lmoe_act; gate_cap / up_cap are the SiTU caps (ignored for SwiGLU)
+ *  gemm      0 = tensor cores (tcgen05) for bf16, CUDA cores for fp32;
+ *            1 = CUDA cores for every GEMM (a slower cross-check path)
+ */
+typedef struct {
+    int32_t d, l, f, E, k, f_shared, n_shared;
+    float eps;
+    int32_t dtype;
+    int32_t act;
+    float gate_cap, up_cap;
+    int32_t gemm;
+} lmoe_config;
+
+/* Weights, all device pointers, read only during lmoe_create:
+ *  W_r    [E, d]  fp32       router projection
+ *  b      [E]     fp32       selection bias
+ *  W_down [l, d]             shared down-projection
+ *  W_up   [d, l]             up-projection
+ *  G, U   [E, f, l]          routed gate / up projections
+ *  D      [E, l, f]          routed down projections
+ *  Gs, Us [2, f_shared, d]   shared gate / up projections
+ *  Ds     [2, d, f_shared]   shared down projections
+ */
+typedef struct {
+    const float *W_r;
+    const float *b;
+    const void *W_down, *W_up;
+    const void *G, *U, *D;
+    const void *Gs, *Us, *Ds;
+} lmoe_weights;
+
+typedef struct lmoe_handle lmoe_handle;
+
+/* Fill *out from the base-MoE description of the PyPI latent_moe README
+ * (LatentMoEConfig: d, m, n_experts N, top_k K, alpha, n_shared, variant) and
+ * its variant list: l = d / alpha, E = alpha * N routed experts; "eff" keeps
+ * k = K, "acc" takes k = alpha * K; f = f_shared = m.  eps = 1e-6, bf16,
+ * SwiGLU, tensor cores.  INVALID_ARG if a value is not positive, alpha does
+ * not divide d, the variant is neither "acc" nor "eff", or k > E. */
+LMOE_API lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int32_t K, int32_t alpha,
+                                  int32_t n_shared, const char *variant, lmoe_config *out);
+
+/* Validate cfg, allocate handle-owned device memory on the current device and
+ * repack the weights into it (gate/up rows interleaved per tile, the shared
+ * down projections and W_up concatenated, the router split for the tensor
+ * cores).  Work is enqueued on `stream`, which is synchronised before return,
+ * so the caller may free its weight copies afterwards.
+ * INVALID_ARG: null pointer, non-positive size, l > d, k < 1 or k > E,
+ *              n_shared != 2, eps < 0, unknown dtype/act.
+ * UNSUPPORTED: d, l, f or f_shared not a multiple of 64, E > 1024, or (bf16
+ *              tensor-core path) f or f_shared not a multiple of 128.
+ * OOM / CUDA on allocation or launch failure (nothing is leaked). */
+LMOE_API lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *stream, lmoe_handle **out);
+
+/* Device workspace bytes that lmoe_forward needs for T tokens (0 for T = 0). */
+LMOE_API lmoe_status lmoe_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes);
+
+/* The layer forward ("Stable LatentMoE", equations for r, T_k, p_i, u, y, and
+ * its return contract) for T tokens, enqueued on `stream`:
+ *  x                        [T, d] device, token dtype (input)
+ *  output                   [T, d] device, token dtype
+ *  selected_experts         [T, k] device int32, per row in selection order
+ *                           (biased score descending, equal scores to the
+ *                           lower expert index)
+ *  mixture_weights          [T, k] device, token dtype, aligned with
+ *                           selected_experts; each row sums to one
+ *  latent_routed_aggregate  [T, l] device, token dtype: u before RMSNorm
+ *  workspace                device scratch of >= lmoe_workspace_size(T) bytes,
+ *                           256-byte aligned; its contents on entry are
+ *                           irrelevant and it is clobbered
+ * Outputs must not overlap x, each other or the workspace.  T = 0 is a no-op.
+ * Inputs must be finite.  Overlapping calls on one handle are allowed; calls
+ * that share a workspace must be ordered on one stream.
+ * INVALID_ARG for null pointers (T > 0) or T < 0; WORKSPACE if ws_bytes is too
+ * small or misaligned; CUDA if a launch fails. */
+LMOE_API lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
+                         void *mixture_weights, void *latent_routed_aggregate, void *workspace,
+                         size_t ws_bytes, void *stream);
+
+/* Device workspace bytes for lmoe_forward_host with T tokens: staging for x
+ * and the four outputs plus the lmoe_forward workspace. */
+LMOE_API lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes);
+
+/* lmoe_forward on HOST buffers (same shapes and dtypes as lmoe_forward; use
+ * pinned memory for asynchronous copies): copies x to the device, runs the
+ * forward, and copies the four outputs back, all enqueued on `stream`.  The
+ * host outputs are valid once the stream has been synchronised.
+ * Errors as lmoe_forward. */
+LMOE_API lmoe_status lmoe_forward_host(lmoe_handle *h, const void *x_host, int64_t T, void *output_host,
+                              int32_t *selected_experts_host, void *mixture_weights_host,
+                              void *latent_routed_aggregate_host, void *workspace, size_t ws_bytes,
+                              void *stream);
+
+/* Replace the selection bias with b [E] (device fp32), enqueued on `stream`.
+ * The bias changes only which experts are selected ("Stable LatentMoE": "The
+ * bias changes selection only"; the cooking-agi page, section "Quantile
+ * Balancing", updates it between steps and freezes it for inference). */
+LMOE_API lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream);
+
+/* Stages of one forward, in launch order (for lmoe_set_stage_events):
+ *  0 router GEMM, 1 top-k, 2 counting-sort scan, 3 dispatch, 4 down-projection
+ *  GEMM, 5 routed gate/up GEMM, 6 routed down GEMM + weighting, 7 combine +
+ *  RMSNorm, 8 shared gate/up GEMM, 9 final GEMM (shared down + up-projection). */
+#define LMOE_NUM_STAGES 10
+
+/* Ask subsequent lmoe_forward calls on this handle to record events[i] (each
+ * a cudaEvent_t created by the caller) on the forward's stream right before
+ * stage i, and events[LMOE_NUM_STAGES] after the last stage, so that the
+ * caller can time every kernel with cudaEventElapsedTime.  n must be
+ * LMOE_NUM_STAGES + 1, or 0 with events NULL to stop recording.  The array is
+ * read at each forward, not copied: the caller keeps it alive. */
+LMOE_API lmoe_status lmoe_set_stage_events(lmoe_handle *h, void *const *events, int32_t n);
+
+/* Number of kernel launches one lmoe_forward of T tokens makes. */
+LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches);
+
+/* Byte offset and size of one intermediate inside the forward workspace, so
+ * tests can read stage results after a forward on the same stream.
+ * region: 0 router scores r [T, E] fp32; 1 mixture weights fp32 [T, k];
+ * 2 per-expert counts [E] int32; 3 expert offsets [E+1] int32;
+ * 4 slot index of (t, j) [T, k] int32; 5 token of each permuted slot [T*k]
+ * int32; 6 permuted latent rows Z [T*k, l]; 7 routed hidden H [T*k, f];
+ * 8 p-weighted expert outputs [T*k, l] fp32; 9 [shared hidden | RMSNorm(u)]
+ * [T, 2 f_shared + l]; 10 device status word (int32).
+ * INVALID_ARG for an unknown region. */
+LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t region, size_t *offset,
+                                  size_t *bytes);
+
+/* Synchronise `stream`, then read and clear the device status word that the
+ * kernels of the last forward on this workspace wrote: LMOE_OK, or
+ * LMOE_ERR_DEVICE_TIMEOUT if a bounded wait gave up (its outputs are then
+ * invalid).  `workspace` is the one passed to lmoe_forward. */
+LMOE_API lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream);
+
+/* Message for the last failure on the calling thread ("" if none). */
+LMOE_API const char *lmoe_last_error(void);
+
+/* Free the handle and its device memory (after pending work on it is done).
+ * NULL is ignored. */
+LMOE_API void lmoe_destroy(lmoe_handle *h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMOE_H */

@@ -1,0 +1,486 @@
+// Host runtime behind the C ABI of include/lmoe.h: configuration checks,
+// handle-owned repacked weights, the workspace plan, and the launch sequence
+// of one layer forward on one stream.
+//
+// Forward sequence for T tokens (S = T k slot rows):
+//   1 router GEMM      r = sigmoid(x W_r^T)                     [T, E] fp32
+//   2 top-k            sel, p (fp32 and token dtype), per-block expert counts
+//   3 scan             counts, offsets, per-block bases, m-tile prefix
+//   4 dispatch         slot_of[t, j], token and weight of every slot row
+//   5 down GEMM        z = x W_down^T, each row written to its k slot rows
+//   6 gate/up GEMM     per expert: h = act(G z, U z)            [S, f]
+//   7 down GEMM        per expert: Y = p * (h D^T)              [S, l] fp32
+//   8 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
+//   9 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
+//  10 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "lmoe_internal.cuh"
+#include "gemm_tc.cuh"
+
+using namespace lmoe;
+
+namespace {
+
+thread_local std::string g_err;
+
+lmoe_status fail(lmoe_status s, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return s;
+}
+
+#define LMOE_CUDA(call)                                                                         \
+    do {                                                                                        \
+        cudaError_t e_ = (call);                                                                \
+        if (e_ != cudaSuccess)                                                                  \
+            return fail(LMOE_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),  \
+                        __FILE__, __LINE__);                                                    \
+    } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+    size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, Zp, H, Yp, HS, status;
+    size_t total;
+};
+
+}  // namespace
+
+struct lmoe_handle {
+    lmoe_config cfg;
+    int device;
+    bool tc;          // tensor-core GEMMs
+    int ib;           // gate/up interleave block
+    int bm;           // m-tile of the grouped GEMMs
+    size_t tb;        // token dtype bytes
+    float *Wr;        // [E, d] fp32 (CUDA-core router)
+    bf16 *Wr3;        // [3, E, d] bf16 split (tensor-core router)
+    float *b;         // [E]
+    void *Wdown;      // [l, d]
+    void *Wgu;        // [E, 2f, l] interleaved
+    void *D;          // [E, l, f]
+    void *Wgu_s;      // [4 f_s, d] interleaved (both shared experts as one of width 2 f_s)
+    void *Wcat;       // [d, 2 f_s + l]
+    void *const *stage_events;  // caller's cudaEvent_t[LMOE_NUM_STAGES + 1] or NULL
+};
+
+namespace {
+
+Layout plan(const lmoe_handle *h, int64_t T)
+{
+    const lmoe_config &c = h->cfg;
+    const int64_t S = T * c.k;
+    const int64_t nb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
+    Layout L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+    L.r32 = take(sizeof(float) * T * c.E);
+    L.p32 = take(sizeof(float) * S);
+    L.blockhist = take(sizeof(int32_t) * nb * c.E);
+    L.base = take(sizeof(int32_t) * nb * c.E);
+    L.counts = take(sizeof(int32_t) * c.E);
+    L.offsets = take(sizeof(int32_t) * (c.E + 1));
+    L.tile_off = take(sizeof(int32_t) * (c.E + 1));
+    L.slot_of = take(sizeof(int32_t) * S);
+    L.perm_tok = take(sizeof(int32_t) * S);
+    L.perm_w = take(sizeof(float) * S);
+    L.Zp = take(h->tb * S * c.l);
+    L.H = take(h->tb * S * c.f);
+    L.Yp = take(sizeof(float) * S * c.l);
+    L.HS = take(h->tb * T * (2 * (int64_t)c.f_shared + c.l));
+    L.status = take(256);
+    L.total = o;
+    return L;
+}
+
+lmoe_status check_config(const lmoe_config *c, bool *tc)
+{
+    if (!c) return fail(LMOE_ERR_INVALID_ARG, "config is NULL");
+    if (c->d < 1 || c->l < 1 || c->f < 1 || c->E < 1 || c->f_shared < 1)
+        return fail(LMOE_ERR_INVALID_ARG, "dimensions must be positive");
+    if (c->l > c->d) return fail(LMOE_ERR_INVALID_ARG, "latent width l=%d exceeds d=%d", c->l, c->d);
+    if (c->k < 1 || c->k > c->E) return fail(LMOE_ERR_INVALID_ARG, "k=%d must satisfy 1 <= k <= E=%d", c->k, c->E);
+    if (c->n_shared != 2) return fail(LMOE_ERR_INVALID_ARG, "exactly two shared experts are required");
+    if (!(c->eps >= 0.f)) return fail(LMOE_ERR_INVALID_ARG, "eps must be >= 0");
+    if (c->dtype != LMOE_F32 && c->dtype != LMOE_BF16) return fail(LMOE_ERR_INVALID_ARG, "unknown dtype");
+    if (c->act != LMOE_ACT_SWIGLU && c->act != LMOE_ACT_SITU) return fail(LMOE_ERR_INVALID_ARG, "unknown act");
+    if (c->act == LMOE_ACT_SITU && !(c->gate_cap > 0.f && c->up_cap > 0.f))
+        return fail(LMOE_ERR_INVALID_ARG, "SiTU caps must be positive");
+    if (c->gemm != 0 && c->gemm != 1) return fail(LMOE_ERR_INVALID_ARG, "gemm must be 0 or 1");
+    if (c->E > 1024) return fail(LMOE_ERR_UNSUPPORTED, "E=%d > 1024", c->E);
+    if (c->k > 64) return fail(LMOE_ERR_UNSUPPORTED, "k=%d > 64", c->k);
+    if (c->d % 64 || c->l % 64 || c->f % 64 || c->f_shared % 64)
+        return fail(LMOE_ERR_UNSUPPORTED, "d, l, f and f_shared must be multiples of 64");
+    *tc = (c->dtype == LMOE_BF16 && c->gemm == 0);
+    if (*tc && (c->f % (TC_BN / 2) || c->f_shared % (TC_BN / 2)))
+        return fail(LMOE_ERR_UNSUPPORTED, "tensor-core path needs f and f_shared multiples of %d", TC_BN / 2);
+    return LMOE_OK;
+}
+
+void free_handle(lmoe_handle *h)
+{
+    if (!h) return;
+    void *ptrs[] = {h->Wr, h->Wr3, h->b, h->Wdown, h->Wgu, h->D, h->Wgu_s, h->Wcat};
+    for (void *p : ptrs)
+        if (p) cudaFree(p);
+    delete h;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lmoe_last_error(void) { return g_err.c_str(); }
+
+lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int32_t K, int32_t alpha, int32_t n_shared,
+                                  const char *variant, lmoe_config *out)
+{
+    g_err.clear();
+    if (!out || !variant) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (d < 1 || m < 1 || N < 1 || K < 1 || alpha < 1 || n_shared < 1)
+        return fail(LMOE_ERR_INVALID_ARG, "all base values must be positive");
+    if (d % alpha) return fail(LMOE_ERR_INVALID_ARG, "alpha=%d does not divide d=%d", alpha, d);
+    int k;
+    if (!strcmp(variant, "eff")) k = K;
+    else if (!strcmp(variant, "acc")) k = alpha * K;
+    else return fail(LMOE_ERR_INVALID_ARG, "variant must be \"acc\" or \"eff\"");
+    const int E = alpha * N;
+    if (k > E) return fail(LMOE_ERR_INVALID_ARG, "top-k %d exceeds %d experts", k, E);
+    lmoe_config c;
+    memset(&c, 0, sizeof c);
+    c.d = d; c.l = d / alpha; c.f = m; c.E = E; c.k = k; c.f_shared = m; c.n_shared = n_shared;
+    c.eps = 1e-6f; c.dtype = LMOE_BF16; c.act = LMOE_ACT_SWIGLU; c.gate_cap = 4.f; c.up_cap = 25.f; c.gemm = 0;
+    *out = c;
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *stream, lmoe_handle **out)
+{
+    g_err.clear();
+    if (!out) return fail(LMOE_ERR_INVALID_ARG, "out is NULL");
+    *out = nullptr;
+    bool tc = false;
+    lmoe_status st = check_config(cfg, &tc);
+    if (st != LMOE_OK) return st;
+    if (!w || !w->W_r || !w->b || !w->W_down || !w->W_up || !w->G || !w->U || !w->D || !w->Gs || !w->Us || !w->Ds)
+        return fail(LMOE_ERR_INVALID_ARG, "a weight pointer is NULL");
+    if (tc) {
+        st = tc_check_device();
+        if (st != LMOE_OK) return st;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    lmoe_handle *h = new lmoe_handle();
+    memset(h, 0, sizeof *h);
+    h->cfg = *cfg;
+    cudaGetDevice(&h->device);
+    h->tc = tc;
+    h->ib = tc ? TC_BN / 2 : SIMT_BN / 2;
+    h->bm = tc ? TC_BM : SIMT_BM;
+    h->tb = cfg->dtype == LMOE_BF16 ? 2 : 4;
+    const lmoe_config &c = *cfg;
+    const size_t tb = h->tb;
+    const int64_t fs = c.f_shared;
+
+#define ALLOC(ptr, bytes)                                                                        \
+    do {                                                                                         \
+        if (cudaMalloc((void **)&(ptr), (bytes)) != cudaSuccess) {                              \
+            cudaGetLastError();                                                                  \
+            free_handle(h);                                                                      \
+            return fail(LMOE_ERR_OOM, "cudaMalloc of %zu bytes failed", (size_t)(bytes));        \
+        }                                                                                        \
+    } while (0)
+#define STEP(call)                                                                               \
+    do {                                                                                         \
+        cudaError_t e_ = (call);                                                                 \
+        if (e_ != cudaSuccess) {                                                                 \
+            free_handle(h);                                                                      \
+            return fail(LMOE_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));                 \
+        }                                                                                        \
+    } while (0)
+
+    ALLOC(h->Wr, sizeof(float) * c.E * c.d);
+    ALLOC(h->b, sizeof(float) * c.E);
+    ALLOC(h->Wdown, tb * c.l * c.d);
+    ALLOC(h->Wgu, tb * (size_t)c.E * 2 * c.f * c.l);
+    ALLOC(h->D, tb * (size_t)c.E * c.l * c.f);
+    ALLOC(h->Wgu_s, tb * 4 * fs * c.d);
+    ALLOC(h->Wcat, tb * c.d * (2 * fs + c.l));
+    STEP(cudaMemcpyAsync(h->Wr, w->W_r, sizeof(float) * c.E * c.d, cudaMemcpyDeviceToDevice, s));
+    STEP(cudaMemcpyAsync(h->b, w->b, sizeof(float) * c.E, cudaMemcpyDeviceToDevice, s));
+    STEP(cudaMemcpyAsync(h->Wdown, w->W_down, tb * c.l * c.d, cudaMemcpyDeviceToDevice, s));
+    STEP(cudaMemcpyAsync(h->D, w->D, tb * (size_t)c.E * c.l * c.f, cudaMemcpyDeviceToDevice, s));
+    STEP(launch_pack_glu(w->G, w->U, h->Wgu, c.E, c.f, c.l, h->ib, (int)tb, s));
+    // [2, f_s, d] stacks are the rows of one expert of width 2 f_s
+    STEP(launch_pack_glu(w->Gs, w->Us, h->Wgu_s, 1, 2 * c.f_shared, c.d, h->ib, (int)tb, s));
+    STEP(launch_pack_cat(w->Ds, w->W_up, h->Wcat, c.d, c.f_shared, c.l, (int)tb, s));
+    if (tc) {
+        ALLOC(h->Wr3, sizeof(bf16) * 3 * c.E * c.d);
+        STEP(launch_split_router(h->Wr, h->Wr3, (int64_t)c.E * c.d, s));
+    }
+    STEP(cudaStreamSynchronize(s));
+#undef ALLOC
+#undef STEP
+    *out = h;
+    return LMOE_OK;
+}
+
+void lmoe_destroy(lmoe_handle *h) { free_handle(h); }
+
+lmoe_status lmoe_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes)
+{
+    g_err.clear();
+    if (!h || !bytes) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
+    *bytes = T == 0 ? 0 : plan(h, T).total;
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t region, size_t *offset, size_t *bytes)
+{
+    g_err.clear();
+    if (!h || !offset || !bytes) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 1) return fail(LMOE_ERR_INVALID_ARG, "T < 1");
+    const Layout L = plan(h, T);
+    const lmoe_config &c = h->cfg;
+    const int64_t S = T * c.k;
+    switch (region) {
+    case 0: *offset = L.r32; *bytes = sizeof(float) * T * c.E; break;
+    case 1: *offset = L.p32; *bytes = sizeof(float) * S; break;
+    case 2: *offset = L.counts; *bytes = sizeof(int32_t) * c.E; break;
+    case 3: *offset = L.offsets; *bytes = sizeof(int32_t) * (c.E + 1); break;
+    case 4: *offset = L.slot_of; *bytes = sizeof(int32_t) * S; break;
+    case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
+    case 6: *offset = L.Zp; *bytes = h->tb * S * c.l; break;
+    case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
+    case 8: *offset = L.Yp; *bytes = sizeof(float) * S * c.l; break;
+    case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
+    case 10: *offset = L.status; *bytes = sizeof(int32_t); break;
+    default: return fail(LMOE_ERR_INVALID_ARG, "unknown region %d", region);
+    }
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_set_stage_events(lmoe_handle *h, void *const *events, int32_t n)
+{
+    g_err.clear();
+    if (!h) return fail(LMOE_ERR_INVALID_ARG, "handle is NULL");
+    if (n == 0 && !events) { h->stage_events = nullptr; return LMOE_OK; }
+    if (n != LMOE_NUM_STAGES + 1 || !events)
+        return fail(LMOE_ERR_INVALID_ARG, "need %d events", LMOE_NUM_STAGES + 1);
+    h->stage_events = events;
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches)
+{
+    g_err.clear();
+    if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    // status reset, router, top-k, scan, dispatch, down, gate/up, down+combine, norm, shared, final
+    *launches = T == 0 ? 0 : 11;
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream)
+{
+    g_err.clear();
+    if (!h || !b) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    LMOE_CUDA(cudaMemcpyAsync(h->b, b, sizeof(float) * h->cfg.E, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
+                         void *mixture_weights, void *latent_routed_aggregate, void *workspace, size_t ws_bytes,
+                         void *stream)
+{
+    g_err.clear();
+    if (!h) return fail(LMOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) return LMOE_OK;
+    if (!x || !output || !selected_experts || !mixture_weights || !latent_routed_aggregate || !workspace)
+        return fail(LMOE_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (T * h->cfg.k > 0x7fffffffLL) return fail(LMOE_ERR_UNSUPPORTED, "T * k exceeds 2^31 - 1");
+    const Layout L = plan(h, T);
+    if (ws_bytes < L.total) return fail(LMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+    if ((uintptr_t)workspace % 256) return fail(LMOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
+
+    if (h->tc && (((uintptr_t)x | (uintptr_t)output) & 15u))
+        return fail(LMOE_ERR_UNSUPPORTED, "x and output must be 16-byte aligned for the tensor-core path");
+    const lmoe_config &c = h->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    float *r32 = (float *)(ws + L.r32);
+    float *p32 = (float *)(ws + L.p32);
+    int32_t *blockhist = (int32_t *)(ws + L.blockhist);
+    int32_t *base = (int32_t *)(ws + L.base);
+    int32_t *counts = (int32_t *)(ws + L.counts);
+    int32_t *offsets = (int32_t *)(ws + L.offsets);
+    int32_t *tile_off = (int32_t *)(ws + L.tile_off);
+    int32_t *slot_of = (int32_t *)(ws + L.slot_of);
+    int32_t *perm_tok = (int32_t *)(ws + L.perm_tok);
+    float *perm_w = (float *)(ws + L.perm_w);
+    void *Zp = ws + L.Zp, *H = ws + L.H, *HS = ws + L.HS;
+    float *Yp = (float *)(ws + L.Yp);
+    int32_t *status = (int32_t *)(ws + L.status);
+
+    const int64_t S = T * c.k;
+    const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
+    const int tk = c.dtype == LMOE_BF16 ? 1 : 0;
+    const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
+    const int max_mtiles = (int)((S + h->bm - 1) / h->bm + c.E);
+
+    LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+#define STAGE(i)                                                                                 \
+    if (h->stage_events) LMOE_CUDA(cudaEventRecord((cudaEvent_t)h->stage_events[i], s))
+
+    // 1 router: r = sigmoid(x W_r^T)
+    STAGE(0);
+    {
+        GemmArgs g = {};
+        g.A = x; g.lda = c.d; g.M = (int)T; g.N = c.E; g.K = c.d;
+        g.epi.out = r32; g.epi.ldo = c.E;
+        if (h->tc) {
+            LMOE_CUDA(tc_gemm_router(h->Wr3, g, status, s));
+        } else {
+            g.B = h->Wr; g.ldb = c.d;
+            LMOE_CUDA(launch_simt_gemm(EPI_SIGMOID, tk, 0, 0, g, 0, s));
+        }
+    }
+    // 2-4 selection and dispatch
+    STAGE(1);
+    LMOE_CUDA(launch_topk(r32, h->b, T, c.E, c.k, selected_experts, p32, mixture_weights, tk, blockhist, s));
+    STAGE(2);
+    LMOE_CUDA(launch_scan(blockhist, nb, c.E, h->bm, counts, offsets, base, tile_off, s));
+    STAGE(3);
+    LMOE_CUDA(launch_dispatch(selected_experts, p32, base, T, c.E, c.k, slot_of, perm_tok, perm_w, s));
+
+    // 5 z = x W_down^T scattered to the k slot rows of each token
+    GemmArgs gd = {};
+    gd.A = x; gd.lda = c.d; gd.B = h->Wdown; gd.ldb = c.d; gd.M = (int)T; gd.N = c.l; gd.K = c.d;
+    gd.epi.out = Zp; gd.epi.ldo = c.l; gd.epi.slot_of = slot_of; gd.epi.k = c.k;
+    // 6 per expert h = act(G z, U z)
+    GemmArgs gu = {};
+    gu.A = Zp; gu.lda = c.l; gu.B = h->Wgu; gu.ldb = c.l; gu.b_group_stride = 2 * (int64_t)c.f * c.l;
+    gu.M = (int)S; gu.N = 2 * c.f; gu.K = c.l; gu.offsets = offsets; gu.tile_off = tile_off; gu.E = c.E;
+    gu.epi.out = H; gu.epi.ldo = c.f; gu.epi.act = c.act; gu.epi.gate_cap = c.gate_cap; gu.epi.up_cap = c.up_cap;
+    gu.epi.ib = h->ib;
+    // 7 per expert Y = p (h D^T)
+    GemmArgs gc = {};
+    gc.A = H; gc.lda = c.f; gc.B = h->D; gc.ldb = c.f; gc.b_group_stride = (int64_t)c.l * c.f;
+    gc.M = (int)S; gc.N = c.l; gc.K = c.f; gc.offsets = offsets; gc.tile_off = tile_off; gc.E = c.E;
+    gc.epi.out = Yp; gc.epi.ldo = c.l; gc.epi.row_w = perm_w;
+    // 9 shared experts' hidden, both as one expert of width 2 f_s
+    GemmArgs gs = {};
+    gs.A = x; gs.lda = c.d; gs.B = h->Wgu_s; gs.ldb = c.d; gs.M = (int)T; gs.N = 4 * c.f_shared; gs.K = c.d;
+    gs.epi.out = HS; gs.epi.ldo = ld_hs; gs.epi.act = c.act; gs.epi.gate_cap = c.gate_cap;
+    gs.epi.up_cap = c.up_cap; gs.epi.ib = h->ib;
+    // 10 y = [h_s | n] [D_s1 | D_s2 | W_up]^T
+    GemmArgs gf = {};
+    gf.A = HS; gf.lda = ld_hs; gf.B = h->Wcat; gf.ldb = ld_hs; gf.M = (int)T; gf.N = c.d; gf.K = (int)ld_hs;
+    gf.epi.out = output; gf.epi.ldo = c.d;
+
+    STAGE(4);
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_SCATTER, gd, 0, status, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_SCATTER, tk, tk, tk, gd, 0, s));
+    STAGE(5);
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, status, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, s));
+    STAGE(6);
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, status, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, 0, gc, max_mtiles, s));
+    // 8 u, RMSNorm(u) into the columns after the shared hidden
+    STAGE(7);
+    LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
+                                  2 * (int64_t)c.f_shared, tk, s));
+    STAGE(8);
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gs, 0, status, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, s));
+    STAGE(9);
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gf, 0, status, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, s));
+    STAGE(LMOE_NUM_STAGES);
+#undef STAGE
+    (void)perm_tok;
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes)
+{
+    g_err.clear();
+    if (!h || !bytes) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) { *bytes = 0; return LMOE_OK; }
+    const lmoe_config &c = h->cfg;
+    size_t o = 0;
+    o = align_up(o + h->tb * T * c.d, 256);          // x
+    o = align_up(o + h->tb * T * c.d, 256);          // output
+    o = align_up(o + sizeof(int32_t) * T * c.k, 256);
+    o = align_up(o + h->tb * T * c.k, 256);
+    o = align_up(o + h->tb * T * c.l, 256);
+    *bytes = o + plan(h, T).total;
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_forward_host(lmoe_handle *h, const void *x_host, int64_t T, void *output_host,
+                              int32_t *selected_experts_host, void *mixture_weights_host,
+                              void *latent_routed_aggregate_host, void *workspace, size_t ws_bytes, void *stream)
+{
+    g_err.clear();
+    if (!h) return fail(LMOE_ERR_INVALID_ARG, "handle is NULL");
+    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) return LMOE_OK;
+    if (!x_host || !output_host || !selected_experts_host || !mixture_weights_host || !latent_routed_aggregate_host ||
+        !workspace)
+        return fail(LMOE_ERR_INVALID_ARG, "NULL pointer");
+    size_t need = 0;
+    lmoe_host_workspace_size(h, T, &need);
+    if (ws_bytes < need) return fail(LMOE_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+    if ((uintptr_t)workspace % 256) return fail(LMOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    const lmoe_config &c = h->cfg;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    size_t o = 0;
+    const size_t bx = h->tb * T * c.d, bs = sizeof(int32_t) * T * c.k, bp = h->tb * T * c.k, bu = h->tb * T * c.l;
+    char *dx = ws + o; o = align_up(o + bx, 256);
+    char *dy = ws + o; o = align_up(o + bx, 256);
+    char *dsel = ws + o; o = align_up(o + bs, 256);
+    char *dp = ws + o; o = align_up(o + bp, 256);
+    char *du = ws + o; o = align_up(o + bu, 256);
+    LMOE_CUDA(cudaMemcpyAsync(dx, x_host, bx, cudaMemcpyHostToDevice, s));
+    lmoe_status st = lmoe_forward(h, dx, T, dy, (int32_t *)dsel, dp, du, ws + o, ws_bytes - o, stream);
+    if (st != LMOE_OK) return st;
+    LMOE_CUDA(cudaMemcpyAsync(output_host, dy, bx, cudaMemcpyDeviceToHost, s));
+    LMOE_CUDA(cudaMemcpyAsync(selected_experts_host, dsel, bs, cudaMemcpyDeviceToHost, s));
+    LMOE_CUDA(cudaMemcpyAsync(mixture_weights_host, dp, bp, cudaMemcpyDeviceToHost, s));
+    LMOE_CUDA(cudaMemcpyAsync(latent_routed_aggregate_host, du, bu, cudaMemcpyDeviceToHost, s));
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream)
+{
+    g_err.clear();
+    if (!h || !workspace) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 1) return LMOE_OK;
+    const Layout L = plan(h, T);
+    int32_t v = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    LMOE_CUDA(cudaMemcpyAsync(&v, (char *)workspace + L.status, sizeof v, cudaMemcpyDeviceToHost, s));
+    LMOE_CUDA(cudaStreamSynchronize(s));
+    if (v != 0) {
+        LMOE_CUDA(cudaMemsetAsync((char *)workspace + L.status, 0, sizeof(int32_t), s));
+        LMOE_CUDA(cudaStreamSynchronize(s));
+        return fail(LMOE_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait gave up (status word 0x%x)", v);
+    }
+    return LMOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+// Internal declarations shared by the kernel files of liblmoe (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lmoe.h"
+
+namespace lmoe {
+
+typedef __nv_bfloat16 bf16;
+
+// ---------------------------------------------------------------- conversions
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + expf(-a)); }
+
+// Gate of every expert: SwiGLU silu(g) * v, or the capped SiTU-GLU
+// cg tanh(g/cg) sigmoid(g) * cu tanh(v/cu) ("Stable LatentMoE" names SiTU-GLU;
+// this capped form reproduces its worked example).
+__device__ __forceinline__ float glu_act(int act, float g, float v, float cg, float cu)
+{
+    const float sg = sigmoidf_(g);
+    if (act == LMOE_ACT_SITU) return cg * tanhf(g / cg) * sg * (cu * tanhf(v / cu));
+    return g * sg * v;
+}
+
+// ---------------------------------------------------------------- epilogues
+// Every GEMM here computes C[m, n] = sum_k A[m, k] B[n, k] (both K-major) and
+// hands each row chunk of fp32 accumulators to one of these epilogues.
+enum EpiMode {
+    EPI_STORE = 0,    // out[m, n] = C                      (final GEMM -> y)
+    EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
+    EPI_SCATTER = 2,  // out[slot_of[m, j], n] = C, j < k   (down-projection -> Z slots)
+    EPI_GLU = 3,      // out[m, n'] = act(C[gate], C[up])   (gate/up GEMMs -> h)
+    EPI_COMBINE = 4   // out32[m, n] = w[m] * C             (routed down -> p-weighted rows)
+};
+
+struct EpiArgs {
+    void *out;
+    int64_t ldo;             // row stride of out, elements
+    const int32_t *slot_of;  // EPI_SCATTER: [rows, k]
+    int k;
+    const float *row_w;      // EPI_COMBINE: weight of each row
+    int act;                 // EPI_GLU
+    float gate_cap, up_cap;
+    int ib;                  // EPI_GLU: gate/up interleave block (columns)
+};
+
+// Write n <= 32 consecutive values v[0..n) of row `row` starting at output column `col`.
+template <int MODE, typename TO>
+__device__ __forceinline__ void epi_store_chunk(const EpiArgs &e, int64_t row, int64_t col, const float *v, int n)
+{
+    if (MODE == EPI_SIGMOID) {
+        float *o = (float *)e.out + row * e.ldo + col;
+        #pragma unroll
+        for (int i = 0; i < 32; ++i) if (i < n) o[i] = sigmoidf_(v[i]);
+    } else if (MODE == EPI_COMBINE) {
+        float *o = (float *)e.out + row * e.ldo + col;
+        const float w = e.row_w[row];
+        #pragma unroll
+        for (int i = 0; i < 32; ++i) if (i < n) o[i] = w * v[i];
+    } else if (MODE == EPI_SCATTER) {
+        for (int j = 0; j < e.k; ++j) {
+            const int64_t dst = e.slot_of[row * e.k + j];
+            TO *o = (TO *)e.out + dst * e.ldo + col;
+            #pragma unroll
+            for (int i = 0; i < 32; ++i) if (i < n) o[i] = from_f32<TO>(v[i]);
+        }
+    } else {
+        TO *o = (TO *)e.out + row * e.ldo + col;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) if (i < n) o[i] = from_f32<TO>(v[i]);
+    }
+}
+
+// ---------------------------------------------------------------- GEMM description
+struct GemmArgs {
+    const void *A;
+    int64_t lda;        // elements
+    const void *B;
+    int64_t ldb;        // elements
+    int64_t b_group_stride;  // elements between consecutive experts' B
+    int M, N, K;        // dense: M rows; grouped: M = total rows (upper bound)
+    const int32_t *offsets;   // grouped: [E+1] row offsets, else nullptr
+    const int32_t *tile_off;  // grouped: [E+1] m-tile prefix for this kernel's BM
+    int E;
+    EpiArgs epi;
+};
+
+// ---------------------------------------------------------------- launchers
+// CUDA-core GEMM (fp32 FFMA): the fp32 path, and a cross-check path for bf16.
+// ta/tb/to: 0 = fp32, 1 = bf16.  Returns the launch error.
+cudaError_t launch_simt_gemm(int mode, int ta, int tb, int to, const GemmArgs &g, int max_mtiles, cudaStream_t s);
+constexpr int SIMT_BM = 64;
+constexpr int SIMT_BN = 128;
+
+// Router top-k + renormalisation + per-block expert histogram.
+constexpr int ROUTE_TPB = 128;  // tokens per block (also the dispatch block)
+cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
+                        void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s);
+cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int bm, int32_t *counts, int32_t *offsets,
+                        int32_t *base, int32_t *tile_off, cudaStream_t s);
+cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, int64_t T, int E, int k,
+                            int32_t *slot_of, int32_t *perm_tok, float *perm_w, cudaStream_t s);
+cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
+                                void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s);
+
+// Weight repacking (create time).
+cudaError_t launch_pack_glu(const void *G, const void *U, void *P, int nE, int F, int K, int ib, int elem_bytes,
+                            cudaStream_t s);
+cudaError_t launch_pack_cat(const void *Ds, const void *Wup, void *P, int d, int fs, int l, int elem_bytes,
+                            cudaStream_t s);
+cudaError_t launch_split_router(const float *Wr, bf16 *split, int64_t n, cudaStream_t s);
+
+// ---------------------------------------------------------------- tensor-core GEMM (sm_100a)
+struct TcGemm;  // defined in gemm_tc.cu
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 256;
+constexpr int TC_BK = 64;
+
+}  // namespace lmoe

@@ -1,0 +1,142 @@
+// Weighted combine + RMSNorm, and create-time weight repacking.
+//
+// combine_norm ("Stable LatentMoE", equations for u and y): for token t,
+//   u = sum_j Y[slot_of[t, j]]        (rows already scaled by p_j, summed in
+//                                      slot order j = 0..k-1: deterministic)
+//   n = u / sqrt(mean(u^2) + eps)     (RMSNorm, unit gain, eps inside the root)
+// u is written out as latent_routed_aggregate (token dtype); n goes to the
+// columns [col0, col0 + l) of the final GEMM's A operand, right after the
+// shared experts' hidden columns, so that W_up n and both shared down
+// projections are one K-concatenated GEMM.
+#include "lmoe_internal.cuh"
+
+namespace lmoe {
+namespace {
+
+constexpr int NT = 256;
+
+template <typename TT>
+__global__ void __launch_bounds__(NT)
+combine_norm_kernel(const float *__restrict__ Yp, const int32_t *__restrict__ slot_of, int l, int k, float eps,
+                    TT *__restrict__ u_out, TT *__restrict__ hs, int64_t ld_hs, int64_t col0)
+{
+    extern __shared__ float u[];   // [l]
+    __shared__ int slots[64];
+    __shared__ float red[NT / 32];
+    const int64_t t = blockIdx.x;
+    for (int j = threadIdx.x; j < k; j += NT) slots[j] = slot_of[t * k + j];
+    __syncthreads();
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < l; c += NT) {
+        float acc = 0.f;
+        for (int j = 0; j < k; ++j) acc += Yp[(int64_t)slots[j] * l + c];
+        u[c] = acc;
+        u_out[t * l + c] = from_f32<TT>(acc);
+        ss += acc * acc;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) tot += red[w];
+    const float inv = 1.0f / sqrtf(tot / (float)l + eps);
+    for (int c = threadIdx.x; c < l; c += NT) hs[t * ld_hs + col0 + c] = from_f32<TT>(u[c] * inv);
+}
+
+// P[e, 2F, K]: for every block q of ib rows, ib gate rows then the matching ib up rows.
+template <typename T>
+__global__ void pack_glu_kernel(const T *__restrict__ G, const T *__restrict__ U, T *__restrict__ P, int nE, int F,
+                                int K, int ib)
+{
+    const int64_t total = (int64_t)nE * 2 * F * K;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t kk = i % K;
+        const int64_t row = (i / K) % (2 * F);
+        const int64_t e = i / ((int64_t)K * 2 * F);
+        const int64_t q = row / (2 * ib), w = row % (2 * ib);
+        const int64_t src_row = q * ib + (w % ib);
+        const T *src = (w < ib) ? G : U;
+        P[i] = src[(e * F + src_row) * K + kk];
+    }
+}
+
+// P[d, 2 fs + l] = [Ds[0] | Ds[1] | W_up] row by row.
+template <typename T>
+__global__ void pack_cat_kernel(const T *__restrict__ Ds, const T *__restrict__ Wup, T *__restrict__ P, int d, int fs,
+                                int l)
+{
+    const int64_t W = 2 * (int64_t)fs + l;
+    const int64_t total = (int64_t)d * W;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / W, c = i % W;
+        T v;
+        if (c < fs) v = Ds[row * fs + c];
+        else if (c < 2 * fs) v = Ds[((int64_t)d + row) * fs + (c - fs)];
+        else v = Wup[row * l + (c - 2 * fs)];
+        P[i] = v;
+    }
+}
+
+// fp32 W -> three bf16 terms hi + mid + lo (each the rounding of what is left),
+// stored as [3][n]; with bf16 activations every product is exact in fp32, so the
+// three tensor-core passes reproduce an fp32 router to ~2^-24 relative.
+__global__ void split_router_kernel(const float *__restrict__ W, bf16 *__restrict__ out, int64_t n)
+{
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const float w = W[i];
+        const bf16 hi = __float2bfloat16_rn(w);
+        const float r1 = w - __bfloat162float(hi);
+        const bf16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);
+        out[i] = hi;
+        out[n + i] = mid;
+        out[2 * n + i] = __float2bfloat16_rn(r2);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
+                                void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s)
+{
+    if (T == 0) return cudaSuccess;
+    if (k > 64) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(float) * l;
+    if (tok_bf16)
+        combine_norm_kernel<bf16><<<(unsigned)T, NT, smem, s>>>(Yp, slot_of, l, k, eps, (bf16 *)u_out, (bf16 *)hs,
+                                                                  ld_hs, col0);
+    else
+        combine_norm_kernel<float><<<(unsigned)T, NT, smem, s>>>(Yp, slot_of, l, k, eps, (float *)u_out,
+                                                                   (float *)hs, ld_hs, col0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_glu(const void *G, const void *U, void *P, int nE, int F, int K, int ib, int elem_bytes,
+                            cudaStream_t s)
+{
+    if (elem_bytes == 2)
+        pack_glu_kernel<bf16><<<2048, 256, 0, s>>>((const bf16 *)G, (const bf16 *)U, (bf16 *)P, nE, F, K, ib);
+    else
+        pack_glu_kernel<float><<<2048, 256, 0, s>>>((const float *)G, (const float *)U, (float *)P, nE, F, K, ib);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_cat(const void *Ds, const void *Wup, void *P, int d, int fs, int l, int elem_bytes,
+                            cudaStream_t s)
+{
+    if (elem_bytes == 2)
+        pack_cat_kernel<bf16><<<1024, 256, 0, s>>>((const bf16 *)Ds, (const bf16 *)Wup, (bf16 *)P, d, fs, l);
+    else
+        pack_cat_kernel<float><<<1024, 256, 0, s>>>((const float *)Ds, (const float *)Wup, (float *)P, d, fs, l);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_split_router(const float *Wr, bf16 *split, int64_t n, cudaStream_t s)
+{
+    split_router_kernel<<<256, 256, 0, s>>>(Wr, split, n);
+    return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -1,0 +1,200 @@
+// Selection and dispatch: biased top-k with raw-score renormalisation, and a
+// stable counting sort of the T*k (token, slot) pairs by expert.
+//
+// Selection ("Stable LatentMoE", equations for T_k(x) and p_i): s = r + b,
+// T_k = TopK(s, k) with equal scores going to the lower expert index (the
+// cooking-agi LatentMoE page's routed_example picks index 0 when v0 >= v1),
+// p_i = r_i / sum_{j in T_k} r_j over the raw scores r.
+//
+// Dispatch: slot rows are ordered by (expert, token); a token selects an
+// expert at most once, so the position of (t, j) with e = sel[t, j] is
+//   offsets[e] + #{t' < t : t' selected e}.
+// Blocks of ROUTE_TPB tokens count per expert (topk kernel), one block scans
+// the counts over blocks and experts (scan kernel), and each block ranks its
+// tokens within an expert with a bit mask and popcounts (dispatch kernel).
+// Integer-only, hence bit-exact and deterministic.
+#include <float.h>
+
+#include "lmoe_internal.cuh"
+
+namespace lmoe {
+namespace {
+
+constexpr int TOPK_WARPS = 8;
+constexpr int KMAX = 64;
+
+template <typename TO>
+__global__ void __launch_bounds__(TOPK_WARPS * 32)
+topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t T, int E, int k,
+            int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
+            int32_t *__restrict__ blockhist)
+{
+    extern __shared__ float smem[];
+    float *s_all = smem;                              // [warps][E] biased scores (taken -> -inf)
+    float *r_all = s_all + TOPK_WARPS * E;            // [warps][E] raw scores
+    int *hist = (int *)(r_all + TOPK_WARPS * E);      // [E]
+    __shared__ int chosen[TOPK_WARPS][KMAX];
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+
+    float *sw = s_all + warp * E;
+    float *rw = r_all + warp * E;
+    const int64_t t_begin = (int64_t)blockIdx.x * ROUTE_TPB;
+    for (int i = warp; i < ROUTE_TPB; i += TOPK_WARPS) {
+        const int64_t t = t_begin + i;
+        if (t >= T) break;
+        for (int e = lane; e < E; e += 32) {
+            const float rv = r[t * E + e];
+            rw[e] = rv;
+            // NaN / -inf map to -FLT_MAX so that a candidate always exists and
+            // the chosen index stays in range whatever the input holds
+            sw[e] = fmaxf(rv + bias[e], -FLT_MAX);
+        }
+        __syncwarp();
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int e = lane; e < E; e += 32) {
+                const float v = sw[e];
+                if (v > bv) { bv = v; bi = e; }   // ascending e: strict > keeps the lower index
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if (lane == 0) {
+                chosen[warp][j] = bi;
+                sw[bi] = -INFINITY;
+            }
+            __syncwarp();
+        }
+        float sum = 0.f;   // every lane sums in selection order: identical result
+        for (int j = 0; j < k; ++j) sum += rw[chosen[warp][j]];
+        for (int j = lane; j < k; j += 32) {
+            const int e = chosen[warp][j];
+            const float p = rw[e] / sum;
+            sel[t * k + j] = e;
+            p32[t * k + j] = p;
+            p_out[t * k + j] = from_f32<TO>(p);
+            atomicAdd(&hist[e], 1);
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) blockhist[(int64_t)blockIdx.x * E + e] = hist[e];
+}
+
+// One block: per-expert totals and per-(block, expert) starting positions.
+__global__ void __launch_bounds__(1024)
+scan_kernel(const int32_t *__restrict__ blockhist, int nb, int E, int bm, int32_t *__restrict__ counts,
+            int32_t *__restrict__ offsets, int32_t *__restrict__ base, int32_t *__restrict__ tile_off)
+{
+    __shared__ int s_cnt[1024];
+    __shared__ int s_tiles[1024];
+    const int tid = threadIdx.x;
+    for (int e = tid; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int b = 0; b < nb; ++b) {
+            const int64_t i = (int64_t)b * E + e;
+            const int h = blockhist[i];
+            base[i] = run;
+            run += h;
+        }
+        counts[e] = run;
+        s_cnt[e] = run;
+        s_tiles[e] = (run + bm - 1) / bm;
+    }
+    __syncthreads();
+    if (tid == 0) {   // E <= 1024: a serial exclusive scan is a few microseconds at most
+        int acc = 0, tacc = 0;
+        for (int e = 0; e < E; ++e) {
+            offsets[e] = acc;
+            tile_off[e] = tacc;
+            const int c = s_cnt[e], tt = s_tiles[e];
+            s_cnt[e] = acc;
+            acc += c;
+            tacc += tt;
+        }
+        offsets[E] = acc;
+        tile_off[E] = tacc;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += blockDim.x) {
+        const int off = s_cnt[e];
+        for (int b = 0; b < nb; ++b) base[(int64_t)b * E + e] += off;
+    }
+}
+
+constexpr int WORDS = ROUTE_TPB / 32;
+
+__global__ void __launch_bounds__(256)
+dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, const int32_t *__restrict__ base,
+                int64_t T, int E, int k, int32_t *__restrict__ slot_of, int32_t *__restrict__ perm_tok,
+                float *__restrict__ perm_w)
+{
+    extern __shared__ uint32_t bits[];   // [E][WORDS]: bit i of expert e = token t_begin+i chose e
+    const int64_t t_begin = (int64_t)blockIdx.x * ROUTE_TPB;
+    const int ntok = (int)min((int64_t)ROUTE_TPB, T - t_begin);
+    for (int i = threadIdx.x; i < E * WORDS; i += blockDim.x) bits[i] = 0u;
+    __syncthreads();
+    const int n = ntok * k;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int tl = i / k;
+        const int e = sel[t_begin * k + i];
+        atomicOr(&bits[e * WORDS + (tl >> 5)], 1u << (tl & 31));
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int tl = i / k;
+        const int e = sel[t_begin * k + i];
+        const uint32_t *w = bits + e * WORDS;
+        int rank = __popc(w[tl >> 5] & ((1u << (tl & 31)) - 1u));
+        for (int q = 0; q < (tl >> 5); ++q) rank += __popc(w[q]);
+        const int pos = base[(int64_t)blockIdx.x * E + e] + rank;
+        slot_of[t_begin * k + i] = pos;
+        perm_tok[pos] = (int32_t)(t_begin + tl);
+        perm_w[pos] = p32[t_begin * k + i];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
+                        void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
+{
+    if (k > KMAX) return cudaErrorInvalidValue;
+    const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
+    const size_t smem = sizeof(float) * 2 * TOPK_WARPS * E + sizeof(int) * E;
+    if (out_bf16) {
+        cudaFuncSetAttribute(topk_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        topk_kernel<bf16><<<nb, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (bf16 *)p_out, blockhist);
+    } else {
+        cudaFuncSetAttribute(topk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        topk_kernel<float><<<nb, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (float *)p_out,
+                                                               blockhist);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int bm, int32_t *counts, int32_t *offsets,
+                        int32_t *base, int32_t *tile_off, cudaStream_t s)
+{
+    if (E > 1024) return cudaErrorInvalidValue;
+    scan_kernel<<<1, 1024, 0, s>>>(blockhist, nb, E, bm, counts, offsets, base, tile_off);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, int64_t T, int E, int k,
+                            int32_t *slot_of, int32_t *perm_tok, float *perm_w, cudaStream_t s)
+{
+    const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
+    const size_t smem = sizeof(uint32_t) * E * WORDS;
+    dispatch_kernel<<<nb, 256, smem, s>>>(sel, p32, base, T, E, k, slot_of, perm_tok, perm_w);
+    return cudaGetLastError();
+}
+
+}  // namespace lmoe

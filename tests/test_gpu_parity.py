@@ -1,0 +1,198 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle on B200.
+
+Sizes: small cases span several 128 x 256 tiles with ragged tails and are
+compared element by element on every row; the full-size workloads run the
+whole batch on the GPU (the launch configuration the benchmark times) and are
+compared on a seeded sample of token rows that the oracle computes one by one.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import lmoe_inputs as li
+import oracle
+from parity import compare, SEL_GAP
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def _lm():
+    import latent_space_routed_b200 as lm
+    return lm
+
+
+@functools.lru_cache(maxsize=2)
+def _weights(w):
+    return li.weights(w)
+
+
+def _layer(w, gemm=0, act=0):
+    lm = _lm()
+    W = _weights(w)
+    return lm.LatentMoE(lm.config_for(w, gemm=gemm, act=act), {k: v.cuda() for k, v in W.items()})
+
+
+def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0):
+    lm = _lm()
+    T = w.T if T is None else T
+    W = _weights(w)
+    x = li.tokens(w, T)
+    layer = _layer(w, gemm, lm.LMOE_ACT_SITU if act == "situ" else lm.LMOE_ACT_SWIGLU)
+    out = layer(x.cuda())
+    torch.cuda.synchronize()
+    layer.check_device(T)
+    rows = None
+    if n_rows is not None and n_rows < T:
+        rng = np.random.default_rng(1234 + seed)
+        rows = np.sort(rng.choice(T, size=n_rows, replace=False))
+        rows[-1] = T - 1   # always include the ragged tail
+        rows = np.unique(rows)
+    ora = oracle.forward(x, W, w.k, act=act, rows=rows, eps=w.eps)
+
+    def rerun(idx, sel):
+        r = idx if rows is None else rows[idx]
+        return oracle.forward(x, W, w.k, act=act, rows=r, sel=sel, eps=w.eps)
+
+    errs = compare({k: v.cpu() for k, v in out.items()}, ora, W["b"].numpy(), TOL[w.dtype], rerun, rows)
+    layer.close()
+    return errs, out
+
+
+# ---------------------------------------------------------------- small, all rows
+MULTI = li.custom("multi_tile_ragged", 1000, 512, 256, 256, 32, 6, 256, dtype="bf16", seed=21)
+
+
+def test_tiny_fp32_all_rows():
+    errs, _ = run_parity(li.WORKLOADS["tiny_fp32"])
+    assert errs["output"] < 1e-4
+
+
+def test_tiny_fp32_situ_gate():
+    run_parity(li.WORKLOADS["tiny_fp32"], act="situ")
+
+
+@pytest.mark.parametrize("gemm", [0, 1], ids=["tensor_cores", "cuda_cores"])
+def test_bf16_multi_tile_ragged(gemm):
+    run_parity(MULTI, gemm=gemm)
+
+
+def test_bf16_situ_tensor_cores():
+    run_parity(MULTI, act="situ")
+
+
+@pytest.mark.parametrize("T", [1, 2, 127, 129, 333])
+def test_bf16_token_counts(T):
+    run_parity(MULTI, T=T)
+
+
+@pytest.mark.parametrize("E,k", [(8, 8), (64, 1), (40, 17)])
+def test_bf16_selection_extremes(E, k):
+    w = li.custom(f"sel_{E}_{k}", 300, 256, 128, 256, E, k, 256, dtype="bf16", seed=22)
+    run_parity(w)
+
+
+def test_fp32_multi_tile_ragged():
+    w = li.custom("multi_f32", 333, 256, 128, 128, 24, 5, 192, dtype="f32", seed=23)
+    run_parity(w)
+
+
+# ---------------------------------------------------------------- stages
+def test_router_scores_and_dispatch_are_exact():
+    """Scores r match the fp64 oracle to fp32 rounding; counts, offsets, slot
+    positions and the slot -> token map equal a host stable counting sort of the
+    GPU's own selection, bit for bit."""
+    w = MULTI
+    T = w.T
+    W = _weights(w)
+    x = li.tokens(w)
+    layer = _layer(w)
+    out = layer(x.cuda())
+    torch.cuda.synchronize()
+    r_gpu = layer.region(T, "scores", torch.float32, (T, w.E)).cpu().numpy().astype(np.float64)
+    ora = oracle.forward(x, W, w.k, rows=np.arange(64))
+    assert np.abs(r_gpu[:64] - ora["scores"]).max() < 2e-6
+    sel = out["selected_experts"].cpu().numpy().astype(np.int64)
+    counts = np.bincount(sel.ravel(), minlength=w.E)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    slot_expected = np.zeros_like(sel)
+    perm_expected = np.zeros(T * w.k, np.int64)
+    fill = offsets[:-1].copy()
+    for t in range(T):
+        for j in range(w.k):
+            e = sel[t, j]
+            slot_expected[t, j] = fill[e]
+            perm_expected[fill[e]] = t
+            fill[e] += 1
+    np.testing.assert_array_equal(layer.region(T, "counts", torch.int32, (w.E,)).cpu().numpy(), counts)
+    np.testing.assert_array_equal(layer.region(T, "offsets", torch.int32, (w.E + 1,)).cpu().numpy(), offsets)
+    np.testing.assert_array_equal(layer.region(T, "slot_of", torch.int32, (T, w.k)).cpu().numpy(), slot_expected)
+    np.testing.assert_array_equal(layer.region(T, "perm_tok", torch.int32, (T * w.k,)).cpu().numpy(), perm_expected)
+    # every slot row of Z is the token's latent z = W_down x (bf16-rounded)
+    z = layer.region(T, "Z", torch.bfloat16, (T * w.k, w.l)).float().cpu()
+    zt = (x.double() @ W["W_down"].double().T)
+    ref = zt[torch.from_numpy(perm_expected)]
+    assert ((z.double() - ref).abs().max() / ref.abs().max()).item() < 1e-2
+    layer.close()
+
+
+def test_deterministic_and_host_entry_matches():
+    w = MULTI
+    lm = _lm()
+    x = li.tokens(w)
+    layer = _layer(w)
+    a = {k: v.clone() for k, v in layer(x.cuda()).items()}
+    b = layer(x.cuda())
+    for key in a:
+        assert torch.equal(a[key], b[key]), key
+    xh = x.pin_memory()
+    oh = layer.empty_outputs(w.T, device="cpu", pin=True)
+    layer.forward_host(xh, oh)
+    torch.cuda.synchronize()
+    for key in a:
+        assert torch.equal(a[key].cpu(), oh[key]), key
+    assert layer.launch_count(w.T) > 0
+    layer.close()
+
+
+def test_zero_tokens_is_a_noop_and_errors_are_reported():
+    lm = _lm()
+    w = MULTI
+    layer = _layer(w)
+    x = torch.empty(0, w.d, dtype=torch.bfloat16, device="cuda")
+    lm.lmoe_forward(layer.handle, x, 0, None, None, None, None, None, 0)
+    x = li.tokens(w, 16).cuda()
+    out = layer.empty_outputs(16)
+    with pytest.raises(lm.LmoeError) as ei:
+        lm.lmoe_forward(layer.handle, x, 16, out["output"], out["selected_experts"], out["mixture_weights"],
+                        out["latent_routed_aggregate"], layer.workspace(16), 64)
+    assert ei.value.status == lm.LMOE_ERR_WORKSPACE
+    ws = layer.workspace(16)
+    xm = torch.empty(16 * w.d + 1, dtype=torch.bfloat16, device="cuda")[1:].view(16, w.d)
+    with pytest.raises(lm.LmoeError) as ei:
+        lm.lmoe_forward(layer.handle, xm, 16, out["output"], out["selected_experts"], out["mixture_weights"],
+                        out["latent_routed_aggregate"], ws, ws.numel())
+    assert ei.value.status == lm.LMOE_ERR_UNSUPPORTED
+    layer.close()
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled rows
+@pytest.mark.parametrize("name,n_rows", [("acc_d2048", 64), ("eff_zipf_d2048", 64)])
+def test_full_size_sampled_rows(name, n_rows):
+    errs, _ = run_parity(li.WORKLOADS[name], n_rows=n_rows)
+    print(name, errs)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 128])
+def test_decode_sweep(T):
+    w = li.WORKLOADS["decode_d7168"]
+    errs, _ = run_parity(w, T=T, n_rows=min(T, 16))
+    print("decode", T, errs)
+
+
+def test_large_sampled_rows():
+    errs, _ = run_parity(li.WORKLOADS["large_d4096"], n_rows=24)
+    print("large", errs)
