@@ -281,6 +281,6 @@ class LatentMoE:
 
 def config_for(workload, gemm: int = 0, act: int = LMOE_ACT_SWIGLU) -> lmoe_config:
     """lmoe_config from an lmoe_inputs.Workload."""
-    return make_config(workload.d, workload.l, workload.f, workload.E, workload.k, workload.f_shared,
+    return make_config(workload.d, workload.l, workload.f, workload.E, workload.k, workload.f_s,
                        workload.n_shared, workload.eps, LMOE_F32 if workload.dtype == "f32" else LMOE_BF16, act,
                        4.0, 25.0, gemm)

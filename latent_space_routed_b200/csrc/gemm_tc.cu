@@ -40,10 +40,11 @@ constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;   // 2 role warps + 8 epilogue warps
 constexpr int TMEM_COLS = 2 * BN;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+constexpr int MAX_E = 1024;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * sizeof(int) * (MAX_E + 1);
 
 // status codes (OR-ed together)
 constexpr int ST_PRODUCER = 0x1, ST_MMA = 0x2, ST_EPILOGUE = 0x4, ST_DRAIN = 0x8;
@@ -60,6 +61,8 @@ struct TcParams {
     const int32_t *tile_off;
     int E;
     int max_tiles;              // dense: exact tile count
+    const int32_t *a_gather;    // gather mode: A row of each logical row
+    int64_t gather_last;        // last valid logical row (indices are clamped to it)
     EpiArgs epi;
     int32_t *status;
 };
@@ -121,6 +124,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
+// Four rows (indices r[0..3]) x one 64-column box of a row-major matrix.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, const int *r)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)map) : "memory");
@@ -156,21 +169,47 @@ __device__ __forceinline__ void umma_commit(uint32_t bar)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
+// bf16 outputs only: the gate with the hardware exp2 and reciprocal
+// approximations (a few ulp of fp32, far below the bf16 rounding that follows).
+__device__ __forceinline__ float rcp_approx(float x)
 {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <bool SITU>
+__device__ __forceinline__ float glu_fast(float g, float v, float cg, float cu)
+{
+    const float sg = rcp_approx(1.0f + __expf(-g));
+    if (SITU) return cg * tanhf(g * rcp_approx(cg)) * sg * (cu * tanhf(v * rcp_approx(cu)));
+    return g * sg * v;
+}
+
+// Two 32x32b.x32 loads in flight, then one wait.
+__device__ __forceinline__ void tmem_ld32_pair(uint32_t ta, uint32_t tb, float *va, float *vb)
+{
+    uint32_t r[32], s[32];
+#define LMOE_TMEM_LD(dst, addr)                                                                                  \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "                                                      \
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "                       \
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"       \
+                 : "=r"(dst[0]), "=r"(dst[1]), "=r"(dst[2]), "=r"(dst[3]), "=r"(dst[4]), "=r"(dst[5]),            \
+                   "=r"(dst[6]), "=r"(dst[7]), "=r"(dst[8]), "=r"(dst[9]), "=r"(dst[10]), "=r"(dst[11]),          \
+                   "=r"(dst[12]), "=r"(dst[13]), "=r"(dst[14]), "=r"(dst[15]), "=r"(dst[16]), "=r"(dst[17]),      \
+                   "=r"(dst[18]), "=r"(dst[19]), "=r"(dst[20]), "=r"(dst[21]), "=r"(dst[22]), "=r"(dst[23]),      \
+                   "=r"(dst[24]), "=r"(dst[25]), "=r"(dst[26]), "=r"(dst[27]), "=r"(dst[28]), "=r"(dst[29]),      \
+                   "=r"(dst[30]), "=r"(dst[31])                                                                   \
+                 : "r"(addr))
+    LMOE_TMEM_LD(r, ta);
+    LMOE_TMEM_LD(s, tb);
+#undef LMOE_TMEM_LD
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    for (int i = 0; i < 32; ++i) {
+        va[i] = __uint_as_float(r[i]);
+        vb[i] = __uint_as_float(s[i]);
+    }
 }
 
 // ------------------------------------------------------------------ epilogue stores
@@ -215,7 +254,9 @@ struct Tile {
     int n0;                 // first output column (GEMM n)
 };
 
-__device__ __forceinline__ Tile decode(const TcParams &p, int tile)
+// Grouped mode reads the expert row offsets and m-tile prefix from shared
+// memory (staged once per CTA), so decoding a tile costs no global round trip.
+__device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off, const int *s_offsets, int tile)
 {
     Tile t;
     const int mt = tile / p.ntn, nt = tile % p.ntn;
@@ -224,10 +265,10 @@ __device__ __forceinline__ Tile decode(const TcParams &p, int tile)
         int lo = 0, hi = p.E - 1;  // last e with tile_off[e] <= mt
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(p.tile_off + mid) <= mt) lo = mid; else hi = mid - 1;
+            if (s_tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
         }
-        t.row0 = (int64_t)__ldg(p.offsets + lo) + (int64_t)(mt - __ldg(p.tile_off + lo)) * BM;
-        t.row_end = __ldg(p.offsets + lo + 1);
+        t.row0 = (int64_t)s_offsets[lo] + (int64_t)(mt - s_tile_off[lo]) * BM;
+        t.row_end = s_offsets[lo + 1];
         t.brow = (int64_t)lo * p.group_rows + t.n0;
     } else {
         t.row0 = (int64_t)mt * BM;
@@ -237,7 +278,7 @@ __device__ __forceinline__ Tile decode(const TcParams &p, int tile)
     return t;
 }
 
-template <int MODE, typename TO>
+template <int MODE, typename TO, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p)
 {
@@ -250,6 +291,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
     int *abort_flag = reinterpret_cast<int *>(tmem_holder + 1);
     int *drain_counts = abort_flag + 1;                      // [0] loads issued, [1] stages consumed
+    int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * STAGE_BYTES + 256);   // [E+1]
+    int *s_offsets = s_tile_off + (MAX_E + 1);                                              // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t bar0 = smem_u32(bars);
@@ -265,7 +308,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(accf_bar(a), 1);
-            mbar_init(acce_bar(a), 4);   // one arrival per epilogue warp
+            mbar_init(acce_bar(a), 8);   // one arrival per epilogue warp
         }
         *abort_flag = 0;
         drain_counts[0] = drain_counts[1] = 0;
@@ -273,6 +316,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+    }
+    if (p.offsets) {
+        for (int i = threadIdx.x; i <= p.E; i += THREADS) {
+            s_tile_off[i] = p.tile_off[i];
+            s_offsets[i] = p.offsets[i];
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
@@ -285,32 +334,48 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    const int total = p.offsets ? __ldg(p.tile_off + p.E) * p.ntn : p.max_tiles;
+    const int total = p.offsets ? s_tile_off[p.E] * p.ntn : p.max_tiles;
     const int nkb_total = p.nkb * p.nterms;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------------------------------------------- TMA producer
-            int it = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode(p, tile);
-                for (int kb = 0; kb < nkb_total; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        // -------------------------------------------------------- TMA producer warp
+        // Lane 0 waits for a free stage, arms its barrier and loads B (and A when
+        // not gathering); with GATHER every lane then loads four A rows of the
+        // 128-row tile with one tile::gather4 (lane i: rows 4i .. 4i+3).
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+            const Tile t = decode(p, s_tile_off, s_offsets, tile);
+            int ridx[4] = {0, 0, 0, 0};
+            if (GATHER) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int64_t lr = t.row0 + 4 * lane + j;
+                    if (lr > p.gather_last) lr = p.gather_last;
+                    ridx[j] = __ldg(p.a_gather + lr);
+                }
+            }
+            for (int kb = 0; kb < nkb_total; ++kb, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
+                const uint32_t sa = sbase + (uint32_t)s * STAGE_BYTES;
+                int good = 1;
+                if (lane == 0) {
                     if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
                         atomicOr(p.status, ST_PRODUCER);
                         *(volatile int *)abort_flag = 1;
-                        ok = false;
-                        break;
+                        good = 0;
+                    } else {
+                        mbar_expect_tx(full_bar(s), STAGE_BYTES);
+                        tma_load_2d(sa + A_BYTES, &tmB, full_bar(s), kk, (int)(t.brow + term * p.term_rows));
+                        if (!GATHER) tma_load_2d(sa, &tmA, full_bar(s), kk, (int)t.row0);
                     }
-                    const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
-                    const uint32_t sa = sbase + (uint32_t)s * STAGE_BYTES;
-                    mbar_expect_tx(full_bar(s), STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, full_bar(s), kk, (int)t.row0);
-                    tma_load_2d(sa + A_BYTES, &tmB, full_bar(s), kk, (int)(t.brow + term * p.term_rows));
-                    drain_counts[0] = it + 1;
                 }
+                good = __shfl_sync(0xffffffffu, good, 0);
+                if (!good) { ok = false; break; }
+                if (GATHER) tma_gather4(sa + 512u * lane, &tmA, full_bar(s), kk, ridx);
+                if (lane == 0) drain_counts[0] = it + 1;
             }
         }
     } else if (warp == 1) {
@@ -352,8 +417,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
         }
     } else {
-        // -------------------------------------------------------- epilogue warps 2..5
+        // -------------------------------------------------------- epilogue warps 2..9
+        // Two warps per TMEM lane quarter; warp set h = 0/1 takes the 32-column
+        // chunks c = 32 h + 64 i, so each warp drains half of its 32 rows' tile.
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
         int local = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
             const int acc = local & 1;
@@ -367,47 +435,47 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const Tile t = decode(p, tile);
+            const Tile t = decode(p, s_tile_off, s_offsets, tile);
             const int64_t row = t.row0 + 32 * q + lane;
             const bool valid = row < t.row_end;
             const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
-            float v[32];
-            if (MODE == EPI_GLU) {
+            float v[32], u[32];
+            if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
                 const int half = BN / 2;
-                for (int c = 0; c < half; c += 32) {
-                    float u[32];
+#pragma unroll 1
+                for (int c = 32 * hset; c < half; c += 64) {
                     __syncwarp();
-                    tmem_ld32(tq + c, v);
-                    tmem_ld32(tq + half + c, u);
+                    tmem_ld32_pair(tq + c, tq + half + c, v, u);   // gate and up columns, one wait
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = glu_act(p.epi.act, v[i], u[i], p.epi.gate_cap, p.epi.up_cap);
+                    for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
+                                                                                       p.epi.up_cap);
                     if (valid) store_n((TO *)p.epi.out + row * p.epi.ldo + t.n0 / 2 + c, v, 32);
                 }
             } else {
-                for (int c = 0; c < BN; c += 32) {
+#pragma unroll 1
+                for (int c = 32 * hset; c < BN; c += 128) {
                     __syncwarp();
-                    tmem_ld32(tq + c, v);            // warp-collective: every lane, every chunk
-                    const int col = t.n0 + c;
-                    int n = p.N - col;
-                    if (n > 32) n = 32;
-                    if (!valid || n <= 0) {
-                        // nothing to store for this lane
-                    } else if (MODE == EPI_SIGMOID) {
+                    tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // warp-collective: every lane
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = sigmoidf_(v[i]);
-                        store_n((float *)p.epi.out + row * p.epi.ldo + col, v, n);
-                    } else if (MODE == EPI_COMBINE) {
-                        const float w = p.epi.row_w[row];
+                    for (int part = 0; part < 2; ++part) {
+                        float *x = part ? u : v;
+                        const int col = t.n0 + c + 64 * part;
+                        int n = p.N - col;
+                        if (n > 32) n = 32;
+                        if (!valid || n <= 0) {
+                            // nothing to store for this lane
+                        } else if (MODE == EPI_SIGMOID) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= w;
-                        store_n((float *)p.epi.out + row * p.epi.ldo + col, v, n);
-                    } else if (MODE == EPI_SCATTER) {
-                        for (int j = 0; j < p.epi.k; ++j) {
-                            const int64_t dst = p.epi.slot_of[row * p.epi.k + j];
-                            store_n((TO *)p.epi.out + dst * p.epi.ldo + col, v, n);
+                            for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
+                            store_n((float *)p.epi.out + row * p.epi.ldo + col, x, n);
+                        } else if (MODE == EPI_COMBINE) {
+                            const float w = p.epi.row_w[row];
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) x[i] *= w;
+                            store_n((float *)p.epi.out + row * p.epi.ldo + col, x, n);
+                        } else {
+                            store_n((TO *)p.epi.out + row * p.epi.ldo + col, x, n);
                         }
-                    } else {
-                        store_n((TO *)p.epi.out + row * p.epi.ldo + col, v, n);
                     }
                 }
             }
@@ -457,10 +525,10 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
 template <int MODE, typename TO>
 cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const TcParams &p, int grid, cudaStream_t s)
 {
-    const cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)SMEM_BYTES);
+    auto kern = p.a_gather ? tc_gemm_kernel<MODE, TO, true> : tc_gemm_kernel<MODE, TO, false>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    tc_gemm_kernel<MODE, TO><<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
+    kern<<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
     return cudaGetLastError();
 }
 
@@ -477,7 +545,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.nkb = g.K / BK;
     p.nterms = nterms;
     p.term_rows = term_rows;
-    p.ntn = mode == EPI_GLU ? g.N / BN : (g.N + BN - 1) / BN;
+    p.ntn = mode == EPI_GLU ? g.N / BN : (g.N + BN - 1) / BN;   // GLU: N = 2F, F % (BN/2) == 0
     p.group_rows = g.offsets ? g.b_group_stride / g.ldb : 0;
     p.offsets = g.offsets;
     p.tile_off = g.tile_off;
@@ -487,16 +555,21 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.epi = g.epi;
     p.status = status;
     if (p.max_tiles == 0) return cudaSuccess;
-    const int64_t a_rows = g.M;   // grouped: M = total slot rows
+    p.a_gather = g.a_gather;
+    p.gather_last = (int64_t)g.M - 1;
+    const int64_t a_rows = g.a_gather ? g.a_rows : g.M;   // grouped: M = total slot rows
     CUtensorMap ta, tb;
-    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)a_rows, (uint64_t)g.lda * 2, BM)) return cudaErrorInvalidValue;
+    // gather: box one row high, four rows per tile::gather4
+    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)a_rows, (uint64_t)g.lda * 2, g.a_gather ? 1 : BM))
+        return cudaErrorInvalidValue;
     if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN))
         return cudaErrorInvalidValue;
     const int grid = p.max_tiles < g_num_sms ? p.max_tiles : g_num_sms;
     switch (mode) {
     case EPI_SIGMOID: return launch<EPI_SIGMOID, float>(ta, tb, p, grid, s);
-    case EPI_SCATTER: return launch<EPI_SCATTER, bf16>(ta, tb, p, grid, s);
-    case EPI_GLU: return launch<EPI_GLU, bf16>(ta, tb, p, grid, s);
+    case EPI_GLU:
+        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16>(ta, tb, p, grid, s);
+        return launch<EPI_GLU, bf16>(ta, tb, p, grid, s);
     case EPI_COMBINE: return launch<EPI_COMBINE, float>(ta, tb, p, grid, s);
     case EPI_STORE: return launch<EPI_STORE, bf16>(ta, tb, p, grid, s);
     default: return cudaErrorInvalidValue;

@@ -7,8 +7,9 @@
 //   2 top-k            sel, p (fp32 and token dtype), per-block expert counts
 //   3 scan             counts, offsets, per-block bases, m-tile prefix
 //   4 dispatch         slot_of[t, j], token and weight of every slot row
-//   5 down GEMM        z = x W_down^T, each row written to its k slot rows
-//   6 gate/up GEMM     per expert: h = act(G z, U z)            [S, f]
+//   5 down GEMM        z = x W_down^T                           [T, l]
+//   6 gate/up GEMM     per expert: h = act(G z, U z), the A rows gathered
+//                      from z through the slot -> token map      [S, f]
 //   7 down GEMM        per expert: Y = p * (h D^T)              [S, l] fp32
 //   8 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
 //   9 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
@@ -94,7 +95,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.slot_of = take(sizeof(int32_t) * S);
     L.perm_tok = take(sizeof(int32_t) * S);
     L.perm_w = take(sizeof(float) * S);
-    L.Zp = take(h->tb * S * c.l);
+    L.Zp = take(h->tb * T * c.l);
     L.H = take(h->tb * S * c.f);
     L.Yp = take(sizeof(float) * S * c.l);
     L.HS = take(h->tb * T * (2 * (int64_t)c.f_shared + c.l));
@@ -260,7 +261,7 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 3: *offset = L.offsets; *bytes = sizeof(int32_t) * (c.E + 1); break;
     case 4: *offset = L.slot_of; *bytes = sizeof(int32_t) * S; break;
     case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
-    case 6: *offset = L.Zp; *bytes = h->tb * S * c.l; break;
+    case 6: *offset = L.Zp; *bytes = h->tb * T * c.l; break;
     case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
     case 8: *offset = L.Yp; *bytes = sizeof(float) * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
@@ -285,8 +286,9 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
 {
     g_err.clear();
     if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
-    // status reset, router, top-k, scan, dispatch, down, gate/up, down+combine, norm, shared, final
-    *launches = T == 0 ? 0 : 11;
+    // status reset, router, histogram reset, top-k, scan, dispatch, down, gate/up, down+combine, norm,
+    // shared, final
+    *launches = T == 0 ? 0 : 12;
     return LMOE_OK;
 }
 
@@ -363,13 +365,13 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     STAGE(3);
     LMOE_CUDA(launch_dispatch(selected_experts, p32, base, T, c.E, c.k, slot_of, perm_tok, perm_w, s));
 
-    // 5 z = x W_down^T scattered to the k slot rows of each token
+    // 5 z = x W_down^T, once per token
     GemmArgs gd = {};
     gd.A = x; gd.lda = c.d; gd.B = h->Wdown; gd.ldb = c.d; gd.M = (int)T; gd.N = c.l; gd.K = c.d;
-    gd.epi.out = Zp; gd.epi.ldo = c.l; gd.epi.slot_of = slot_of; gd.epi.k = c.k;
-    // 6 per expert h = act(G z, U z)
+    gd.epi.out = Zp; gd.epi.ldo = c.l;
+    // 6 per expert h = act(G z, U z); slot row m reads z[perm_tok[m]]
     GemmArgs gu = {};
-    gu.A = Zp; gu.lda = c.l; gu.B = h->Wgu; gu.ldb = c.l; gu.b_group_stride = 2 * (int64_t)c.f * c.l;
+    gu.A = Zp; gu.lda = c.l; gu.a_gather = perm_tok; gu.a_rows = T; gu.B = h->Wgu; gu.ldb = c.l; gu.b_group_stride = 2 * (int64_t)c.f * c.l;
     gu.M = (int)S; gu.N = 2 * c.f; gu.K = c.l; gu.offsets = offsets; gu.tile_off = tile_off; gu.E = c.E;
     gu.epi.out = H; gu.epi.ldo = c.f; gu.epi.act = c.act; gu.epi.gate_cap = c.gate_cap; gu.epi.up_cap = c.up_cap;
     gu.epi.ib = h->ib;
@@ -389,8 +391,8 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     gf.epi.out = output; gf.epi.ldo = c.d;
 
     STAGE(4);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_SCATTER, gd, 0, status, s));
-    else LMOE_CUDA(launch_simt_gemm(EPI_SCATTER, tk, tk, tk, gd, 0, s));
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gd, 0, status, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, s));
     STAGE(5);
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, s));
@@ -409,7 +411,6 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, s));
     STAGE(LMOE_NUM_STAGES);
 #undef STAGE
-    (void)perm_tok;
     return LMOE_OK;
 }
 

@@ -33,19 +33,19 @@ __device__ __forceinline__ float glu_act(int act, float g, float v, float cg, fl
 // ---------------------------------------------------------------- epilogues
 // Every GEMM here computes C[m, n] = sum_k A[m, k] B[n, k] (both K-major) and
 // hands each row chunk of fp32 accumulators to one of these epilogues.
+// (Mode 2 is unused: the down-projection stores z once and the routed GEMM
+// gathers its rows.)
 enum EpiMode {
     EPI_STORE = 0,    // out[m, n] = C                      (final GEMM -> y)
     EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
-    EPI_SCATTER = 2,  // out[slot_of[m, j], n] = C, j < k   (down-projection -> Z slots)
     EPI_GLU = 3,      // out[m, n'] = act(C[gate], C[up])   (gate/up GEMMs -> h)
-    EPI_COMBINE = 4   // out32[m, n] = w[m] * C             (routed down -> p-weighted rows)
+    EPI_COMBINE = 4,  // out32[m, n] = w[m] * C             (routed down -> p-weighted rows)
+    EPI_GLU_SITU = 5  // EPI_GLU with the SiTU gate, as its own instantiation
 };
 
 struct EpiArgs {
     void *out;
     int64_t ldo;             // row stride of out, elements
-    const int32_t *slot_of;  // EPI_SCATTER: [rows, k]
-    int k;
     const float *row_w;      // EPI_COMBINE: weight of each row
     int act;                 // EPI_GLU
     float gate_cap, up_cap;
@@ -65,13 +65,6 @@ __device__ __forceinline__ void epi_store_chunk(const EpiArgs &e, int64_t row, i
         const float w = e.row_w[row];
         #pragma unroll
         for (int i = 0; i < 32; ++i) if (i < n) o[i] = w * v[i];
-    } else if (MODE == EPI_SCATTER) {
-        for (int j = 0; j < e.k; ++j) {
-            const int64_t dst = e.slot_of[row * e.k + j];
-            TO *o = (TO *)e.out + dst * e.ldo + col;
-            #pragma unroll
-            for (int i = 0; i < 32; ++i) if (i < n) o[i] = from_f32<TO>(v[i]);
-        }
     } else {
         TO *o = (TO *)e.out + row * e.ldo + col;
 #pragma unroll
@@ -90,6 +83,8 @@ struct GemmArgs {
     const int32_t *offsets;   // grouped: [E+1] row offsets, else nullptr
     const int32_t *tile_off;  // grouped: [E+1] m-tile prefix for this kernel's BM
     int E;
+    const int32_t *a_gather;  // optional: logical row m reads A row a_gather[m] (m < M)
+    int64_t a_rows;           // physical rows of A (a_gather set), for bounds and the TMA map
     EpiArgs epi;
 };
 

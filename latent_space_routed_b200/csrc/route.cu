@@ -9,9 +9,10 @@
 // Dispatch: slot rows are ordered by (expert, token); a token selects an
 // expert at most once, so the position of (t, j) with e = sel[t, j] is
 //   offsets[e] + #{t' < t : t' selected e}.
-// Blocks of ROUTE_TPB tokens count per expert (topk kernel), one block scans
-// the counts over blocks and experts (scan kernel), and each block ranks its
-// tokens within an expert with a bit mask and popcounts (dispatch kernel).
+// The top-k kernel (one warp per token) counts each expert's selections per
+// block of ROUTE_TPB tokens, one block scans the counts over blocks and
+// experts (scan kernel), and each block of ROUTE_TPB tokens ranks its tokens
+// within an expert with a bit mask and popcounts (dispatch kernel).
 // Integer-only, hence bit-exact and deterministic.
 #include <float.h>
 
@@ -20,7 +21,7 @@
 namespace lmoe {
 namespace {
 
-constexpr int TOPK_WARPS = 8;
+constexpr int TOPK_WARPS = 8;   // one token per warp, 8 tokens per block
 constexpr int KMAX = 64;
 
 template <typename TO>
@@ -30,62 +31,50 @@ topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t
             int32_t *__restrict__ blockhist)
 {
     extern __shared__ float smem[];
-    float *s_all = smem;                              // [warps][E] biased scores (taken -> -inf)
-    float *r_all = s_all + TOPK_WARPS * E;            // [warps][E] raw scores
-    int *hist = (int *)(r_all + TOPK_WARPS * E);      // [E]
     __shared__ int chosen[TOPK_WARPS][KMAX];
-
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-    __syncthreads();
-
-    float *sw = s_all + warp * E;
-    float *rw = r_all + warp * E;
-    const int64_t t_begin = (int64_t)blockIdx.x * ROUTE_TPB;
-    for (int i = warp; i < ROUTE_TPB; i += TOPK_WARPS) {
-        const int64_t t = t_begin + i;
-        if (t >= T) break;
+    float *sw = smem + warp * 2 * E;   // biased scores of this warp's token (taken -> -inf)
+    float *rw = sw + E;                // raw scores
+    const int64_t t = (int64_t)blockIdx.x * TOPK_WARPS + warp;
+    if (t >= T) return;
+    for (int e = lane; e < E; e += 32) {
+        const float rv = r[t * E + e];
+        rw[e] = rv;
+        // NaN / -inf map to -FLT_MAX so that a candidate always exists and
+        // the chosen index stays in range whatever the input holds
+        sw[e] = fmaxf(rv + bias[e], -FLT_MAX);
+    }
+    __syncwarp();
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
         for (int e = lane; e < E; e += 32) {
-            const float rv = r[t * E + e];
-            rw[e] = rv;
-            // NaN / -inf map to -FLT_MAX so that a candidate always exists and
-            // the chosen index stays in range whatever the input holds
-            sw[e] = fmaxf(rv + bias[e], -FLT_MAX);
+            const float v = sw[e];
+            if (v > bv) { bv = v; bi = e; }   // ascending e: strict > keeps the lower index
         }
-        __syncwarp();
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int e = lane; e < E; e += 32) {
-                const float v = sw[e];
-                if (v > bv) { bv = v; bi = e; }   // ascending e: strict > keeps the lower index
-            }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-            }
-            if (lane == 0) {
-                chosen[warp][j] = bi;
-                sw[bi] = -INFINITY;
-            }
-            __syncwarp();
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
         }
-        float sum = 0.f;   // every lane sums in selection order: identical result
-        for (int j = 0; j < k; ++j) sum += rw[chosen[warp][j]];
-        for (int j = lane; j < k; j += 32) {
-            const int e = chosen[warp][j];
-            const float p = rw[e] / sum;
-            sel[t * k + j] = e;
-            p32[t * k + j] = p;
-            p_out[t * k + j] = from_f32<TO>(p);
-            atomicAdd(&hist[e], 1);
+        if (lane == 0) {
+            chosen[warp][j] = bi;
+            sw[bi] = -INFINITY;
         }
         __syncwarp();
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) blockhist[(int64_t)blockIdx.x * E + e] = hist[e];
+    float sum = 0.f;   // every lane sums in selection order: identical result
+    for (int j = 0; j < k; ++j) sum += rw[chosen[warp][j]];
+    int32_t *hist = blockhist + (t / ROUTE_TPB) * E;
+    for (int j = lane; j < k; j += 32) {
+        const int e = chosen[warp][j];
+        const float p = rw[e] / sum;
+        sel[t * k + j] = e;
+        p32[t * k + j] = p;
+        p_out[t * k + j] = from_f32<TO>(p);
+        atomicAdd(&hist[e], 1);
+    }
 }
 
 // One block: per-expert totals and per-(block, expert) starting positions.
@@ -167,8 +156,11 @@ cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int
                         void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
 {
     if (k > KMAX) return cudaErrorInvalidValue;
-    const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
-    const size_t smem = sizeof(float) * 2 * TOPK_WARPS * E + sizeof(int) * E;
+    const int64_t nhb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
+    cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nhb * E, s);
+    if (e != cudaSuccess) return e;
+    const unsigned nb = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
+    const size_t smem = sizeof(float) * 2 * TOPK_WARPS * E;
     if (out_bf16) {
         cudaFuncSetAttribute(topk_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         topk_kernel<bf16><<<nb, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (bf16 *)p_out, blockhist);
