@@ -82,7 +82,8 @@ def stage_model(w, T, touched):
         "topk": (0, 4 * T * w.E + T * w.k * (8 + B)),
         "scan": (0, 0),
         "dispatch": (0, T * w.k * 16),
-        "down_proj": (2 * T * w.d * w.l, T * w.d * B + w.l * w.d * B + S * w.l * B),
+        "down_proj": (2 * T * w.d * w.l, T * w.d * B + w.l * w.d * B + T * w.l * B),
+        "permute": (0, T * w.l * B + S * w.l * B + S * 4),
         "gate_up": (2 * S * 2 * w.f * w.l, touched * 2 * w.f * w.l * B + S * w.l * B + S * w.f * B),
         "down_combine": (2 * S * w.l * w.f, touched * w.l * w.f * B + S * w.f * B + S * w.l * 4),
         "combine_norm": (0, S * w.l * 4 + 2 * T * w.l * B),

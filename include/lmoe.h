@@ -170,9 +170,10 @@ LMOE_API lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream)
 
 /* Stages of one forward, in launch order (for lmoe_set_stage_events):
  *  0 router GEMM, 1 top-k, 2 counting-sort scan, 3 dispatch, 4 down-projection
- *  GEMM, 5 routed gate/up GEMM, 6 routed down GEMM + weighting, 7 combine +
- *  RMSNorm, 8 shared gate/up GEMM, 9 final GEMM (shared down + up-projection). */
-#define LMOE_NUM_STAGES 10
+ *  GEMM, 5 copy of z to the expert-sorted slot rows, 6 routed gate/up GEMM,
+ *  7 routed down GEMM + weighting, 8 combine + RMSNorm, 9 shared gate/up GEMM,
+ *  10 final GEMM (shared down + up-projection). */
+#define LMOE_NUM_STAGES 11
 
 /* Ask subsequent lmoe_forward calls on this handle to record events[i] (each
  * a cudaEvent_t created by the caller) on the forward's stream right before

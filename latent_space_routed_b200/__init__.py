@@ -159,9 +159,9 @@ def lmoe_set_bias(h, b, stream=None):
     _check(_lib.lmoe_set_bias(h, _ptr(b), _stream(stream)))
 
 
-LMOE_NUM_STAGES = 10
-STAGE_NAMES = ("router", "topk", "scan", "dispatch", "down_proj", "gate_up", "down_combine", "combine_norm",
-               "shared_gate_up", "final")
+LMOE_NUM_STAGES = 11
+STAGE_NAMES = ("router", "topk", "scan", "dispatch", "down_proj", "permute", "gate_up", "down_combine",
+               "combine_norm", "shared_gate_up", "final")
 
 
 def lmoe_set_stage_events(h, events, n):

@@ -7,8 +7,8 @@
 // accumulator tile is staged through shared memory so every epilogue sees
 // whole row chunks.
 //
-// Grouped mode (offsets != nullptr): the rows are the expert-sorted slot
-// rows (A row of slot row m: a_gather[m] when set); m-tile i belongs to the expert e with tile_off[e] <= i < tile_off[e+1]
+// Grouped mode (offsets != nullptr): the rows of A are the expert-sorted slot
+// rows; m-tile i belongs to the expert e with tile_off[e] <= i < tile_off[e+1]
 // and covers rows offsets[e] + 64 (i - tile_off[e]) .. min(+64, offsets[e+1]);
 // B for that expert starts at B + e * b_group_stride.
 #include "lmoe_internal.cuh"
@@ -59,9 +59,8 @@ __global__ void __launch_bounds__(NT) simt_gemm_kernel(GemmArgs g)
     // load assignment: A 64 rows x 16 k (4 per thread), B 128 rows x 16 k (8 per thread)
     const int a_r = tid / 4, a_k = (tid % 4) * 4;
     const int b_r = tid / 2, b_k = (tid % 2) * 8;
-    const int64_t a_lrow = row0 + a_r;
-    const bool a_ok = a_lrow < row_end;
-    const int64_t a_row = (g.a_gather && a_ok) ? (int64_t)g.a_gather[a_lrow] : a_lrow;
+    const int64_t a_row = row0 + a_r;
+    const bool a_ok = a_row < row_end;
     const int b_row = n0 + b_r;
     const bool b_ok = b_row < g.N;
 

@@ -24,7 +24,7 @@
 // on whatever the TMA brought in (the next expert's rows, or zero fill past the
 // end) and discarded by the epilogue.
 //
-// Every mbarrier wait is bounded by a wall-clock limit; a wait that gives up
+// Every mbarrier wait is bounded by a cycle-count limit (about 2 s); a wait that gives up
 // ORs a code into the status word, stops its role's loop, and the CTA drains
 // the copies and MMAs it still has in flight (again bounded) before it frees
 // its TMEM and returns.
@@ -42,7 +42,7 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 320;   // 2 role warps + 8 epilogue warps
 constexpr int TMEM_COLS = 2 * BN;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr long long WAIT_LIMIT_CYCLES = 4000000000ll;   // about 2 s at 2 GHz
 constexpr int MAX_E = 1024;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * sizeof(int) * (MAX_E + 1);
 
@@ -61,21 +61,12 @@ struct TcParams {
     const int32_t *tile_off;
     int E;
     int max_tiles;              // dense: exact tile count
-    const int32_t *a_gather;    // gather mode: A row of each logical row
-    int64_t gather_last;        // last valid logical row (indices are clamped to it)
     EpiArgs epi;
     int32_t *status;
 };
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t globaltimer()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
@@ -106,13 +97,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Wait for the phase with the given parity to complete; false after the limit.
+// The limit is counted on the SM's own cycle counter (cheap to read, unlike
+// the global nanosecond timer, which is a long-latency read).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
-    for (uint32_t i = 1;; ++i) {
+    const long long t0 = clock64();
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0 && globaltimer() - t0 > WAIT_LIMIT_NS) return false;
+        if (clock64() - t0 > WAIT_LIMIT_CYCLES) return false;
     }
 }
 
@@ -121,16 +114,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
         ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
-}
-
-// Four rows (indices r[0..3]) x one 64-column box of a row-major matrix.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, const int *r)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
         : "memory");
 }
 
@@ -278,7 +261,7 @@ __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off,
     return t;
 }
 
-template <int MODE, typename TO, bool GATHER>
+template <int MODE, typename TO>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p)
 {
@@ -338,44 +321,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int nkb_total = p.nkb * p.nterms;
 
     if (warp == 0) {
-        // -------------------------------------------------------- TMA producer warp
-        // Lane 0 waits for a free stage, arms its barrier and loads B (and A when
-        // not gathering); with GATHER every lane then loads four A rows of the
-        // 128-row tile with one tile::gather4 (lane i: rows 4i .. 4i+3).
-        int it = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-            const Tile t = decode(p, s_tile_off, s_offsets, tile);
-            int ridx[4] = {0, 0, 0, 0};
-            if (GATHER) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    int64_t lr = t.row0 + 4 * lane + j;
-                    if (lr > p.gather_last) lr = p.gather_last;
-                    ridx[j] = __ldg(p.a_gather + lr);
-                }
-            }
-            for (int kb = 0; kb < nkb_total; ++kb, ++it) {
-                const int s = it % STAGES;
-                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
-                const uint32_t sa = sbase + (uint32_t)s * STAGE_BYTES;
-                int good = 1;
-                if (lane == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------- TMA producer
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const Tile t = decode(p, s_tile_off, s_offsets, tile);
+                for (int kb = 0; kb < nkb_total; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
                         atomicOr(p.status, ST_PRODUCER);
                         *(volatile int *)abort_flag = 1;
-                        good = 0;
-                    } else {
-                        mbar_expect_tx(full_bar(s), STAGE_BYTES);
-                        tma_load_2d(sa + A_BYTES, &tmB, full_bar(s), kk, (int)(t.brow + term * p.term_rows));
-                        if (!GATHER) tma_load_2d(sa, &tmA, full_bar(s), kk, (int)t.row0);
+                        ok = false;
+                        break;
                     }
+                    const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
+                    const uint32_t sa = sbase + (uint32_t)s * STAGE_BYTES;
+                    mbar_expect_tx(full_bar(s), STAGE_BYTES);
+                    tma_load_2d(sa, &tmA, full_bar(s), kk, (int)t.row0);
+                    tma_load_2d(sa + A_BYTES, &tmB, full_bar(s), kk, (int)(t.brow + term * p.term_rows));
+                    drain_counts[0] = it + 1;
                 }
-                good = __shfl_sync(0xffffffffu, good, 0);
-                if (!good) { ok = false; break; }
-                if (GATHER) tma_gather4(sa + 512u * lane, &tmA, full_bar(s), kk, ridx);
-                if (lane == 0) drain_counts[0] = it + 1;
             }
         }
     } else if (warp == 1) {
@@ -525,10 +492,10 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
 template <int MODE, typename TO>
 cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const TcParams &p, int grid, cudaStream_t s)
 {
-    auto kern = p.a_gather ? tc_gemm_kernel<MODE, TO, true> : tc_gemm_kernel<MODE, TO, false>;
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    const cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    kern<<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
+    tc_gemm_kernel<MODE, TO><<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
     return cudaGetLastError();
 }
 
@@ -555,13 +522,9 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.epi = g.epi;
     p.status = status;
     if (p.max_tiles == 0) return cudaSuccess;
-    p.a_gather = g.a_gather;
-    p.gather_last = (int64_t)g.M - 1;
-    const int64_t a_rows = g.a_gather ? g.a_rows : g.M;   // grouped: M = total slot rows
+    const int64_t a_rows = g.M;   // grouped: M = total slot rows
     CUtensorMap ta, tb;
-    // gather: box one row high, four rows per tile::gather4
-    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)a_rows, (uint64_t)g.lda * 2, g.a_gather ? 1 : BM))
-        return cudaErrorInvalidValue;
+    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)a_rows, (uint64_t)g.lda * 2, BM)) return cudaErrorInvalidValue;
     if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN))
         return cudaErrorInvalidValue;
     const int grid = p.max_tiles < g_num_sms ? p.max_tiles : g_num_sms;

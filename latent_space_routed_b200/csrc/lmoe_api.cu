@@ -8,12 +8,12 @@
 //   3 scan             counts, offsets, per-block bases, m-tile prefix
 //   4 dispatch         slot_of[t, j], token and weight of every slot row
 //   5 down GEMM        z = x W_down^T                           [T, l]
-//   6 gate/up GEMM     per expert: h = act(G z, U z), the A rows gathered
-//                      from z through the slot -> token map      [S, f]
-//   7 down GEMM        per expert: Y = p * (h D^T)              [S, l] fp32
-//   8 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
-//   9 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
-//  10 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
+//   6 permute          Zp[m] = z[token of slot m]               [S, l]
+//   7 gate/up GEMM     per expert: h = act(G z, U z)            [S, f]
+//   8 down GEMM        per expert: Y = p * (h D^T)              [S, l] fp32
+//   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
+//  10 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
+//  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -51,7 +51,7 @@ lmoe_status fail(lmoe_status s, const char *fmt, ...)
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-    size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, Zp, H, Yp, HS, status;
+    size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, status;
     size_t total;
 };
 
@@ -95,7 +95,8 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.slot_of = take(sizeof(int32_t) * S);
     L.perm_tok = take(sizeof(int32_t) * S);
     L.perm_w = take(sizeof(float) * S);
-    L.Zp = take(h->tb * T * c.l);
+    L.z = take(h->tb * T * c.l);
+    L.Zp = take(h->tb * S * c.l);
     L.H = take(h->tb * S * c.f);
     L.Yp = take(sizeof(float) * S * c.l);
     L.HS = take(h->tb * T * (2 * (int64_t)c.f_shared + c.l));
@@ -261,7 +262,7 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 3: *offset = L.offsets; *bytes = sizeof(int32_t) * (c.E + 1); break;
     case 4: *offset = L.slot_of; *bytes = sizeof(int32_t) * S; break;
     case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
-    case 6: *offset = L.Zp; *bytes = h->tb * T * c.l; break;
+    case 6: *offset = L.z; *bytes = h->tb * T * c.l; break;
     case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
     case 8: *offset = L.Yp; *bytes = sizeof(float) * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
@@ -286,9 +287,9 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
 {
     g_err.clear();
     if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
-    // status reset, router, histogram reset, top-k, scan, dispatch, down, gate/up, down+combine, norm,
-    // shared, final
-    *launches = T == 0 ? 0 : 12;
+    // status reset, router, histogram reset, top-k, scan, dispatch, down, permute, gate/up,
+    // down+combine, norm, shared, final
+    *launches = T == 0 ? 0 : 13;
     return LMOE_OK;
 }
 
@@ -330,7 +331,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     int32_t *slot_of = (int32_t *)(ws + L.slot_of);
     int32_t *perm_tok = (int32_t *)(ws + L.perm_tok);
     float *perm_w = (float *)(ws + L.perm_w);
-    void *Zp = ws + L.Zp, *H = ws + L.H, *HS = ws + L.HS;
+    void *z = ws + L.z, *Zp = ws + L.Zp, *H = ws + L.H, *HS = ws + L.HS;
     float *Yp = (float *)(ws + L.Yp);
     int32_t *status = (int32_t *)(ws + L.status);
 
@@ -368,10 +369,10 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     // 5 z = x W_down^T, once per token
     GemmArgs gd = {};
     gd.A = x; gd.lda = c.d; gd.B = h->Wdown; gd.ldb = c.d; gd.M = (int)T; gd.N = c.l; gd.K = c.d;
-    gd.epi.out = Zp; gd.epi.ldo = c.l;
-    // 6 per expert h = act(G z, U z); slot row m reads z[perm_tok[m]]
+    gd.epi.out = z; gd.epi.ldo = c.l;
+    // 6 per expert h = act(G z, U z) on the slot rows Zp[m] = z[perm_tok[m]]
     GemmArgs gu = {};
-    gu.A = Zp; gu.lda = c.l; gu.a_gather = perm_tok; gu.a_rows = T; gu.B = h->Wgu; gu.ldb = c.l; gu.b_group_stride = 2 * (int64_t)c.f * c.l;
+    gu.A = Zp; gu.lda = c.l; gu.B = h->Wgu; gu.ldb = c.l; gu.b_group_stride = 2 * (int64_t)c.f * c.l;
     gu.M = (int)S; gu.N = 2 * c.f; gu.K = c.l; gu.offsets = offsets; gu.tile_off = tile_off; gu.E = c.E;
     gu.epi.out = H; gu.epi.ldo = c.f; gu.epi.act = c.act; gu.epi.gate_cap = c.gate_cap; gu.epi.up_cap = c.up_cap;
     gu.epi.ib = h->ib;
@@ -394,19 +395,21 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gd, 0, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, s));
     STAGE(5);
+    LMOE_CUDA(launch_permute_rows(z, perm_tok, Zp, S, c.l, (int)h->tb, s));
+    STAGE(6);
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, s));
-    STAGE(6);
+    STAGE(7);
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, 0, gc, max_mtiles, s));
     // 8 u, RMSNorm(u) into the columns after the shared hidden
-    STAGE(7);
+    STAGE(8);
     LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
                                   2 * (int64_t)c.f_shared, tk, s));
-    STAGE(8);
+    STAGE(9);
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gs, 0, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, s));
-    STAGE(9);
+    STAGE(10);
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gf, 0, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, s));
     STAGE(LMOE_NUM_STAGES);

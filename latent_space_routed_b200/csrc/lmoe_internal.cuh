@@ -33,8 +33,8 @@ __device__ __forceinline__ float glu_act(int act, float g, float v, float cg, fl
 // ---------------------------------------------------------------- epilogues
 // Every GEMM here computes C[m, n] = sum_k A[m, k] B[n, k] (both K-major) and
 // hands each row chunk of fp32 accumulators to one of these epilogues.
-// (Mode 2 is unused: the down-projection stores z once and the routed GEMM
-// gathers its rows.)
+// (Mode 2 is unused: the down-projection stores z once and a permute kernel
+// copies it to the slot rows.)
 enum EpiMode {
     EPI_STORE = 0,    // out[m, n] = C                      (final GEMM -> y)
     EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
@@ -83,8 +83,6 @@ struct GemmArgs {
     const int32_t *offsets;   // grouped: [E+1] row offsets, else nullptr
     const int32_t *tile_off;  // grouped: [E+1] m-tile prefix for this kernel's BM
     int E;
-    const int32_t *a_gather;  // optional: logical row m reads A row a_gather[m] (m < M)
-    int64_t a_rows;           // physical rows of A (a_gather set), for bounds and the TMA map
     EpiArgs epi;
 };
 
@@ -103,6 +101,8 @@ cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int bm, int32_t
                         int32_t *base, int32_t *tile_off, cudaStream_t s);
 cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, int64_t T, int E, int k,
                             int32_t *slot_of, int32_t *perm_tok, float *perm_w, cudaStream_t s);
+cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
+                                cudaStream_t s);
 cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s);
 

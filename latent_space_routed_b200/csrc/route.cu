@@ -150,7 +150,30 @@ dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, 
     }
 }
 
+// Zp[m, :] = z[perm_tok[m], :]: one warp per slot row, 16-byte vectors.
+__global__ void __launch_bounds__(256)
+permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ perm_tok, uint4 *__restrict__ Zp,
+                    int64_t S, int vec_per_row)
+{
+    const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (m >= S) return;
+    const int lane = threadIdx.x & 31;
+    const uint4 *src = z + (int64_t)perm_tok[m] * vec_per_row;
+    uint4 *dst = Zp + m * vec_per_row;
+    for (int i = lane; i < vec_per_row; i += 32) dst[i] = src[i];
+}
+
 }  // namespace
+
+cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
+                                cudaStream_t s)
+{
+    if (S == 0) return cudaSuccess;
+    if (((int64_t)l * elem_bytes) % 16) return cudaErrorInvalidValue;
+    const int vpr = (int)((int64_t)l * elem_bytes / 16);
+    permute_rows_kernel<<<(unsigned)((S + 7) / 8), 256, 0, s>>>((const uint4 *)z, perm_tok, (uint4 *)Zp, S, vpr);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
                         void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
