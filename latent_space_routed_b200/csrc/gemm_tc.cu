@@ -2,32 +2,45 @@
 // -> TMEM -> fused epilogue.
 //
 // C[m, n] = sum_k A[m, k] B[n, k], A and B bf16 and K-major (the "out x in"
-// weights of the layer), fp32 accumulation in tensor memory.
+// weights of the layer), fp32 accumulation in tensor memory.  Output tiles are
+// (128 CG) x 256 with K steps of 64:
 //
-// CTA = 6 warps, one CTA per SM, tiles of 128 x 256 x 64:
-//   warp 0      TMA producer: one thread streams A (128 x 64) and B (256 x 64)
-//               tiles into a 4-stage ring (SWIZZLE_128B), completing the
-//               stage's "full" mbarrier by transaction bytes;
-//   warp 1      TMEM owner and MMA issuer: one thread issues four
-//               tcgen05.mma (M=128, N=256, K=16) per stage into one of two
-//               256-column fp32 accumulators and commits the stage's "empty"
-//               barrier, then the accumulator's "full" barrier per tile;
-//   warps 2-5   epilogue: each warp owns one 32-lane quarter of TMEM (= 32
-//               rows), reads 32-column chunks with tcgen05.ld and applies the
-//               fused epilogue, then frees the accumulator, so the epilogue of
+//   CG = 1  one CTA per tile, tcgen05.mma.cta_group::1 with M = 128, N = 256;
+//   CG = 2  a cluster of two CTAs per tile, tcgen05.mma.cta_group::2 with
+//           M = 256, N = 256: CTA r holds A rows 128 r .. 128 r + 127 and B rows
+//           (output columns) 128 r .. 128 r + 127 of every k-step, the even
+//           ("leader") CTA issues the MMAs for both, and each CTA's tensor memory
+//           receives its own 128 accumulator rows.  Each SM then moves and reads
+//           32 KB of operands per k-step instead of 48 KB for the same work per
+//           SM; with 48 KB the shared-memory traffic of TMA writes plus MMA reads
+//           holds the MMA at about half its rate.
+//
+// Warp roles in each CTA (10 warps):
+//   warp 0      TMA producer (one thread): streams its A and B shares into a
+//               STAGES-deep ring (SWIZZLE_128B) and signals the leader CTA's
+//               "full" barrier of the stage (transaction bytes);
+//   warp 1      TMEM owner; in the leader CTA one thread issues the MMAs into one
+//               of two 256-column fp32 accumulators, commits each stage's "empty"
+//               barrier (in both CTAs) once its MMAs have read it, then the
+//               accumulator's "full" barrier (in both CTAs) per tile;
+//   warps 2-9   epilogue: two warps per 32-lane TMEM quarter read 32-column
+//               chunks with tcgen05.ld, apply the fused epilogue, and arrive on
+//               the leader's accumulator "empty" barrier, so the epilogue of
 //               tile i overlaps the main loop of tile i+1.
-// Tiles are handed out round-robin over a grid of min(SMs, tiles) CTAs, with
-// the n-tile index fastest so that CTAs running together share the A tile.
+// Tiles are handed out round-robin over min(SMs / CG, tiles) CTA groups, with
+// the n-tile index fastest so that groups running together share the A tile.
 //
 // Grouped mode: m-tile i of the expert-sorted slot rows belongs to the expert
-// e with tile_off[e] <= i < tile_off[e+1]; rows past offsets[e+1] are computed
-// on whatever the TMA brought in (the next expert's rows, or zero fill past the
-// end) and discarded by the epilogue.
+// e with tile_off[e] <= i < tile_off[e+1] (tile_off built for 128 CG rows);
+// rows past offsets[e+1] are computed on whatever the TMA brought in (the next
+// expert's rows, or zero fill past the end) and discarded by the epilogue.
 //
-// Every mbarrier wait is bounded by a cycle-count limit (about 2 s); a wait that gives up
-// ORs a code into the status word, stops its role's loop, and the CTA drains
-// the copies and MMAs it still has in flight (again bounded) before it frees
-// its TMEM and returns.
+// Every mbarrier wait is bounded by a cycle-count limit (about 2 s); a wait
+// that gives up ORs a code into the status word, stops its role's loop, and the
+// CTA drains what it still has in flight (again bounded) before it frees its
+// TMEM and returns.
+#include <cstring>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -36,15 +49,28 @@
 namespace lmoe {
 namespace {
 
-constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BN = TC_BN, BK = TC_BK;
 constexpr int THREADS = 320;   // 2 role warps + 8 epilogue warps
 constexpr int TMEM_COLS = 2 * BN;
 constexpr long long WAIT_LIMIT_CYCLES = 4000000000ll;   // about 2 s at 2 GHz
 constexpr int MAX_E = 1024;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + 2 * sizeof(int) * (MAX_E + 1);
+// Epilogue staging: one 32 x 32 output chunk (fp32 at most: 4 KB) per epilogue
+// warp, written swizzled and stored to global memory by TMA.
+constexpr int EPI_CHUNK_BYTES = 32 * 32 * 4;
+constexpr int EPI_STAGING = 8 * EPI_CHUNK_BYTES;
+
+template <int CG> struct Cfg {
+    static constexpr int A_BYTES = 128 * BK * 2;                // this CTA's 128 A rows
+    static constexpr int B_BYTES = (BN / CG) * BK * 2;          // this CTA's share of B rows
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = CG == 2 ? 5 : 3;
+    static constexpr int TILE_M = 128 * CG;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_STAGING + 256 +
+                                   2 * sizeof(int) * (MAX_E + 1);
+    // kind::f16, D fp32, A and B bf16, both K-major, M = 128 CG, N = BN
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                      ((uint32_t)(TILE_M >> 4) << 24);
+};
 
 // status codes (OR-ed together)
 constexpr int ST_PRODUCER = 0x1, ST_MMA = 0x2, ST_EPILOGUE = 0x4, ST_DRAIN = 0x8;
@@ -62,11 +88,33 @@ struct TcParams {
     int E;
     int max_tiles;              // dense: exact tile count
     EpiArgs epi;
+    int out_cols;               // columns of the output tensor map
+    int tma_store;              // 1: full chunks leave through TMA stores
     int32_t *status;
 };
 
 // ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
 {
@@ -78,9 +126,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+// Arrive on a barrier given by its shared::cluster address (own CTA or peer).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
@@ -88,7 +137,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -97,8 +146,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Wait for the phase with the given parity to complete; false after the limit.
-// The limit is counted on the SM's own cycle counter (cheap to read, unlike
-// the global nanosecond timer, which is a long-latency read).
+// The limit is counted on the SM's own cycle counter (cheap to read).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity)) return true;
@@ -109,12 +157,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
     }
 }
 
+// 2D tile load into this CTA's shared memory; completion bytes go to `bar`,
+// a shared::cluster address that is the leader CTA's barrier when CG = 2.
+template <int CG>
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
-        : "memory");
+    if (CG == 2)
+        asm volatile(
+            "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4}], [%2];"
+            ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4}], [%2];"
+            ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
+            : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map)
@@ -130,23 +189,80 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major, M x N.
-constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                           ((uint32_t)(BM >> 4) << 24);
-
+template <int CG>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate));
+    if (CG == 2)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Cfg<CG>::IDESC), "r"(accumulate));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Cfg<CG>::IDESC), "r"(accumulate));
 }
 
+// Arrive on `bar` (the same offset in every CTA of the group) once all MMAs
+// issued so far by this thread have completed.
+template <int CG>
 __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+    if (CG == 2)
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+            ::"r"(bar), "h"((uint16_t)0x3)
+            : "memory");
+    else
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                     : "memory");
+}
+
+// 2D tile store from this CTA's shared memory (bulk group of the calling thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"((uint64_t)map), "r"(src), "r"(c0), "r"(c1)
                  : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Write this lane's 32 outputs as row `lane` of the warp's 32 x 32 staging
+// chunk, in the layout a SWIZZLE_64B (bf16: 64-byte rows) or SWIZZLE_128B
+// (fp32: 128-byte rows) tensor map expects: 16-byte piece c of row r sits at
+// piece c ^ ((r >> 1) & 3), resp. c ^ (r & 7); the pieces of one instruction
+// then fall in distinct banks.
+__device__ __forceinline__ void stage_row(uint32_t buf, int lane, const float *v, bf16 *)
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 pr = __floats2bfloat162_rn(v[c * 8 + 2 * i], v[c * 8 + 2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t *>(&pr);
+        }
+        st_shared_v4(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), w[0], w[1], w[2], w[3]);
+    }
+}
+
+__device__ __forceinline__ void stage_row(uint32_t buf, int lane, const float *v, float *)
+{
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        st_shared_v4(buf + lane * 128 + ((c ^ (lane & 7)) << 4), __float_as_uint(v[4 * c]),
+                     __float_as_uint(v[4 * c + 1]), __float_as_uint(v[4 * c + 2]), __float_as_uint(v[4 * c + 3]));
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -232,13 +348,14 @@ __device__ __forceinline__ void store_n(TO *dst, const float *v, int n)
 
 // ------------------------------------------------------------------ tile decode
 struct Tile {
-    int64_t row0, row_end;  // A rows [row0, row_end) are real for this tile
+    int64_t row0, row_end;  // A rows [row0, row_end) of the whole (128 CG)-row tile are real
     int64_t brow;           // first B row of this tile (term 0)
     int n0;                 // first output column (GEMM n)
 };
 
 // Grouped mode reads the expert row offsets and m-tile prefix from shared
 // memory (staged once per CTA), so decoding a tile costs no global round trip.
+template <int CG>
 __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off, const int *s_offsets, int tile)
 {
     Tile t;
@@ -250,34 +367,41 @@ __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off,
             const int mid = (lo + hi + 1) >> 1;
             if (s_tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
         }
-        t.row0 = (int64_t)s_offsets[lo] + (int64_t)(mt - s_tile_off[lo]) * BM;
+        t.row0 = (int64_t)s_offsets[lo] + (int64_t)(mt - s_tile_off[lo]) * Cfg<CG>::TILE_M;
         t.row_end = s_offsets[lo + 1];
         t.brow = (int64_t)lo * p.group_rows + t.n0;
     } else {
-        t.row0 = (int64_t)mt * BM;
+        t.row0 = (int64_t)mt * Cfg<CG>::TILE_M;
         t.row_end = p.M;
         t.brow = t.n0;
     }
     return t;
 }
 
-template <int MODE, typename TO>
+template <int MODE, typename TO, int CG>
 __global__ void __launch_bounds__(THREADS, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmC, const TcParams p)
 {
+    using C = Cfg<CG>;
+    constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;           // 1024-aligned stage ring
     uint8_t *gbase = smem_raw + (sbase - raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + (size_t)STAGES * STAGE_BYTES);
+    const uint32_t epi_base = sbase + (uint32_t)(STAGES * C::STAGE_BYTES);   // 1024-aligned staging
+    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + (size_t)STAGES * C::STAGE_BYTES + EPI_STAGING);
     // bars[0..S) full, [S..2S) empty, [2S..2S+2) acc full, [2S+2..2S+4) acc empty
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
     int *abort_flag = reinterpret_cast<int *>(tmem_holder + 1);
     int *drain_counts = abort_flag + 1;                      // [0] loads issued, [1] stages consumed
-    int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * STAGE_BYTES + 256);   // [E+1]
-    int *s_offsets = s_tile_off + (MAX_E + 1);                                              // [E+1]
+    int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * C::STAGE_BYTES + EPI_STAGING + 256);
+    int *s_offsets = s_tile_off + (MAX_E + 1);                                                 // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = CG == 2 ? cluster_rank() : 0u;
+    const bool leader = rank == 0;
+    const int group = blockIdx.x / CG, ngroups = gridDim.x / CG;
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -286,12 +410,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
+            mbar_init(full_bar(s), 1);      // the leader's producer arms it for the whole group
+            mbar_init(empty_bar(s), 1);     // one MMA commit
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(accf_bar(a), 1);
-            mbar_init(acce_bar(a), 8);   // one arrival per epilogue warp
+            mbar_init(acce_bar(a), 8 * CG);  // every epilogue warp of the group
         }
         *abort_flag = 0;
         drain_counts[0] = drain_counts[1] = 0;
@@ -307,13 +431,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (CG == 2) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_holder)), "r"(TMEM_COLS) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_holder)), "r"(TMEM_COLS) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();     // peer barriers initialised before any remote signal
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
@@ -325,8 +455,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // ---------------------------------------------------- TMA producer
             int it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-                const Tile t = decode(p, s_tile_off, s_offsets, tile);
+            for (int tile = group; tile < total && ok; tile += ngroups) {
+                const Tile t = decode<CG>(p, s_tile_off, s_offsets, tile);
                 for (int kb = 0; kb < nkb_total; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -337,20 +467,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         break;
                     }
                     const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
-                    const uint32_t sa = sbase + (uint32_t)s * STAGE_BYTES;
-                    mbar_expect_tx(full_bar(s), STAGE_BYTES);
-                    tma_load_2d(sa, &tmA, full_bar(s), kk, (int)t.row0);
-                    tma_load_2d(sa + A_BYTES, &tmB, full_bar(s), kk, (int)(t.brow + term * p.term_rows));
+                    const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
+                    const uint32_t fb = CG == 2 ? map_to_rank(full_bar(s), 0) : full_bar(s);
+                    if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
+                    tma_load_2d<CG>(sa, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
+                    tma_load_2d<CG>(sa + C::A_BYTES, &tmB, fb, kk,
+                                    (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
                     drain_counts[0] = it + 1;
                 }
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------------------------------------------- MMA issuer
+        if (lane == 0 && leader) {
+            // ---------------------------------------------------- MMA issuer (leader CTA)
             int it = 0, local = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+            for (int tile = group; tile < total && ok; tile += ngroups, ++local) {
                 const int acc = local & 1;
                 const uint32_t aph = (uint32_t)(local >> 1) & 1u;
                 if (!mbar_wait(acce_bar(acc), aph ^ 1u)) {
@@ -370,17 +502,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sa = sbase + (uint32_t)s * STAGE_BYTES;
+                    const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint64_t ad = sdesc_sw128(sa + 32u * k);
-                        const uint64_t bd = sdesc_sw128(sa + A_BYTES + 32u * k);
-                        umma_bf16(dt, ad, bd, (kb > 0 || k > 0) ? 1u : 0u);
+                        const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + 32u * k);
+                        umma_bf16<CG>(dt, ad, bd, (kb > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit(empty_bar(s));
+                    umma_commit<CG>(empty_bar(s));
                     drain_counts[1] = it + 1;
                 }
-                if (ok) umma_commit(accf_bar(acc));
+                if (ok) umma_commit<CG>(accf_bar(acc));
             }
         }
     } else {
@@ -389,8 +521,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // chunks c = 32 h + 64 i, so each warp drains half of its 32 rows' tile.
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
+        const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * EPI_CHUNK_BYTES;
         int local = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+        for (int tile = group; tile < total; tile += ngroups, ++local) {
             const int acc = local & 1;
             const uint32_t aph = (uint32_t)(local >> 1) & 1u;
             const bool got = mbar_wait(accf_bar(acc), aph);
@@ -402,11 +535,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const Tile t = decode(p, s_tile_off, s_offsets, tile);
-            const int64_t row = t.row0 + 32 * q + lane;
+            const Tile t = decode<CG>(p, s_tile_off, s_offsets, tile);
+            const int64_t row = t.row0 + 128 * rank + 32 * q + lane;
             const bool valid = row < t.row_end;
             const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
             float v[32], u[32];
+            // Emit 32 output columns [col, col + n) of this warp's 32 rows: whole
+            // chunks go through the staging buffer and one TMA store; chunks that
+            // straddle an expert's last row (or a ragged column edge) store per lane.
+            const int64_t chunk_row = t.row0 + 128 * rank + 32 * q;
+            const bool rows_ok = p.offsets ? (chunk_row + 32 <= t.row_end) : true;
+            auto emit = [&](const float *x, int col, int n) {
+                if (p.tma_store && rows_ok && n == 32) {
+                    if (lane == 0) bulk_wait_read_all();     // the previous store has read the buffer
+                    __syncwarp();
+                    stage_row(ebuf, lane, x, (TO *)nullptr);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&tmC, ebuf, col, (int)chunk_row);
+                } else if (valid) {
+                    store_n((TO *)p.epi.out + row * p.epi.ldo + col, x, n);
+                }
+            };
             if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
                 const int half = BN / 2;
 #pragma unroll 1
@@ -416,7 +566,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
                                                                                        p.epi.up_cap);
-                    if (valid) store_n((TO *)p.epi.out + row * p.epi.ldo + t.n0 / 2 + c, v, 32);
+                    emit(v, t.n0 / 2 + c, 32);
                 }
             } else {
 #pragma unroll 1
@@ -429,31 +579,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         const int col = t.n0 + c + 64 * part;
                         int n = p.N - col;
                         if (n > 32) n = 32;
-                        if (!valid || n <= 0) {
-                            // nothing to store for this lane
-                        } else if (MODE == EPI_SIGMOID) {
+                        if (n <= 0) continue;             // uniform across the warp
+                        if (MODE == EPI_SIGMOID) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
-                            store_n((float *)p.epi.out + row * p.epi.ldo + col, x, n);
                         } else if (MODE == EPI_COMBINE) {
-                            const float w = p.epi.row_w[row];
+                            const float w = valid ? p.epi.row_w[row] : 0.f;
 #pragma unroll
                             for (int i = 0; i < 32; ++i) x[i] *= w;
-                            store_n((float *)p.epi.out + row * p.epi.ldo + col, x, n);
-                        } else {
-                            store_n((TO *)p.epi.out + row * p.epi.ldo + col, x, n);
                         }
+                        emit(x, col, n);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce_bar(acc));
+            if (lane == 0) mbar_arrive_cluster(CG == 2 ? map_to_rank(acce_bar(acc), 0) : acce_bar(acc));
         }
+        if (lane == 0) bulk_wait_all();             // this warp's TMA stores are complete
     }
 
     __syncthreads();
-    if (*(volatile int *)abort_flag && threadIdx.x == 0) {
+    if (*(volatile int *)abort_flag && threadIdx.x == 0 && leader) {
         // Drain: loads issued but never consumed, then the MMAs behind the last commit.
         const int issued = drain_counts[0], consumed = drain_counts[1];
         bool ok = true;
@@ -465,17 +612,38 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         if (!ok) atomicOr(p.status, ST_DRAIN);
     }
+    tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();     // no CTA leaves while its peer may still touch its memory
     tc_fence_after();
     if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
-                     : "memory");
+        if (CG == 2)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                         : "memory");
     }
 }
 
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 int g_num_sms = 0;
+
+// Output map: 32 x 32 boxes, swizzled to match stage_row.
+bool make_out_map(CUtensorMap *m, void *base, bool f32, uint64_t cols, uint64_t rows, uint64_t row_bytes)
+{
+    if (((uintptr_t)base & 15u) || (row_bytes & 15u)) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_outer)
 {
@@ -489,16 +657,47 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
     return r == CUDA_SUCCESS;
 }
 
-template <int MODE, typename TO>
-cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const TcParams &p, int grid, cudaStream_t s)
+// Persistent grid: min(tiles, CTA groups that can be resident at once).
+template <int MODE, typename TO, int CG>
+cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const TcParams &p, cudaStream_t s)
 {
-    const cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<MODE, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)SMEM_BYTES);
+    auto kern = tc_gemm_kernel<MODE, TO, CG>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG>::SMEM);
     if (e != cudaSuccess) return e;
-    tc_gemm_kernel<MODE, TO><<<grid, THREADS, SMEM_BYTES, s>>>(a, b, p);
-    return cudaGetLastError();
+    int max_groups = g_num_sms / CG;
+    if (CG > 1) {
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(g_num_sms / CG * CG);
+        q.blockDim = dim3(THREADS);
+        q.dynamicSmemBytes = Cfg<CG>::SMEM;
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = CG;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        q.attrs = qa;
+        q.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess && n > 0 && n < max_groups) max_groups = n;
+        cudaGetLastError();
+    }
+    const int groups = p.max_tiles < max_groups ? p.max_tiles : max_groups;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(groups * CG);
+    lc.blockDim = dim3(THREADS);
+    lc.dynamicSmemBytes = Cfg<CG>::SMEM;
+    lc.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, a, b, c, p);
 }
 
+template <int CG>
 cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t term_rows, int64_t b_rows_total,
                 int32_t *status, cudaStream_t s)
 {
@@ -506,35 +705,40 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     if (g.K % BK) return cudaErrorInvalidValue;
     if (((uintptr_t)g.A | (uintptr_t)g.B) & 15u) return cudaErrorMisalignedAddress;
     if ((g.lda * 2) % 16 || (g.ldb * 2) % 16) return cudaErrorMisalignedAddress;
+    if (g.offsets && g.E > MAX_E) return cudaErrorInvalidValue;
     TcParams p = {};
     p.M = g.M;
     p.N = g.N;
     p.nkb = g.K / BK;
     p.nterms = nterms;
     p.term_rows = term_rows;
-    p.ntn = mode == EPI_GLU ? g.N / BN : (g.N + BN - 1) / BN;   // GLU: N = 2F, F % (BN/2) == 0
+    p.ntn = (mode == EPI_GLU) ? g.N / BN : (g.N + BN - 1) / BN;   // GLU: N = 2F, F % (BN/2) == 0
     p.group_rows = g.offsets ? g.b_group_stride / g.ldb : 0;
     p.offsets = g.offsets;
     p.tile_off = g.tile_off;
     p.E = g.E;
-    const int mtiles = g.offsets ? max_mtiles : (g.M + BM - 1) / BM;
+    const int mtiles = g.offsets ? max_mtiles : (g.M + Cfg<CG>::TILE_M - 1) / Cfg<CG>::TILE_M;
     p.max_tiles = mtiles * p.ntn;
     p.epi = g.epi;
     p.status = status;
     if (p.max_tiles == 0) return cudaSuccess;
-    const int64_t a_rows = g.M;   // grouped: M = total slot rows
     CUtensorMap ta, tb;
-    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)a_rows, (uint64_t)g.lda * 2, BM)) return cudaErrorInvalidValue;
-    if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN))
+    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG))
         return cudaErrorInvalidValue;
-    const int grid = p.max_tiles < g_num_sms ? p.max_tiles : g_num_sms;
+    const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_COMBINE);
+    p.out_cols = (mode == EPI_GLU) ? g.N / 2 : g.N;
+    CUtensorMap tc;
+    memset(&tc, 0, sizeof tc);
+    p.tma_store = make_out_map(&tc, g.epi.out, out_f32, (uint64_t)p.out_cols, (uint64_t)g.M,
+                               (uint64_t)g.epi.ldo * (out_f32 ? 4 : 2)) ? 1 : 0;
     switch (mode) {
-    case EPI_SIGMOID: return launch<EPI_SIGMOID, float>(ta, tb, p, grid, s);
+    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG>(ta, tb, tc, p, s);
     case EPI_GLU:
-        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16>(ta, tb, p, grid, s);
-        return launch<EPI_GLU, bf16>(ta, tb, p, grid, s);
-    case EPI_COMBINE: return launch<EPI_COMBINE, float>(ta, tb, p, grid, s);
-    case EPI_STORE: return launch<EPI_STORE, bf16>(ta, tb, p, grid, s);
+        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG>(ta, tb, tc, p, s);
+        return launch<EPI_GLU, bf16, CG>(ta, tb, tc, p, s);
+    case EPI_COMBINE: return launch<EPI_COMBINE, float, CG>(ta, tb, tc, p, s);
+    case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tb, tc, p, s);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -560,11 +764,12 @@ lmoe_status tc_check_device()
     return LMOE_OK;
 }
 
-cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int32_t *status, cudaStream_t s)
+cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t *status, cudaStream_t s)
 {
     // B rows: dense N; grouped E * (rows per expert)
     const int64_t b_rows = g.offsets ? (int64_t)g.E * (g.b_group_stride / g.ldb) : g.N;
-    return run(mode, g, max_mtiles, 1, 0, b_rows, status, s);
+    if (cg == 2) return run<2>(mode, g, max_mtiles, 1, 0, b_rows, status, s);
+    return run<1>(mode, g, max_mtiles, 1, 0, b_rows, status, s);
 }
 
 cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s)
@@ -572,7 +777,7 @@ cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, 
     GemmArgs r = g;
     r.B = Wr3;
     r.ldb = g.K;
-    return run(EPI_SIGMOID, r, 0, 3, g.N, 3 * (int64_t)g.N, status, s);
+    return run<1>(EPI_SIGMOID, r, 0, 3, g.N, 3 * (int64_t)g.N, status, s);
 }
 
 }  // namespace lmoe

@@ -9,11 +9,13 @@ namespace lmoe {
 // tensor-map encoder; LMOE_ERR_UNSUPPORTED otherwise.
 lmoe_status tc_check_device();
 
-// C = A B^T with the epilogue `mode` (EPI_SCATTER, EPI_GLU, EPI_COMBINE,
-// EPI_STORE), A and B bf16 K-major, K a multiple of 64, rows 16-byte aligned.
-// Grouped when g.offsets != nullptr (max_mtiles bounds the m-tiles of all
-// experts).  Bounded waits that give up OR a code into *status.
-cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int32_t *status, cudaStream_t s);
+// C = A B^T with the epilogue `mode` (EPI_GLU, EPI_COMBINE, EPI_STORE), A and
+// B bf16 K-major, K a multiple of 64, rows 16-byte aligned.  cg = 1: 128 x 256
+// tiles on one CTA; cg = 2: 256 x 256 tiles on a two-CTA cluster.  Grouped when
+// g.offsets != nullptr (tile_off built for 128 cg rows per m-tile; max_mtiles
+// bounds the m-tiles of all experts).  Bounded waits that give up OR a code
+// into *status.
+cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t *status, cudaStream_t s);
 
 // Router r = sigmoid(x W_r^T) from the three-term bf16 split of fp32 W_r
 // (Wr3 = [3, E, d]): the three products accumulate into one fp32 TMEM tile.

@@ -62,7 +62,6 @@ struct lmoe_handle {
     int device;
     bool tc;          // tensor-core GEMMs
     int ib;           // gate/up interleave block
-    int bm;           // m-tile of the grouped GEMMs
     size_t tb;        // token dtype bytes
     float *Wr;        // [E, d] fp32 (CUDA-core router)
     bf16 *Wr3;        // [3, E, d] bf16 split (tensor-core router)
@@ -187,7 +186,6 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
     cudaGetDevice(&h->device);
     h->tc = tc;
     h->ib = tc ? TC_BN / 2 : SIMT_BN / 2;
-    h->bm = tc ? TC_BM : SIMT_BM;
     h->tb = cfg->dtype == LMOE_BF16 ? 2 : 4;
     const lmoe_config &c = *cfg;
     const size_t tb = h->tb;
@@ -339,7 +337,12 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
     const int tk = c.dtype == LMOE_BF16 ? 1 : 0;
     const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
-    const int max_mtiles = (int)((S + h->bm - 1) / h->bm + c.E);
+    // Tensor-core tiles: 256-row tiles on CTA pairs where rows are plentiful
+    // (grouped: at least ~192 slot rows per expert on average), else 128.
+    const int cg_grouped = (h->tc && S >= 192LL * c.E) ? 2 : 1;
+    const int cg_dense = (h->tc && T >= 256) ? 2 : 1;
+    const int bm = h->tc ? TC_BM * cg_grouped : SIMT_BM;
+    const int max_mtiles = (int)((S + bm - 1) / bm + c.E);
 
     LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
 #define STAGE(i)                                                                                 \
@@ -362,7 +365,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     STAGE(1);
     LMOE_CUDA(launch_topk(r32, h->b, T, c.E, c.k, selected_experts, p32, mixture_weights, tk, blockhist, s));
     STAGE(2);
-    LMOE_CUDA(launch_scan(blockhist, nb, c.E, h->bm, counts, offsets, base, tile_off, s));
+    LMOE_CUDA(launch_scan(blockhist, nb, c.E, bm, counts, offsets, base, tile_off, s));
     STAGE(3);
     LMOE_CUDA(launch_dispatch(selected_experts, p32, base, T, c.E, c.k, slot_of, perm_tok, perm_w, s));
 
@@ -392,25 +395,25 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     gf.epi.out = output; gf.epi.ldo = c.d;
 
     STAGE(4);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gd, 0, status, s));
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gd, 0, cg_dense, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, s));
     STAGE(5);
     LMOE_CUDA(launch_permute_rows(z, perm_tok, Zp, S, c.l, (int)h->tb, s));
     STAGE(6);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, status, s));
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, cg_grouped, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, s));
     STAGE(7);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, status, s));
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, cg_grouped, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, 0, gc, max_mtiles, s));
     // 8 u, RMSNorm(u) into the columns after the shared hidden
     STAGE(8);
     LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
                                   2 * (int64_t)c.f_shared, tk, s));
     STAGE(9);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gs, 0, status, s));
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gs, 0, cg_dense, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, s));
     STAGE(10);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gf, 0, status, s));
+    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gf, 0, cg_dense, status, s));
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, s));
     STAGE(LMOE_NUM_STAGES);
 #undef STAGE
