@@ -204,6 +204,31 @@ LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int3
  * invalid).  `workspace` is the one passed to lmoe_forward. */
 LMOE_API lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream);
 
+/* Size of the scratch area built into the library for lmoe_forward_noalloc. */
+#define LMOE_NOALLOC_WORKSPACE_BYTES ((size_t)64 << 20)
+
+/* lmoe_forward without a caller workspace, for callers that cannot allocate
+ * device memory where they run the layer (inside a stream capture that must
+ * not allocate, under an allocator owned by another runtime, or on a path
+ * that must not take allocator locks).  There is no counterpart in the
+ * LatentMoE pages: this is a deployment convenience of this library.
+ * Arguments and outputs are those of lmoe_forward minus the workspace; the
+ * scratch is a fixed 64 MiB device array inside the library
+ * (LMOE_NOALLOC_WORKSPACE_BYTES), which every GPU that loads the library holds
+ * until the process exits.  Nothing is allocated by the call.
+ *  - If lmoe_workspace_size(h, T) exceeds the area, it returns
+ *    LMOE_ERR_WORKSPACE and launches nothing (the area covers, for example,
+ *    about 128 tokens of a d = 7168, l = 1792, k = 32 layer).
+ *  - The first call on a device looks up the area's device address with that
+ *    device current; make it before any stream capture.
+ *  - All calls on a device share the area and find the previous call's data
+ *    in it (the forward resets what must start at zero itself).  Calls that
+ *    overlap on the GPU race on it: order them on one stream.
+ * Errors as lmoe_forward. */
+LMOE_API lmoe_status lmoe_forward_noalloc(lmoe_handle *h, const void *x, int64_t T, void *output,
+                                          int32_t *selected_experts, void *mixture_weights,
+                                          void *latent_routed_aggregate, void *stream);
+
 /* Message for the last failure on the calling thread ("" if none). */
 LMOE_API const char *lmoe_last_error(void);
 

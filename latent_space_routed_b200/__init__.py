@@ -33,7 +33,7 @@ REGION = {"scores": 0, "p32": 1, "counts": 2, "offsets": 3, "slot_of": 4, "perm_
           "Y": 8, "HS": 9, "status": 10}
 
 EXPORTS = ("lmoe_config_from_base", "lmoe_create", "lmoe_workspace_size", "lmoe_forward", "lmoe_host_workspace_size",
-           "lmoe_forward_host", "lmoe_set_bias", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
+           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_set_bias", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
            "lmoe_last_error", "lmoe_destroy")
 
 
@@ -66,6 +66,7 @@ def _load() -> ctypes.CDLL:
         "lmoe_forward": (I32, [P, P, I64, P, P, P, P, P, SZ, P]),
         "lmoe_host_workspace_size": (I32, [P, I64, ctypes.POINTER(SZ)]),
         "lmoe_forward_host": (I32, [P, P, I64, P, P, P, P, P, SZ, P]),
+        "lmoe_forward_noalloc": (I32, [P, P, I64, P, P, P, P, P]),
         "lmoe_set_bias": (I32, [P, P, P]),
         "lmoe_set_stage_events": (I32, [P, P, I32]),
         "lmoe_launch_count": (I32, [P, I64, ctypes.POINTER(I32)]),
@@ -153,6 +154,16 @@ def lmoe_forward_host(h, x_host, T, output_host, selected_experts_host, mixture_
     _check(_lib.lmoe_forward_host(h, _ptr(x_host), T, _ptr(output_host), _ptr(selected_experts_host),
                                   _ptr(mixture_weights_host), _ptr(latent_routed_aggregate_host), _ptr(workspace),
                                   ws_bytes, _stream(stream)))
+
+
+LMOE_NOALLOC_WORKSPACE_BYTES = 64 << 20
+
+
+def lmoe_forward_noalloc(h, x, T, output, selected_experts, mixture_weights, latent_routed_aggregate, stream=None):
+    """lmoe_forward on the library's built-in 64 MiB scratch area (no caller
+    workspace, no allocation); see include/lmoe.h for its rules."""
+    _check(_lib.lmoe_forward_noalloc(h, _ptr(x), T, _ptr(output), _ptr(selected_experts), _ptr(mixture_weights),
+                                     _ptr(latent_routed_aggregate), _stream(stream)))
 
 
 def lmoe_set_bias(h, b, stream=None):

@@ -57,6 +57,12 @@ struct Layout {
 
 }  // namespace
 
+lmoe_status lmoe::report_error(lmoe_status s, const char *msg)
+{
+    g_err = msg;
+    return s;
+}
+
 struct lmoe_handle {
     lmoe_config cfg;
     int device;

@@ -11,6 +11,9 @@ namespace lmoe {
 
 typedef __nv_bfloat16 bf16;
 
+// Record `msg` as the calling thread's lmoe_last_error() and return `s`.
+lmoe_status report_error(lmoe_status s, const char *msg);
+
 // ---------------------------------------------------------------- conversions
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }

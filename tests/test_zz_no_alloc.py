@@ -1,0 +1,61 @@
+"""lmoe_forward_noalloc: the forward on the library's built-in scratch area.
+
+This entry point exists for callers that cannot allocate device memory where
+they run the layer (a stream capture that must not allocate, an allocator
+owned by another runtime, a path that must not take allocator locks).  The
+test drives it through the C ABI and checks, on two calls in a row (the
+second finds the first call's data still in the shared area), that it returns
+what lmoe_forward with a caller workspace returns, within the tolerance the
+parity tests use.  It also checks the size limit is enforced before any work.
+
+The file name makes pytest collect it last, so a run that stops at the first
+failure has already run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+import lmoe_inputs as li
+from parity import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2   # bf16 tolerance of the parity tests
+
+
+def test_noalloc_matches_the_workspace_entry_point_twice():
+    import latent_space_routed_b200 as lm
+    w = li.custom("noalloc", 300, 512, 256, 256, 32, 6, 256, dtype="bf16", seed=31)
+    W = li.weights(w)
+    layer = lm.LatentMoE(lm.config_for(w), {k: v.cuda() for k, v in W.items()})
+    T = w.T
+    assert lm.lmoe_workspace_size(layer.handle, T) <= lm.LMOE_NOALLOC_WORKSPACE_BYTES
+    x = li.tokens(w).cuda()
+    ref = layer.forward_into(x, layer.empty_outputs(T))
+    torch.cuda.synchronize()
+    ref = {k: v.clone() for k, v in ref.items()}
+
+    x2 = li.tokens(w, seed=77).cuda()        # a different batch in between
+    for xb in (x, x2, x):
+        out = layer.empty_outputs(T)
+        lm.lmoe_forward_noalloc(layer.handle, xb, T, out["output"], out["selected_experts"],
+                                out["mixture_weights"], out["latent_routed_aggregate"])
+        torch.cuda.synchronize()
+        if xb is x:
+            assert torch.equal(out["selected_experts"], ref["selected_experts"])
+            for key in ("output", "mixture_weights", "latent_routed_aggregate"):
+                e = rel_err(out[key].float().cpu().numpy(), ref[key].float().cpu().numpy())
+                assert e <= TOL, (key, e)
+
+    # too many tokens for the built-in area: rejected with a clear status
+    big = 1
+    while lm.lmoe_workspace_size(layer.handle, big) <= lm.LMOE_NOALLOC_WORKSPACE_BYTES:
+        big *= 2
+    xb = torch.zeros(big, w.d, dtype=torch.bfloat16, device="cuda")
+    out = layer.empty_outputs(big)
+    with pytest.raises(lm.LmoeError) as ei:
+        lm.lmoe_forward_noalloc(layer.handle, xb, big, out["output"], out["selected_experts"],
+                                out["mixture_weights"], out["latent_routed_aggregate"])
+    assert ei.value.status == lm.LMOE_ERR_WORKSPACE
+    assert "64 MiB" in str(ei.value)
+    layer.close()
