@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--gemm", type=int, default=0, help="0 tensor cores, 1 CUDA cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--graph", action="store_true", help="also time the forward replayed from a CUDA graph")
     return ap.parse_args()
 
 
@@ -215,6 +216,13 @@ def run_own(args, rank, world, local_rank):
     layer.check_device(T)
     counts = layer.region(T, "counts", torch.int32, (w.E,)).cpu().numpy()
     touched = int((counts > 0).sum())
+    # host cost of one call (enqueue only): tells whether small batches starve the GPU
+    torch.cuda.synchronize()
+    t_h = time.perf_counter()
+    for _ in range(10):
+        layer.forward_into(x, out)
+    host_us = (time.perf_counter() - t_h) / 10 * 1e6
+    torch.cuda.synchronize()
 
     ns = lm.LMOE_NUM_STAGES + 1
     ev_stage = [[torch.cuda.Event(enable_timing=True) for _ in range(ns)] for _ in range(args.steps)]
@@ -258,6 +266,34 @@ def run_own(args, rank, world, local_rank):
     stage_ms = {}
     for si, name in enumerate(lm.STAGE_NAMES):
         stage_ms[name] = sum(ev_stage[i][si].elapsed_time(ev_stage[i][si + 1]) for i in range(args.steps)) / args.steps
+
+    graph_ms = None
+    if args.graph:
+        # the same forward captured once into a CUDA graph and replayed (no host launch gaps)
+        layer.workspace(T)
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            layer.forward_into(x, out, stream=side)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layer.forward_into(x, out, stream=torch.cuda.current_stream())
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        g_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        g_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            g_a[i].record(stream)
+            graph.replay()
+            g_b[i].record(stream)
+        torch.cuda.synchronize()
+        graph_ms = sum(a.elapsed_time(b) for a, b in zip(g_a, g_b)) / args.steps
+        del graph
+        layer.check_device(T)
 
     # end to end through the public API: pinned host x in, host outputs back, copies inside the timing
     x_host = x_cpu.pin_memory()
@@ -331,7 +367,11 @@ def run_own(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "e2e": {"value": world * T / (e2e_ms / args.steps / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": layer.launch_count(T) * args.steps, "clocks": clk}
+            "gpu_launches": layer.launch_count(T) * args.steps, "clocks": clk,
+            "host_us_per_call": host_us}
+    if graph_ms is not None:
+        line["graph"] = {"ms_per_step": graph_ms, "value": world * T / (graph_ms / 1e3), "unit": UNIT,
+                         "layer_frac": t_roof / (graph_ms / 1e3)}
     print(json.dumps(line), flush=True)
     layer.close()
 

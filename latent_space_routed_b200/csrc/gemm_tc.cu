@@ -39,6 +39,7 @@
 // that gives up ORs a code into the status word, stops its role's loop, and the
 // CTA drains what it still has in flight (again bounded) before it frees its
 // TMEM and returns.
+#include <atomic>
 #include <cstring>
 
 #include <cuda.h>
@@ -87,6 +88,8 @@ struct TcParams {
     const int32_t *tile_off;
     int E;
     int max_tiles;              // dense: exact tile count
+    int ksplit;                 // >1: K split into ksplit ranges, partial tiles to row slab `split`
+    int64_t split_rows;         // rows of one partial slab (= M)
     EpiArgs epi;
     int out_cols;               // columns of the output tensor map
     int tma_store;              // 1: full chunks leave through TMA stores
@@ -447,7 +450,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    const int total = p.offsets ? s_tile_off[p.E] * p.ntn : p.max_tiles;
+    const int total = (p.offsets ? s_tile_off[p.E] * p.ntn : p.max_tiles) * p.ksplit;   // work items
     const int nkb_total = p.nkb * p.nterms;
 
     if (warp == 0) {
@@ -455,9 +458,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // ---------------------------------------------------- TMA producer
             int it = 0;
             bool ok = true;
-            for (int tile = group; tile < total && ok; tile += ngroups) {
-                const Tile t = decode<CG>(p, s_tile_off, s_offsets, tile);
-                for (int kb = 0; kb < nkb_total; ++kb, ++it) {
+            for (int item = group; item < total && ok; item += ngroups) {
+                const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
+                const int split = item % p.ksplit;
+                const int kb_end = (split + 1) * nkb_total / p.ksplit;
+                for (int kb = split * nkb_total / p.ksplit; kb < kb_end; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
@@ -482,9 +487,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // ---------------------------------------------------- MMA issuer (leader CTA)
             int it = 0, local = 0;
             bool ok = true;
-            for (int tile = group; tile < total && ok; tile += ngroups, ++local) {
+            for (int item = group; item < total && ok; item += ngroups, ++local) {
                 const int acc = local & 1;
                 const uint32_t aph = (uint32_t)(local >> 1) & 1u;
+                const int split = item % p.ksplit;
+                const int kb_begin = split * nkb_total / p.ksplit, kb_end = (split + 1) * nkb_total / p.ksplit;
                 if (!mbar_wait(acce_bar(acc), aph ^ 1u)) {
                     atomicOr(p.status, ST_MMA);
                     *(volatile int *)abort_flag = 1;
@@ -492,7 +499,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 tc_fence_after();
                 const uint32_t dt = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < nkb_total; ++kb, ++it) {
+                for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     if (!mbar_wait(full_bar(s), ph) || *(volatile int *)abort_flag) {
@@ -507,7 +514,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint64_t ad = sdesc_sw128(sa + 32u * k);
                         const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + 32u * k);
-                        umma_bf16<CG>(dt, ad, bd, (kb > 0 || k > 0) ? 1u : 0u);
+                        umma_bf16<CG>(dt, ad, bd, (kb > kb_begin || k > 0) ? 1u : 0u);
                     }
                     umma_commit<CG>(empty_bar(s));
                     drain_counts[1] = it + 1;
@@ -523,7 +530,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
         const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * EPI_CHUNK_BYTES;
         int local = 0;
-        for (int tile = group; tile < total; tile += ngroups, ++local) {
+        for (int item = group; item < total; item += ngroups, ++local) {
             const int acc = local & 1;
             const uint32_t aph = (uint32_t)(local >> 1) & 1u;
             const bool got = mbar_wait(accf_bar(acc), aph);
@@ -535,7 +542,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const Tile t = decode<CG>(p, s_tile_off, s_offsets, tile);
+            const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
+            const int64_t slab = (int64_t)(item % p.ksplit) * p.split_rows;   // 0 unless split K
             const int64_t row = t.row0 + 128 * rank + 32 * q + lane;
             const bool valid = row < t.row_end;
             const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
@@ -544,7 +552,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // chunks go through the staging buffer and one TMA store; chunks that
             // straddle an expert's last row (or a ragged column edge) store per lane.
             const int64_t chunk_row = t.row0 + 128 * rank + 32 * q;
-            const bool rows_ok = p.offsets ? (chunk_row + 32 <= t.row_end) : true;
+            const bool rows_ok = (p.offsets || p.ksplit > 1) ? (chunk_row + 32 <= t.row_end) : true;
             auto emit = [&](const float *x, int col, int n) {
                 if (p.tma_store && rows_ok && n == 32) {
                     if (lane == 0) bulk_wait_read_all();     // the previous store has read the buffer
@@ -552,9 +560,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     stage_row(ebuf, lane, x, (TO *)nullptr);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) tma_store_2d(&tmC, ebuf, col, (int)chunk_row);
+                    if (lane == 0) tma_store_2d(&tmC, ebuf, col, (int)(slab + chunk_row));
                 } else if (valid) {
-                    store_n((TO *)p.epi.out + row * p.epi.ldo + col, x, n);
+                    store_n((TO *)p.epi.out + (slab + row) * p.epi.ldo + col, x, n);
                 }
             };
             if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
@@ -657,14 +665,25 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
     return r == CUDA_SUCCESS;
 }
 
-// Persistent grid: min(tiles, CTA groups that can be resident at once).
+// Per-device, per-instantiation launch setup (shared-memory opt-in and, for
+// CTA pairs, how many pairs fit at once), done on first use and cached.
+constexpr int MAX_DEVICES = 64;
+
 template <int MODE, typename TO, int CG>
-cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const TcParams &p, cudaStream_t s)
+cudaError_t group_capacity(int *max_groups)
 {
-    auto kern = tc_gemm_kernel<MODE, TO, CG>;
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG>::SMEM);
+    static std::atomic<int> cached[MAX_DEVICES];   // 0 = not yet known
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    int max_groups = g_num_sms / CG;
+    if (dev >= 0 && dev < MAX_DEVICES && cached[dev] > 0) {
+        *max_groups = cached[dev];
+        return cudaSuccess;
+    }
+    auto kern = tc_gemm_kernel<MODE, TO, CG>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG>::SMEM);
+    if (e != cudaSuccess) return e;
+    int groups = g_num_sms / CG;
     if (CG > 1) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(g_num_sms / CG * CG);
@@ -678,10 +697,24 @@ cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap
         q.attrs = qa;
         q.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess && n > 0 && n < max_groups) max_groups = n;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess && n > 0 && n < groups) groups = n;
         cudaGetLastError();
     }
-    const int groups = p.max_tiles < max_groups ? p.max_tiles : max_groups;
+    if (dev >= 0 && dev < MAX_DEVICES) cached[dev] = groups;
+    *max_groups = groups;
+    return cudaSuccess;
+}
+
+// Persistent grid: min(work items, CTA groups that can be resident at once).
+template <int MODE, typename TO, int CG>
+cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const TcParams &p, cudaStream_t s)
+{
+    auto kern = tc_gemm_kernel<MODE, TO, CG>;
+    int max_groups = 0;
+    const cudaError_t e = group_capacity<MODE, TO, CG>(&max_groups);
+    if (e != cudaSuccess) return e;
+    const int items = p.max_tiles * p.ksplit;
+    const int groups = items < max_groups ? items : max_groups;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(groups * CG);
     lc.blockDim = dim3(THREADS);
@@ -699,7 +732,7 @@ cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap
 
 template <int CG>
 cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t term_rows, int64_t b_rows_total,
-                int32_t *status, cudaStream_t s)
+                int ksplit, int32_t *status, cudaStream_t s)
 {
     if (!g_encode) return cudaErrorInitializationError;
     if (g.K % BK) return cudaErrorInvalidValue;
@@ -719,6 +752,11 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.E = g.E;
     const int mtiles = g.offsets ? max_mtiles : (g.M + Cfg<CG>::TILE_M - 1) / Cfg<CG>::TILE_M;
     p.max_tiles = mtiles * p.ntn;
+    p.ksplit = ksplit < 1 ? 1 : ksplit;
+    p.split_rows = g.M;
+    if (p.ksplit > 1 && (g.offsets || (mode != EPI_STORE_F32 && mode != EPI_SIGMOID_PARTIAL) ||
+                         p.ksplit > p.nkb * nterms))
+        return cudaErrorInvalidValue;
     p.epi = g.epi;
     p.status = status;
     if (p.max_tiles == 0) return cudaSuccess;
@@ -726,11 +764,12 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128)) return cudaErrorInvalidValue;
     if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG))
         return cudaErrorInvalidValue;
-    const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_COMBINE);
+    if (mode == EPI_SIGMOID_PARTIAL) mode = EPI_STORE_F32;   // raw fp32 partial tiles; sigmoid after the sum
+    const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_COMBINE || mode == EPI_STORE_F32);
     p.out_cols = (mode == EPI_GLU) ? g.N / 2 : g.N;
     CUtensorMap tc;
     memset(&tc, 0, sizeof tc);
-    p.tma_store = make_out_map(&tc, g.epi.out, out_f32, (uint64_t)p.out_cols, (uint64_t)g.M,
+    p.tma_store = make_out_map(&tc, g.epi.out, out_f32, (uint64_t)p.out_cols, (uint64_t)g.M * p.ksplit,
                                (uint64_t)g.epi.ldo * (out_f32 ? 4 : 2)) ? 1 : 0;
     switch (mode) {
     case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG>(ta, tb, tc, p, s);
@@ -739,6 +778,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
         return launch<EPI_GLU, bf16, CG>(ta, tb, tc, p, s);
     case EPI_COMBINE: return launch<EPI_COMBINE, float, CG>(ta, tb, tc, p, s);
     case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tb, tc, p, s);
+    case EPI_STORE_F32: return launch<EPI_STORE, float, CG>(ta, tb, tc, p, s);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -764,20 +804,23 @@ lmoe_status tc_check_device()
     return LMOE_OK;
 }
 
-cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t *status, cudaStream_t s)
+cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t *status, cudaStream_t s,
+                    int ksplit)
 {
     // B rows: dense N; grouped E * (rows per expert)
     const int64_t b_rows = g.offsets ? (int64_t)g.E * (g.b_group_stride / g.ldb) : g.N;
-    if (cg == 2) return run<2>(mode, g, max_mtiles, 1, 0, b_rows, status, s);
-    return run<1>(mode, g, max_mtiles, 1, 0, b_rows, status, s);
+    if (cg == 2) return run<2>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
+    return run<1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
 }
 
-cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s)
+int tc_num_sms() { return g_num_sms; }
+
+cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s, int ksplit)
 {
     GemmArgs r = g;
     r.B = Wr3;
     r.ldb = g.K;
-    return run<1>(EPI_SIGMOID, r, 0, 3, g.N, 3 * (int64_t)g.N, status, s);
+    return run<1>(ksplit > 1 ? EPI_SIGMOID_PARTIAL : EPI_SIGMOID, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
 }
 
 }  // namespace lmoe

@@ -15,10 +15,19 @@ lmoe_status tc_check_device();
 // g.offsets != nullptr (tile_off built for 128 cg rows per m-tile; max_mtiles
 // bounds the m-tiles of all experts).  Bounded waits that give up OR a code
 // into *status.
-cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t *status, cudaStream_t s);
+// ksplit > 1 (dense, mode EPI_STORE_F32 only): the K range is split into
+// ksplit parts whose fp32 partial tiles go to rows [split M, split M + M) of
+// g.epi.out; launch_splitk_reduce sums them and applies the real epilogue.
+cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t *status, cudaStream_t s,
+                    int ksplit = 1);
+
+// Number of SMs of the current device (after tc_check_device).
+int tc_num_sms();
 
 // Router r = sigmoid(x W_r^T) from the three-term bf16 split of fp32 W_r
 // (Wr3 = [3, E, d]): the three products accumulate into one fp32 TMEM tile.
-cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s);
+// ksplit > 1: the 3 d/64 k-blocks are split into ksplit ranges whose raw fp32
+// partial tiles go to g.epi.out slabs (launch_splitk_reduce applies sigmoid).
+cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s, int ksplit = 1);
 
 }  // namespace lmoe

@@ -51,7 +51,8 @@ lmoe_status fail(lmoe_status s, const char *fmt, ...)
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-    size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, status;
+    size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, partial,
+        status;
     size_t total;
 };
 
@@ -82,6 +83,54 @@ struct lmoe_handle {
 
 namespace {
 
+// Few-token plans.  The router runs on CUDA cores for a handful of tokens;
+// a dense tensor-core GEMM (the router included) whose tiles cover fewer than
+// half the SMs is split along K into as many parts as keep all parts in one
+// wave (fp32 partial tiles, then an ordered reduction that applies the
+// epilogue).
+constexpr int64_t ROUTER_SMALL_MAX_T = 8;
+constexpr int SPLIT_MAX = 16;
+
+// K splits for a dense GEMM of M rows, N columns (tiles of 128 x 256), nkb
+// k-blocks of 64.
+int plan_ksplit(const lmoe_handle *h, int64_t M, int64_t N, int64_t nkb)
+{
+    if (!h->tc) return 1;
+    const int sms = tc_num_sms() > 0 ? tc_num_sms() : 148;
+    const int64_t tiles = ((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN);
+    if (tiles * 2 >= sms) return 1;
+    int64_t ks = sms / tiles;
+    if (ks > nkb / 4) ks = nkb / 4;
+    if (ks > SPLIT_MAX) ks = SPLIT_MAX;
+    return ks >= 2 ? (int)ks : 1;
+}
+
+struct SplitPlan {
+    int router, down, shared, final_;
+    size_t partial_floats;   // largest ks * T * N over the split GEMMs
+};
+
+SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
+{
+    const lmoe_config &c = h->cfg;
+    const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
+    SplitPlan sp;
+    sp.router = (h->tc && T > ROUTER_SMALL_MAX_T) ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK) : 1;
+    sp.down = plan_ksplit(h, T, c.l, c.d / TC_BK);
+    sp.shared = plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
+    sp.final_ = plan_ksplit(h, T, c.d, ld_hs / TC_BK);
+    size_t m = 0;
+    auto upd = [&](int ks, int64_t n) {
+        if (ks > 1 && (size_t)ks * (size_t)n * (size_t)T > m) m = (size_t)ks * (size_t)n * (size_t)T;
+    };
+    upd(sp.router, c.E);
+    upd(sp.down, c.l);
+    upd(sp.shared, 4 * (int64_t)c.f_shared);
+    upd(sp.final_, c.d);
+    sp.partial_floats = m;
+    return sp;
+}
+
 Layout plan(const lmoe_handle *h, int64_t T)
 {
     const lmoe_config &c = h->cfg;
@@ -105,6 +154,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.H = take(h->tb * S * c.f);
     L.Yp = take(sizeof(float) * S * c.l);
     L.HS = take(h->tb * T * (2 * (int64_t)c.f_shared + c.l));
+    L.partial = take(sizeof(float) * plan_splits(h, T).partial_floats);
     L.status = take(256);
     L.total = o;
     return L;
@@ -292,8 +342,13 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
     g_err.clear();
     if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
     // status reset, router, histogram reset, top-k, scan, dispatch, down, permute, gate/up,
-    // down+combine, norm, shared, final
-    *launches = T == 0 ? 0 : 13;
+    // down+combine, norm, shared, final; plus one reduction per split-K GEMM
+    if (T == 0) { *launches = 0; return LMOE_OK; }
+    const lmoe_config &c = h->cfg;
+    const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
+    const SplitPlan sp = plan_splits(h, T);
+    (void)ld_hs;
+    *launches = 13 + (sp.router > 1) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
     return LMOE_OK;
 }
 
@@ -351,6 +406,8 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     const int max_mtiles = (int)((S + bm - 1) / bm + c.E);
 
     LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    const SplitPlan sp = plan_splits(h, T);
+    float *partial = (float *)(ws + L.partial);
 #define STAGE(i)                                                                                 \
     if (h->stage_events) LMOE_CUDA(cudaEventRecord((cudaEvent_t)h->stage_events[i], s))
 
@@ -360,7 +417,15 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
         GemmArgs g = {};
         g.A = x; g.lda = c.d; g.M = (int)T; g.N = c.E; g.K = c.d;
         g.epi.out = r32; g.epi.ldo = c.E;
-        if (h->tc) {
+        if (h->tc && T <= ROUTER_SMALL_MAX_T) {
+            LMOE_CUDA(launch_router_small((const bf16 *)x, h->Wr, T, c.E, c.d, r32, s));
+        } else if (h->tc && sp.router > 1) {
+            GemmArgs gp = g;
+            gp.epi.out = partial;
+            gp.epi.ldo = c.E;
+            LMOE_CUDA(tc_gemm_router(h->Wr3, gp, status, s, sp.router));
+            LMOE_CUDA(launch_splitk_reduce(partial, sp.router, T, c.E, EPI_SIGMOID, 0, 0.f, 0.f, 0, r32, c.E, s));
+        } else if (h->tc) {
             LMOE_CUDA(tc_gemm_router(h->Wr3, g, status, s));
         } else {
             g.B = h->Wr; g.ldb = c.d;
@@ -400,8 +465,19 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     gf.A = HS; gf.lda = ld_hs; gf.B = h->Wcat; gf.ldb = ld_hs; gf.M = (int)T; gf.N = c.d; gf.K = (int)ld_hs;
     gf.epi.out = output; gf.epi.ldo = c.d;
 
+    // Dense tensor-core GEMM, split along K per the plan.
+    auto dense_tc = [&](int mode, const GemmArgs &g, int ks) -> cudaError_t {
+        if (ks <= 1) return tc_gemm(mode, g, 0, cg_dense, status, s);
+        GemmArgs gp = g;
+        gp.epi.out = partial;
+        gp.epi.ldo = g.N;
+        cudaError_t e = tc_gemm(EPI_STORE_F32, gp, 0, 1, status, s, ks);
+        if (e != cudaSuccess) return e;
+        return launch_splitk_reduce(partial, ks, g.M, g.N, mode, g.epi.act, g.epi.gate_cap, g.epi.up_cap, TC_BN / 2,
+                                    g.epi.out, g.epi.ldo, s);
+    };
     STAGE(4);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gd, 0, cg_dense, status, s));
+    if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down));
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, s));
     STAGE(5);
     LMOE_CUDA(launch_permute_rows(z, perm_tok, Zp, S, c.l, (int)h->tb, s));
@@ -416,10 +492,10 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
                                   2 * (int64_t)c.f_shared, tk, s));
     STAGE(9);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gs, 0, cg_dense, status, s));
+    if (h->tc) LMOE_CUDA(dense_tc(EPI_GLU, gs, sp.shared));
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, s));
     STAGE(10);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_STORE, gf, 0, cg_dense, status, s));
+    if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gf, sp.final_));
     else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, s));
     STAGE(LMOE_NUM_STAGES);
 #undef STAGE

@@ -43,7 +43,9 @@ enum EpiMode {
     EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
     EPI_GLU = 3,      // out[m, n'] = act(C[gate], C[up])   (gate/up GEMMs -> h)
     EPI_COMBINE = 4,  // out32[m, n] = w[m] * C             (routed down -> p-weighted rows)
-    EPI_GLU_SITU = 5  // EPI_GLU with the SiTU gate, as its own instantiation
+    EPI_GLU_SITU = 5, // EPI_GLU with the SiTU gate, as its own instantiation
+    EPI_STORE_F32 = 6, // out32[m, n] = C                   (split-K partial tiles)
+    EPI_SIGMOID_PARTIAL = 7  // router split-K: EPI_STORE_F32 partials, sigmoid in the reduction
 };
 
 struct EpiArgs {
@@ -108,6 +110,16 @@ cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp
                                 cudaStream_t s);
 cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s);
+
+// Sum ksplit fp32 partial tiles [ksplit][M][N] in split order and apply the
+// epilogue: EPI_STORE (bf16 out[m, n]), EPI_GLU (gate/up column pairs
+// interleaved in blocks of ib, bf16 out[m, n'] for n' < N / 2) or EPI_SIGMOID
+// (fp32 out[m, n] = sigmoid(sum)).
+cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
+                                 float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s);
+// Router scores for a few tokens on CUDA cores: r[t, e] = sigmoid(sum_k x[t, k] W[e, k]),
+// x bf16 [T, d], W fp32 [E, d] (fixed summation order, deterministic).
+cudaError_t launch_router_small(const bf16 *x, const float *W, int64_t T, int E, int d, float *r, cudaStream_t s);
 
 // Weight repacking (create time).
 cudaError_t launch_pack_glu(const void *G, const void *U, void *P, int nE, int F, int K, int ib, int elem_bytes,

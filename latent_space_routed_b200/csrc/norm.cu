@@ -13,9 +13,10 @@
 namespace lmoe {
 namespace {
 
-constexpr int NT = 256;
-
-template <typename TT>
+// NT threads per token: 256 when tokens fill the GPU, 1024 for a few tokens
+// (more loads in flight per token).  The slot loads of a column are issued
+// eight at a time, then added in slot order.
+template <typename TT, int NT>
 __global__ void __launch_bounds__(NT)
 combine_norm_kernel(const float *__restrict__ Yp, const int32_t *__restrict__ slot_of, int l, int k, float eps,
                     TT *__restrict__ u_out, TT *__restrict__ hs, int64_t ld_hs, int64_t col0)
@@ -29,7 +30,15 @@ combine_norm_kernel(const float *__restrict__ Yp, const int32_t *__restrict__ sl
     float ss = 0.f;
     for (int c = threadIdx.x; c < l; c += NT) {
         float acc = 0.f;
-        for (int j = 0; j < k; ++j) acc += Yp[(int64_t)slots[j] * l + c];
+        int j = 0;
+        for (; j + 8 <= k; j += 8) {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = Yp[(int64_t)slots[j + i] * l + c];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc += v[i];
+        }
+        for (; j < k; ++j) acc += Yp[(int64_t)slots[j] * l + c];
         u[c] = acc;
         u_out[t * l + c] = from_f32<TT>(acc);
         ss += acc * acc;
@@ -96,7 +105,74 @@ __global__ void split_router_kernel(const float *__restrict__ W, bf16 *__restric
     }
 }
 
+// Split-K reduction: out[m, :] from the sum over splits of partial[s, m, :],
+// four output columns per thread, splits summed in order (deterministic).
+template <int MODE>
+__global__ void __launch_bounds__(256)
+splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, int N, int act, float gate_cap,
+                     float up_cap, int ib, void *__restrict__ out_, int64_t ldo)
+{
+    const int64_t m = blockIdx.y;
+    const int nout = (MODE == EPI_GLU) ? N / 2 : N;
+    const int j0 = (blockIdx.x * 256 + threadIdx.x) * 4;
+    if (j0 >= nout) return;
+    const int64_t slab = M * (int64_t)N;
+    float r[4];
+    if (MODE == EPI_SIGMOID) {
+        r[0] = r[1] = r[2] = r[3] = 0.f;
+        const int n = N - j0 < 4 ? N - j0 : 4;
+        for (int sp = 0; sp < ksplit; ++sp)
+            for (int i = 0; i < n; ++i) r[i] += partial[sp * slab + m * N + j0 + i];
+        float *o = reinterpret_cast<float *>(out_) + m * ldo + j0;
+        for (int i = 0; i < n; ++i) o[i] = sigmoidf_(r[i]);
+        return;
+    }
+    if (MODE == EPI_GLU) {
+        // output column j: gate column (j / ib) 2 ib + j % ib, up column ib after it
+        const int g0 = (j0 / ib) * 2 * ib + (j0 % ib);
+        float gv[4] = {0.f, 0.f, 0.f, 0.f}, uv[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int sp = 0; sp < ksplit; ++sp) {
+            const float4 a = *reinterpret_cast<const float4 *>(partial + sp * slab + m * N + g0);
+            const float4 b = *reinterpret_cast<const float4 *>(partial + sp * slab + m * N + g0 + ib);
+            gv[0] += a.x; gv[1] += a.y; gv[2] += a.z; gv[3] += a.w;
+            uv[0] += b.x; uv[1] += b.y; uv[2] += b.z; uv[3] += b.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] = glu_act(act, gv[i], uv[i], gate_cap, up_cap);
+    } else {
+        r[0] = r[1] = r[2] = r[3] = 0.f;
+        for (int sp = 0; sp < ksplit; ++sp) {
+            const float4 a = *reinterpret_cast<const float4 *>(partial + sp * slab + m * N + j0);
+            r[0] += a.x; r[1] += a.y; r[2] += a.z; r[3] += a.w;
+        }
+    }
+    bf16 *out = reinterpret_cast<bf16 *>(out_);
+    const __nv_bfloat162 p0 = __floats2bfloat162_rn(r[0], r[1]);
+    const __nv_bfloat162 p1 = __floats2bfloat162_rn(r[2], r[3]);
+    uint2 w;
+    w.x = *reinterpret_cast<const uint32_t *>(&p0);
+    w.y = *reinterpret_cast<const uint32_t *>(&p1);
+    *reinterpret_cast<uint2 *>(out + m * ldo + j0) = w;
+}
+
 }  // namespace
+
+cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
+                                 float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s)
+{
+    if (M == 0) return cudaSuccess;
+    if (mode != EPI_SIGMOID && (N % 8 || ldo % 4 || (mode == EPI_GLU && ib % 4))) return cudaErrorInvalidValue;
+    const int nout = mode == EPI_GLU ? N / 2 : N;
+    dim3 grid((unsigned)(((nout + 3) / 4 + 255) / 256), (unsigned)M);
+    if (mode == EPI_GLU)
+        splitk_reduce_kernel<EPI_GLU><<<grid, 256, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
+    else if (mode == EPI_SIGMOID)
+        splitk_reduce_kernel<EPI_SIGMOID><<<grid, 256, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out,
+                                                               ldo);
+    else
+        splitk_reduce_kernel<EPI_STORE><<<grid, 256, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s)
@@ -104,12 +180,22 @@ cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t
     if (T == 0) return cudaSuccess;
     if (k > 64) return cudaErrorInvalidValue;
     const size_t smem = sizeof(float) * l;
-    if (tok_bf16)
-        combine_norm_kernel<bf16><<<(unsigned)T, NT, smem, s>>>(Yp, slot_of, l, k, eps, (bf16 *)u_out, (bf16 *)hs,
-                                                                  ld_hs, col0);
-    else
-        combine_norm_kernel<float><<<(unsigned)T, NT, smem, s>>>(Yp, slot_of, l, k, eps, (float *)u_out,
-                                                                   (float *)hs, ld_hs, col0);
+    const bool few = T < 296;   // fewer tokens than two per SM: wide blocks
+    if (tok_bf16) {
+        if (few)
+            combine_norm_kernel<bf16, 1024><<<(unsigned)T, 1024, smem, s>>>(Yp, slot_of, l, k, eps, (bf16 *)u_out,
+                                                                           (bf16 *)hs, ld_hs, col0);
+        else
+            combine_norm_kernel<bf16, 256><<<(unsigned)T, 256, smem, s>>>(Yp, slot_of, l, k, eps, (bf16 *)u_out,
+                                                                         (bf16 *)hs, ld_hs, col0);
+    } else {
+        if (few)
+            combine_norm_kernel<float, 1024><<<(unsigned)T, 1024, smem, s>>>(Yp, slot_of, l, k, eps, (float *)u_out,
+                                                                            (float *)hs, ld_hs, col0);
+        else
+            combine_norm_kernel<float, 256><<<(unsigned)T, 256, smem, s>>>(Yp, slot_of, l, k, eps, (float *)u_out,
+                                                                          (float *)hs, ld_hs, col0);
+    }
     return cudaGetLastError();
 }
 

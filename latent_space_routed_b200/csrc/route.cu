@@ -150,6 +150,59 @@ dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, 
     }
 }
 
+// Router for a few tokens: one block per (expert row e, ROUTER_TB tokens).
+// The block's 8 warps stream W[e] (fp32, 16-byte loads) in interleaved
+// 512-byte pieces against the same columns of each token; each warp adds its
+// lanes in a fixed butterfly order and the warps' partial sums are added in
+// warp order, so the result does not depend on timing.
+constexpr int ROUTER_TB = 8;
+constexpr int ROUTER_WARPS = 8;
+
+__global__ void __launch_bounds__(ROUTER_WARPS * 32)
+router_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ W, int64_t T, int E, int d,
+                    float *__restrict__ r)
+{
+    __shared__ float part[ROUTER_WARPS][ROUTER_TB];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int e = blockIdx.x;
+    const int64_t t0 = (int64_t)blockIdx.y * ROUTER_TB;
+    float acc[ROUTER_TB];
+#pragma unroll
+    for (int j = 0; j < ROUTER_TB; ++j) acc[j] = 0.f;
+    const float4 *w = reinterpret_cast<const float4 *>(W + (int64_t)e * d);
+    for (int c = warp * 32 + lane; c < d / 4; c += ROUTER_WARPS * 32) {
+        const float4 wv = __ldg(w + c);
+#pragma unroll
+        for (int j = 0; j < ROUTER_TB; ++j) {
+            if (t0 + j < T) {
+                const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (t0 + j) * d) + c);
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
+                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
+                acc[j] = fmaf(wv.x, a.x, acc[j]);
+                acc[j] = fmaf(wv.y, a.y, acc[j]);
+                acc[j] = fmaf(wv.z, b.x, acc[j]);
+                acc[j] = fmaf(wv.w, b.y, acc[j]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < ROUTER_TB; ++j) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < ROUTER_TB; ++j) part[warp][j] = acc[j];
+    }
+    __syncthreads();
+    if (threadIdx.x < ROUTER_TB && t0 + threadIdx.x < T) {
+        float a = 0.f;
+#pragma unroll
+        for (int q = 0; q < ROUTER_WARPS; ++q) a += part[q][threadIdx.x];
+        r[(t0 + threadIdx.x) * E + e] = sigmoidf_(a);
+    }
+}
+
 // Zp[m, :] = z[perm_tok[m], :]: one warp per slot row, 16-byte vectors.
 __global__ void __launch_bounds__(256)
 permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ perm_tok, uint4 *__restrict__ Zp,
@@ -164,6 +217,15 @@ permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ per
 }
 
 }  // namespace
+
+cudaError_t launch_router_small(const bf16 *x, const float *W, int64_t T, int E, int d, float *r, cudaStream_t s)
+{
+    if (T == 0) return cudaSuccess;
+    if (d % 4) return cudaErrorInvalidValue;
+    dim3 grid((unsigned)E, (unsigned)((T + ROUTER_TB - 1) / ROUTER_TB));
+    router_small_kernel<<<grid, ROUTER_WARPS * 32, 0, s>>>(x, W, T, E, d, r);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
                                 cudaStream_t s)
