@@ -52,6 +52,27 @@ def parse():
     return ap.parse_args()
 
 
+def measured_traffic(workload, T, kernel):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary under
+    profiles/, or None when none matches or the kernel sources changed since."""
+    import glob
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in ("latent_space_routed_b200/csrc/gemm_tc.cu", "latent_space_routed_b200/csrc/lmoe_api.cu"):
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    pat = re.compile(r"^traffic: workload=(\S+) T=(\d+) kernel=(\S+) bytes=(\d+) sources=(\w+)")
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        with open(path) as fh:
+            for line in fh:
+                m = pat.match(line.strip())
+                if m and m.group(1) == workload and int(m.group(2)) == T and m.group(3) == kernel:
+                    return int(m.group(4)) if m.group(5) == sha else None
+    return None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -204,6 +225,7 @@ def run_own(args, rank, world, local_rank):
     W = li.weights(w)
     x_cpu = li.tokens(w, T, seed=w.seed + 1000 * rank)
     layer = lm.LatentMoE(lm.config_for(w, gemm=args.gemm), {k: v.to(dev) for k, v in W.items()})
+    torch.cuda.empty_cache()   # the caller-side weight copies are no longer needed (the handle repacked them)
     x = x_cpu.to(dev)
     out = layer.empty_outputs(T)
     stream = torch.cuda.current_stream()
@@ -336,7 +358,7 @@ def run_own(args, rank, world, local_rank):
     else:
         roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(w.name, T, dom)
     roof["kernel"] = dom
     roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stage_ms[dom]}
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst bf16 / copy bandwidth)"
