@@ -107,8 +107,8 @@ def stage_model(w, T, touched):
         "down_proj": (2 * T * w.d * w.l, T * w.d * B + w.l * w.d * B + T * w.l * B),
         "permute": (0, T * w.l * B + S * w.l * B + S * 4),
         "gate_up": (2 * S * 2 * w.f * w.l, touched * 2 * w.f * w.l * B + S * w.l * B + S * w.f * B),
-        "down_combine": (2 * S * w.l * w.f, touched * w.l * w.f * B + S * w.f * B + S * w.l * 4),
-        "combine_norm": (0, S * w.l * 4 + 2 * T * w.l * B),
+        "down_combine": (2 * S * w.l * w.f, touched * w.l * w.f * B + S * w.f * B + S * w.l * B),
+        "combine_norm": (0, S * w.l * B + 2 * T * w.l * B),
         "shared_gate_up": (2 * T * w.d * 4 * w.f_s, T * w.d * B + 4 * w.f_s * w.d * B + T * 2 * w.f_s * B),
         "final": (2 * T * w.d * (2 * w.f_s + w.l),
                   T * (2 * w.f_s + w.l) * B + w.d * (2 * w.f_s + w.l) * B + T * w.d * B),

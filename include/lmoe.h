@@ -192,7 +192,7 @@ LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t 
  * 2 per-expert counts [E] int32; 3 expert offsets [E+1] int32;
  * 4 slot index of (t, j) [T, k] int32; 5 token of each permuted slot [T*k]
  * int32; 6 latent rows z [T, l]; 7 routed hidden H [T*k, f] (slot order);
- * 8 p-weighted expert outputs [T*k, l] fp32; 9 [shared hidden | RMSNorm(u)]
+ * 8 p-weighted expert outputs [T*k, l] (token dtype); 9 [shared hidden | RMSNorm(u)]
  * [T, 2 f_shared + l]; 10 device status word (int32).
  * INVALID_ARG for an unknown region. */
 LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t region, size_t *offset,

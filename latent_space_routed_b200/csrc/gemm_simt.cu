@@ -149,7 +149,7 @@ cudaError_t launch_simt_gemm(int mode, int ta, int tb, int to, const GemmArgs &g
     LMOE_SIMT_CASE(bf16, bf16, bf16, EPI_STORE)
     LMOE_SIMT_CASE(bf16, float, float, EPI_SIGMOID)
     LMOE_SIMT_CASE(bf16, bf16, bf16, EPI_GLU)
-    LMOE_SIMT_CASE(bf16, bf16, float, EPI_COMBINE)
+    LMOE_SIMT_CASE(bf16, bf16, bf16, EPI_COMBINE)
 #undef LMOE_SIMT_CASE
     return cudaErrorInvalidValue;
 }

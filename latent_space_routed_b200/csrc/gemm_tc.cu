@@ -592,7 +592,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
                             for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
                         } else if (MODE == EPI_COMBINE) {
-                            const float w = valid ? p.epi.row_w[row] : 0.f;
+                            const float w = valid ? p.epi.row_w[row] : 0.f;   // bf16 rows: p-weighted here
 #pragma unroll
                             for (int i = 0; i < 32; ++i) x[i] *= w;
                         }
@@ -765,7 +765,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG))
         return cudaErrorInvalidValue;
     if (mode == EPI_SIGMOID_PARTIAL) mode = EPI_STORE_F32;   // raw fp32 partial tiles; sigmoid after the sum
-    const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_COMBINE || mode == EPI_STORE_F32);
+    const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_STORE_F32);
     p.out_cols = (mode == EPI_GLU) ? g.N / 2 : g.N;
     CUtensorMap tc;
     memset(&tc, 0, sizeof tc);
@@ -776,7 +776,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     case EPI_GLU:
         if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG>(ta, tb, tc, p, s);
         return launch<EPI_GLU, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_COMBINE: return launch<EPI_COMBINE, float, CG>(ta, tb, tc, p, s);
+    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG>(ta, tb, tc, p, s);
     case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tb, tc, p, s);
     case EPI_STORE_F32: return launch<EPI_STORE, float, CG>(ta, tb, tc, p, s);
     default: return cudaErrorInvalidValue;

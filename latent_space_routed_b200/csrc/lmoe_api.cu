@@ -10,7 +10,7 @@
 //   5 down GEMM        z = x W_down^T                           [T, l]
 //   6 permute          Zp[m] = z[token of slot m]               [S, l]
 //   7 gate/up GEMM     per expert: h = act(G z, U z)            [S, f]
-//   8 down GEMM        per expert: Y = p * (h D^T)              [S, l] fp32
+//   8 down GEMM        per expert: Y = p * (h D^T)              [S, l] token dtype
 //   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
 //  10 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
 //  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
@@ -152,7 +152,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.z = take(h->tb * T * c.l);
     L.Zp = take(h->tb * S * c.l);
     L.H = take(h->tb * S * c.f);
-    L.Yp = take(sizeof(float) * S * c.l);
+    L.Yp = take(h->tb * S * c.l);
     L.HS = take(h->tb * T * (2 * (int64_t)c.f_shared + c.l));
     L.partial = take(sizeof(float) * plan_splits(h, T).partial_floats);
     L.status = take(256);
@@ -318,7 +318,7 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
     case 6: *offset = L.z; *bytes = h->tb * T * c.l; break;
     case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
-    case 8: *offset = L.Yp; *bytes = sizeof(float) * S * c.l; break;
+    case 8: *offset = L.Yp; *bytes = h->tb * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
     case 10: *offset = L.status; *bytes = sizeof(int32_t); break;
     default: return fail(LMOE_ERR_INVALID_ARG, "unknown region %d", region);
@@ -391,7 +391,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     int32_t *perm_tok = (int32_t *)(ws + L.perm_tok);
     float *perm_w = (float *)(ws + L.perm_w);
     void *z = ws + L.z, *Zp = ws + L.Zp, *H = ws + L.H, *HS = ws + L.HS;
-    float *Yp = (float *)(ws + L.Yp);
+    void *Yp = ws + L.Yp;
     int32_t *status = (int32_t *)(ws + L.status);
 
     const int64_t S = T * c.k;
@@ -486,7 +486,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, s));
     STAGE(7);
     if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, cg_grouped, status, s));
-    else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, 0, gc, max_mtiles, s));
+    else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, tk, gc, max_mtiles, s));
     // 8 u, RMSNorm(u) into the columns after the shared hidden
     STAGE(8);
     LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,

@@ -42,7 +42,7 @@ enum EpiMode {
     EPI_STORE = 0,    // out[m, n] = C                      (final GEMM -> y)
     EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
     EPI_GLU = 3,      // out[m, n'] = act(C[gate], C[up])   (gate/up GEMMs -> h)
-    EPI_COMBINE = 4,  // out32[m, n] = w[m] * C             (routed down -> p-weighted rows)
+    EPI_COMBINE = 4,  // out[m, n] = w[m] * C               (routed down -> p-weighted rows)
     EPI_GLU_SITU = 5, // EPI_GLU with the SiTU gate, as its own instantiation
     EPI_STORE_F32 = 6, // out32[m, n] = C                   (split-K partial tiles)
     EPI_SIGMOID_PARTIAL = 7  // router split-K: EPI_STORE_F32 partials, sigmoid in the reduction
@@ -66,10 +66,10 @@ __device__ __forceinline__ void epi_store_chunk(const EpiArgs &e, int64_t row, i
         #pragma unroll
         for (int i = 0; i < 32; ++i) if (i < n) o[i] = sigmoidf_(v[i]);
     } else if (MODE == EPI_COMBINE) {
-        float *o = (float *)e.out + row * e.ldo + col;
+        TO *o = (TO *)e.out + row * e.ldo + col;
         const float w = e.row_w[row];
         #pragma unroll
-        for (int i = 0; i < 32; ++i) if (i < n) o[i] = w * v[i];
+        for (int i = 0; i < 32; ++i) if (i < n) o[i] = from_f32<TO>(w * v[i]);
     } else {
         TO *o = (TO *)e.out + row * e.ldo + col;
 #pragma unroll
@@ -108,7 +108,8 @@ cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t 
                             int32_t *slot_of, int32_t *perm_tok, float *perm_w, cudaStream_t s);
 cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
                                 cudaStream_t s);
-cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
+// Yp in the token dtype.
+cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s);
 
 // Sum ksplit fp32 partial tiles [ksplit][M][N] in split order and apply the

@@ -1,8 +1,9 @@
 // Weighted combine + RMSNorm, and create-time weight repacking.
 //
 // combine_norm ("Stable LatentMoE", equations for u and y): for token t,
-//   u = sum_j Y[slot_of[t, j]]        (rows already scaled by p_j, summed in
-//                                      slot order j = 0..k-1: deterministic)
+//   u = sum_j Y[slot_of[t, j]]        (rows already scaled by p_j, stored in the
+//                                      token dtype, summed in fp32 in slot
+//                                      order j = 0..k-1: deterministic)
 //   n = u / sqrt(mean(u^2) + eps)     (RMSNorm, unit gain, eps inside the root)
 // u is written out as latent_routed_aggregate (token dtype); n goes to the
 // columns [col0, col0 + l) of the final GEMM's A operand, right after the
@@ -18,7 +19,7 @@ namespace {
 // eight at a time, then added in slot order.
 template <typename TT, int NT>
 __global__ void __launch_bounds__(NT)
-combine_norm_kernel(const float *__restrict__ Yp, const int32_t *__restrict__ slot_of, int l, int k, float eps,
+combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_of, int l, int k, float eps,
                     TT *__restrict__ u_out, TT *__restrict__ hs, int64_t ld_hs, int64_t col0)
 {
     extern __shared__ float u[];   // [l]
@@ -34,11 +35,11 @@ combine_norm_kernel(const float *__restrict__ Yp, const int32_t *__restrict__ sl
         for (; j + 8 <= k; j += 8) {
             float v[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = Yp[(int64_t)slots[j + i] * l + c];
+            for (int i = 0; i < 8; ++i) v[i] = to_f32(Yp[(int64_t)slots[j + i] * l + c]);
 #pragma unroll
             for (int i = 0; i < 8; ++i) acc += v[i];
         }
-        for (; j < k; ++j) acc += Yp[(int64_t)slots[j] * l + c];
+        for (; j < k; ++j) acc += to_f32(Yp[(int64_t)slots[j] * l + c]);
         u[c] = acc;
         u_out[t * l + c] = from_f32<TT>(acc);
         ss += acc * acc;
@@ -121,10 +122,19 @@ splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, i
     if (MODE == EPI_SIGMOID) {
         r[0] = r[1] = r[2] = r[3] = 0.f;
         const int n = N - j0 < 4 ? N - j0 : 4;
-        for (int sp = 0; sp < ksplit; ++sp)
-            for (int i = 0; i < n; ++i) r[i] += partial[sp * slab + m * N + j0 + i];
         float *o = reinterpret_cast<float *>(out_) + m * ldo + j0;
-        for (int i = 0; i < n; ++i) o[i] = sigmoidf_(r[i]);
+        if (n == 4 && (N & 3) == 0 && (ldo & 3) == 0) {
+            for (int sp = 0; sp < ksplit; ++sp) {
+                const float4 a = *reinterpret_cast<const float4 *>(partial + sp * slab + m * N + j0);
+                r[0] += a.x; r[1] += a.y; r[2] += a.z; r[3] += a.w;
+            }
+            *reinterpret_cast<float4 *>(o) = make_float4(sigmoidf_(r[0]), sigmoidf_(r[1]), sigmoidf_(r[2]),
+                                                         sigmoidf_(r[3]));
+        } else {
+            for (int sp = 0; sp < ksplit; ++sp)
+                for (int i = 0; i < n; ++i) r[i] += partial[sp * slab + m * N + j0 + i];
+            for (int i = 0; i < n; ++i) o[i] = sigmoidf_(r[i]);
+        }
         return;
     }
     if (MODE == EPI_GLU) {
@@ -174,7 +184,7 @@ cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, in
     return cudaGetLastError();
 }
 
-cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
+cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s)
 {
     if (T == 0) return cudaSuccess;
@@ -183,17 +193,17 @@ cudaError_t launch_combine_norm(const float *Yp, const int32_t *slot_of, int64_t
     const bool few = T < 296;   // fewer tokens than two per SM: wide blocks
     if (tok_bf16) {
         if (few)
-            combine_norm_kernel<bf16, 1024><<<(unsigned)T, 1024, smem, s>>>(Yp, slot_of, l, k, eps, (bf16 *)u_out,
+            combine_norm_kernel<bf16, 1024><<<(unsigned)T, 1024, smem, s>>>((const bf16 *)Yp, slot_of, l, k, eps, (bf16 *)u_out,
                                                                            (bf16 *)hs, ld_hs, col0);
         else
-            combine_norm_kernel<bf16, 256><<<(unsigned)T, 256, smem, s>>>(Yp, slot_of, l, k, eps, (bf16 *)u_out,
+            combine_norm_kernel<bf16, 256><<<(unsigned)T, 256, smem, s>>>((const bf16 *)Yp, slot_of, l, k, eps, (bf16 *)u_out,
                                                                          (bf16 *)hs, ld_hs, col0);
     } else {
         if (few)
-            combine_norm_kernel<float, 1024><<<(unsigned)T, 1024, smem, s>>>(Yp, slot_of, l, k, eps, (float *)u_out,
+            combine_norm_kernel<float, 1024><<<(unsigned)T, 1024, smem, s>>>((const float *)Yp, slot_of, l, k, eps, (float *)u_out,
                                                                             (float *)hs, ld_hs, col0);
         else
-            combine_norm_kernel<float, 256><<<(unsigned)T, 256, smem, s>>>(Yp, slot_of, l, k, eps, (float *)u_out,
+            combine_norm_kernel<float, 256><<<(unsigned)T, 256, smem, s>>>((const float *)Yp, slot_of, l, k, eps, (float *)u_out,
                                                                           (float *)hs, ld_hs, col0);
     }
     return cudaGetLastError();
