@@ -115,6 +115,29 @@ def stage_model(w, T, touched):
     }
 
 
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank float over the process group (the job's time is its
+    slowest rank's); the value itself when there is no group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, T: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own T-token batch per step."""
+    return world * T / (ms_per_step / 1e3)
+
+
+def replica_seed(w, rank: int) -> int:
+    """Each replica draws its own token batch (same weights)."""
+    return w.seed + 1000 * rank
+
+
 # ---------------------------------------------------------------- clocks
 class Clocks:
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -223,7 +246,7 @@ def run_own(args, rank, world, local_rank):
     w = li.WORKLOADS[args.workload]
     T = args.T or w.T
     W = li.weights(w)
-    x_cpu = li.tokens(w, T, seed=w.seed + 1000 * rank)
+    x_cpu = li.tokens(w, T, seed=replica_seed(w, rank))
     layer = lm.LatentMoE(lm.config_for(w, gemm=args.gemm), {k: v.to(dev) for k, v in W.items()})
     torch.cuda.empty_cache()   # the caller-side weight copies are no longer needed (the handle repacked them)
     x = x_cpu.to(dev)
@@ -280,11 +303,7 @@ def run_own(args, rank, world, local_rank):
     layer.check_device(T)
 
     step_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     stage_ms = {}
     for si, name in enumerate(lm.STAGE_NAMES):
         stage_ms[name] = sum(ev_stage[i][si].elapsed_time(ev_stage[i][si + 1]) for i in range(args.steps)) / args.steps
@@ -333,11 +352,7 @@ def run_own(args, rank, world, local_rank):
         layer.forward_host(x_host, out_host)
         e_b[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in zip(e_a, e_b))
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_a, e_b)), dev)
     B = w.item_bytes
     h2d = T * w.d * B
     d2h = T * w.d * B + T * w.k * 4 + T * w.k * B + T * w.l * B
@@ -348,7 +363,7 @@ def run_own(args, rank, world, local_rank):
 
     hbm, tf_burst, tf_sus, peak_src = peaks()
     ms = total_ms / args.steps
-    value = world * T / (ms / 1e3)
+    value = job_tokens_per_s(world, T, ms)
     model = stage_model(w, T, touched)
     dom = max(stage_ms, key=lambda k: stage_ms[k])
     fl, by = model[dom]
@@ -387,7 +402,7 @@ def run_own(args, rank, world, local_rank):
             "roofline": roof, "layer_roofline": layer_roof,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "cpu_baseline": cpu,
-            "e2e": {"value": world * T / (e2e_ms / args.steps / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_tokens_per_s(world, T, e2e_ms / args.steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": layer.launch_count(T) * args.steps, "clocks": clk,
             "host_us_per_call": host_us}

@@ -183,6 +183,21 @@ LMOE_API lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream)
  * read at each forward, not copied: the caller keeps it alive. */
 LMOE_API lmoe_status lmoe_set_stage_events(lmoe_handle *h, void *const *events, int32_t n);
 
+/* Test hooks for failure detection (no counterpart in the pages):
+ *  LMOE_INJECT_STALL_NEXT_GEMM  the next tensor-core GEMM this process launches
+ *      makes its MMA warp wait on a barrier that nothing signals.  The wait is
+ *      bounded (about 2 s of SM cycles): it gives up, the kernel records the
+ *      failure in the forward's status word, drains and returns, and
+ *      lmoe_check_device then reports LMOE_ERR_DEVICE_TIMEOUT.  Nothing faults
+ *      or hangs; the context stays usable.  (arg ignored.)
+ *  LMOE_INJECT_FAIL_ALLOC  the arg-th device allocation (1-based) of the next
+ *      lmoe_create fails as if cudaMalloc had: lmoe_create returns LMOE_ERR_OOM
+ *      and frees what it had allocated.
+ * INVALID_ARG for an unknown `what` or arg < 1 with LMOE_INJECT_FAIL_ALLOC. */
+#define LMOE_INJECT_STALL_NEXT_GEMM 1
+#define LMOE_INJECT_FAIL_ALLOC 2
+LMOE_API lmoe_status lmoe_debug_inject(int32_t what, int32_t arg);
+
 /* Number of kernel launches one lmoe_forward of T tokens makes. */
 LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches);
 

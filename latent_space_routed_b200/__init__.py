@@ -33,7 +33,7 @@ REGION = {"scores": 0, "p32": 1, "counts": 2, "offsets": 3, "slot_of": 4, "perm_
           "Y": 8, "HS": 9, "status": 10}
 
 EXPORTS = ("lmoe_config_from_base", "lmoe_create", "lmoe_workspace_size", "lmoe_forward", "lmoe_host_workspace_size",
-           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_set_bias", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
+           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_debug_inject", "lmoe_set_bias", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
            "lmoe_last_error", "lmoe_destroy")
 
 
@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "lmoe_host_workspace_size": (I32, [P, I64, ctypes.POINTER(SZ)]),
         "lmoe_forward_host": (I32, [P, P, I64, P, P, P, P, P, SZ, P]),
         "lmoe_forward_noalloc": (I32, [P, P, I64, P, P, P, P, P]),
+        "lmoe_debug_inject": (I32, [I32, I32]),
         "lmoe_set_bias": (I32, [P, P, P]),
         "lmoe_set_stage_events": (I32, [P, P, I32]),
         "lmoe_launch_count": (I32, [P, I64, ctypes.POINTER(I32)]),
@@ -157,6 +158,13 @@ def lmoe_forward_host(h, x_host, T, output_host, selected_experts_host, mixture_
 
 
 LMOE_NOALLOC_WORKSPACE_BYTES = 64 << 20
+LMOE_INJECT_STALL_NEXT_GEMM, LMOE_INJECT_FAIL_ALLOC = 1, 2
+
+
+def lmoe_debug_inject(what, arg=0):
+    """Failure-detection test hooks (see include/lmoe.h)."""
+    _check(_lib.lmoe_debug_inject(what, arg))
+
 
 
 def lmoe_forward_noalloc(h, x, T, output, selected_experts, mixture_weights, latent_routed_aggregate, stream=None):

@@ -92,6 +92,7 @@ struct TcParams {
     int64_t split_rows;         // rows of one partial slab (= M)
     EpiArgs epi;
     int out_cols;               // columns of the output tensor map
+    int stall_test;             // failure-detection test: the MMA warp waits on a barrier nobody signals
     int tma_store;              // 1: full chunks leave through TMA stores
     int32_t *status;
 };
@@ -498,6 +499,12 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     break;
                 }
                 tc_fence_after();
+                if (p.stall_test && local == 0 && !mbar_wait(accf_bar(acc), 0u)) {
+                    // only this thread commits that barrier: the wait runs out by design
+                    atomicOr(p.status, ST_MMA);
+                    *(volatile int *)abort_flag = 1;
+                    break;
+                }
                 const uint32_t dt = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
                     const int s = it % STAGES;
@@ -636,6 +643,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_stall_next{0};
 int g_num_sms = 0;
 
 // Output map: 32 x 32 boxes, swizzled to match stage_row.
@@ -759,6 +767,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
         return cudaErrorInvalidValue;
     p.epi = g.epi;
     p.status = status;
+    p.stall_test = g_stall_next.exchange(0);
     if (p.max_tiles == 0) return cudaSuccess;
     CUtensorMap ta, tb;
     if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128)) return cudaErrorInvalidValue;
@@ -814,6 +823,8 @@ cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t
 }
 
 int tc_num_sms() { return g_num_sms; }
+
+void tc_debug_stall_next() { g_stall_next.store(1); }
 
 cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s, int ksplit)
 {

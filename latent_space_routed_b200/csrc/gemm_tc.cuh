@@ -24,6 +24,11 @@ cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t
 // Number of SMs of the current device (after tc_check_device).
 int tc_num_sms();
 
+// Failure-detection test hook: the next tensor-core GEMM launch makes its MMA
+// warp wait on a barrier that nothing signals; the bounded wait runs out, the
+// status word records it and the kernel returns.
+void tc_debug_stall_next();
+
 // Router r = sigmoid(x W_r^T) from the three-term bf16 split of fp32 W_r
 // (Wr3 = [3, E, d]): the three products accumulate into one fp32 TMEM tile.
 // ksplit > 1: the 3 d/64 k-blocks are split into ksplit ranges whose raw fp32

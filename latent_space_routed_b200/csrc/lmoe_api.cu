@@ -14,6 +14,7 @@
 //   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
 //  10 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
 //  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -28,6 +29,7 @@ using namespace lmoe;
 namespace {
 
 thread_local std::string g_err;
+std::atomic<int> g_fail_alloc_at{0};   // test hook: this allocation of the next lmoe_create fails
 
 lmoe_status fail(lmoe_status s, const char *fmt, ...)
 {
@@ -247,9 +249,12 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
     const size_t tb = h->tb;
     const int64_t fs = c.f_shared;
 
+    int alloc_index = 0;
+    const int fail_at = g_fail_alloc_at.exchange(0);
 #define ALLOC(ptr, bytes)                                                                        \
     do {                                                                                         \
-        if (cudaMalloc((void **)&(ptr), (bytes)) != cudaSuccess) {                              \
+        ++alloc_index;                                                                           \
+        if (alloc_index == fail_at || cudaMalloc((void **)&(ptr), (bytes)) != cudaSuccess) {   \
             cudaGetLastError();                                                                  \
             free_handle(h);                                                                      \
             return fail(LMOE_ERR_OOM, "cudaMalloc of %zu bytes failed", (size_t)(bytes));        \
@@ -324,6 +329,21 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     default: return fail(LMOE_ERR_INVALID_ARG, "unknown region %d", region);
     }
     return LMOE_OK;
+}
+
+lmoe_status lmoe_debug_inject(int32_t what, int32_t arg)
+{
+    g_err.clear();
+    if (what == LMOE_INJECT_STALL_NEXT_GEMM) {
+        tc_debug_stall_next();
+        return LMOE_OK;
+    }
+    if (what == LMOE_INJECT_FAIL_ALLOC) {
+        if (arg < 1) return fail(LMOE_ERR_INVALID_ARG, "allocation index must be >= 1");
+        g_fail_alloc_at.store(arg);
+        return LMOE_OK;
+    }
+    return fail(LMOE_ERR_INVALID_ARG, "unknown injection %d", what);
 }
 
 lmoe_status lmoe_set_stage_events(lmoe_handle *h, void *const *events, int32_t n)

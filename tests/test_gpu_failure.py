@@ -1,0 +1,57 @@
+"""Failure detection without a GPU fault.
+
+The tensor-core GEMM bounds every wait; a test hook makes one GEMM's MMA warp
+wait on a barrier that nothing signals, so that wait runs out.  The forward
+must report LMOE_ERR_DEVICE_TIMEOUT through the device status word, and the
+context must stay usable: the next forward is correct.  An injected
+allocation failure in lmoe_create must return LMOE_ERR_OOM and leave the
+process able to create layers.
+"""
+import pytest
+import torch
+
+import lmoe_inputs as li
+from parity import rel_err
+
+pytestmark = pytest.mark.gpu
+
+W = li.custom("failure", 256, 256, 128, 256, 16, 4, 256, dtype="bf16", seed=41)
+
+
+def test_bounded_wait_runs_out_and_is_reported():
+    import latent_space_routed_b200 as lm
+    weights = {k: v.cuda() for k, v in li.weights(W).items()}
+    layer = lm.LatentMoE(lm.config_for(W), weights)
+    x = li.tokens(W).cuda()
+    ref = {k: v.clone() for k, v in layer(x).items()}
+    torch.cuda.synchronize()
+    layer.check_device(W.T)
+
+    lm.lmoe_debug_inject(lm.LMOE_INJECT_STALL_NEXT_GEMM)
+    layer(x)
+    with pytest.raises(lm.LmoeError) as ei:
+        layer.check_device(W.T)
+    assert ei.value.status == lm.LMOE_ERR_DEVICE_TIMEOUT
+
+    out = layer(x)                       # the context is still usable
+    torch.cuda.synchronize()
+    layer.check_device(W.T)
+    assert torch.equal(out["selected_experts"], ref["selected_experts"])
+    for key in ("output", "mixture_weights", "latent_routed_aggregate"):
+        assert rel_err(out[key].float().cpu().numpy(), ref[key].float().cpu().numpy()) == 0.0
+    layer.close()
+
+
+@pytest.mark.parametrize("which", [1, 3, 7])
+def test_injected_allocation_failure(which):
+    import latent_space_routed_b200 as lm
+    weights = {k: v.cuda() for k, v in li.weights(W).items()}
+    free0 = torch.cuda.mem_get_info()[0]
+    lm.lmoe_debug_inject(lm.LMOE_INJECT_FAIL_ALLOC, which)
+    with pytest.raises(lm.LmoeError) as ei:
+        lm.LatentMoE(lm.config_for(W), weights)
+    assert ei.value.status == lm.LMOE_ERR_OOM
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] >= free0 - (8 << 20)   # nothing of note leaked
+    layer = lm.LatentMoE(lm.config_for(W), weights)            # and creation works again
+    layer.close()
