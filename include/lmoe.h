@@ -118,7 +118,8 @@ LMOE_API lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int3
  * so the caller may free its weight copies afterwards.
  * INVALID_ARG: null pointer, non-positive size, l > d, k < 1 or k > E,
  *              n_shared != 2, eps < 0, unknown dtype/act.
- * UNSUPPORTED: d, l, f or f_shared not a multiple of 64, E > 1024, or (bf16
+ * UNSUPPORTED: d, l, f or f_shared not a multiple of 64, E > 1024, k > 64,
+ *              l > 8192, or (bf16
  *              tensor-core path) f or f_shared not a multiple of 128.
  * OOM / CUDA on allocation or launch failure (nothing is leaked). */
 LMOE_API lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *stream, lmoe_handle **out);

@@ -235,6 +235,10 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
 }
 
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all_but_one()
+{
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
@@ -536,6 +540,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
         const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * EPI_CHUNK_BYTES;
+        uint32_t ebuf_flip = 0;
         int local = 0;
         for (int item = group; item < total; item += ngroups, ++local) {
             const int acc = local & 1;
@@ -562,12 +567,22 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const bool rows_ok = (p.offsets || p.ksplit > 1) ? (chunk_row + 32 <= t.row_end) : true;
             auto emit = [&](const float *x, int col, int n) {
                 if (p.tma_store && rows_ok && n == 32) {
-                    if (lane == 0) bulk_wait_read_all();     // the previous store has read the buffer
+                    // bf16 chunks (2 KB) alternate between the two halves of the
+                    // warp's 4 KB buffer, so only the store before last must have
+                    // finished reading; fp32 chunks use the whole buffer
+                    uint32_t buf = ebuf;
+                    if (sizeof(TO) == 2) {
+                        buf += (uint32_t)(ebuf_flip & 1) * 2048u;
+                        ++ebuf_flip;
+                        if (lane == 0) bulk_wait_read_all_but_one();
+                    } else if (lane == 0) {
+                        bulk_wait_read_all();
+                    }
                     __syncwarp();
-                    stage_row(ebuf, lane, x, (TO *)nullptr);
+                    stage_row(buf, lane, x, (TO *)nullptr);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) tma_store_2d(&tmC, ebuf, col, (int)(slab + chunk_row));
+                    if (lane == 0) tma_store_2d(&tmC, buf, col, (int)(slab + chunk_row));
                 } else if (valid) {
                     store_n((TO *)p.epi.out + (slab + row) * p.epi.ldo + col, x, n);
                 }

@@ -95,9 +95,10 @@ constexpr int SPLIT_MAX = 16;
 
 // K splits for a dense GEMM of M rows, N columns (tiles of 128 x 256), nkb
 // k-blocks of 64.
-int plan_ksplit(const lmoe_handle *h, int64_t M, int64_t N, int64_t nkb)
+int plan_ksplit(const lmoe_handle *h, int64_t M, int64_t N, int64_t nkb, bool any_m = false)
 {
     if (!h->tc) return 1;
+    if (!any_m && M >= 256) return 1;   // 256-row pair tiles without a split do better there
     const int sms = tc_num_sms() > 0 ? tc_num_sms() : 148;
     const int64_t tiles = ((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN);
     if (tiles * 2 >= sms) return 1;
@@ -117,7 +118,7 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     const lmoe_config &c = h->cfg;
     const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
     SplitPlan sp;
-    sp.router = (h->tc && T > ROUTER_SMALL_MAX_T) ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK) : 1;
+    sp.router = (h->tc && T > ROUTER_SMALL_MAX_T) ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true) : 1;
     sp.down = plan_ksplit(h, T, c.l, c.d / TC_BK);
     sp.shared = plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
     sp.final_ = plan_ksplit(h, T, c.d, ld_hs / TC_BK);
@@ -177,6 +178,7 @@ lmoe_status check_config(const lmoe_config *c, bool *tc)
         return fail(LMOE_ERR_INVALID_ARG, "SiTU caps must be positive");
     if (c->gemm != 0 && c->gemm != 1) return fail(LMOE_ERR_INVALID_ARG, "gemm must be 0 or 1");
     if (c->E > 1024) return fail(LMOE_ERR_UNSUPPORTED, "E=%d > 1024", c->E);
+    if (c->l > 8192) return fail(LMOE_ERR_UNSUPPORTED, "l=%d > 8192", c->l);
     if (c->k > 64) return fail(LMOE_ERR_UNSUPPORTED, "k=%d > 64", c->k);
     if (c->d % 64 || c->l % 64 || c->f % 64 || c->f_shared % 64)
         return fail(LMOE_ERR_UNSUPPORTED, "d, l, f and f_shared must be multiples of 64");
@@ -456,9 +458,10 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     STAGE(1);
     LMOE_CUDA(launch_topk(r32, h->b, T, c.E, c.k, selected_experts, p32, mixture_weights, tk, blockhist, s));
     STAGE(2);
-    LMOE_CUDA(launch_scan(blockhist, nb, c.E, bm, counts, offsets, base, tile_off, s));
+    LMOE_CUDA(launch_scan(blockhist, nb, c.E, counts, base, s));
     STAGE(3);
-    LMOE_CUDA(launch_dispatch(selected_experts, p32, base, T, c.E, c.k, slot_of, perm_tok, perm_w, s));
+    LMOE_CUDA(launch_dispatch(selected_experts, p32, base, counts, T, c.E, c.k, bm, offsets, tile_off, slot_of,
+                              perm_tok, perm_w, s));
 
     // 5 z = x W_down^T, once per token
     GemmArgs gd = {};

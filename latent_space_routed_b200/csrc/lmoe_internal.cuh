@@ -99,13 +99,16 @@ constexpr int SIMT_BM = 64;
 constexpr int SIMT_BN = 128;
 
 // Router top-k + renormalisation + per-block expert histogram.
-constexpr int ROUTE_TPB = 128;  // tokens per block (also the dispatch block)
+constexpr int ROUTE_TPB = 32;   // tokens per counting block (also the dispatch block)
 cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
                         void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s);
-cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int bm, int32_t *counts, int32_t *offsets,
-                        int32_t *base, int32_t *tile_off, cudaStream_t s);
-cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, int64_t T, int E, int k,
-                            int32_t *slot_of, int32_t *perm_tok, float *perm_w, cudaStream_t s);
+// blockhist is expert-major [E][nb]; base (same layout) gets each block's
+// starting rank within its expert, counts[e] the expert totals.
+cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s);
+// Also writes offsets[E+1] and the m-tile prefix tile_off[E+1] for tiles of bm rows.
+cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, const int32_t *counts,
+                            int64_t T, int E, int k, int bm, int32_t *offsets, int32_t *tile_off, int32_t *slot_of,
+                            int32_t *perm_tok, float *perm_w, cudaStream_t s);
 cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
                                 cudaStream_t s);
 // Yp in the token dtype.

@@ -14,45 +14,92 @@
 namespace lmoe {
 namespace {
 
-// NT threads per token: 256 when tokens fill the GPU, 1024 for a few tokens
-// (more loads in flight per token).  The slot loads of a column are issued
-// eight at a time, then added in slot order.
-template <typename TT, int NT>
-__global__ void __launch_bounds__(NT)
+// Eight consecutive values as fp32 (16-byte loads) and back.
+__device__ __forceinline__ void load8(const bf16 *p, float *v)
+{
+    const uint4 q = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void load8(const float *p, float *v)
+{
+    const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void store8(bf16 *p, const float *v)
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ void store8(float *p, const float *v)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// One block per token, one thread per 8 consecutive latent columns: the
+// thread loads its columns from the token's k slot rows (four rows in flight
+// at a time), adds them in fp32 in slot order, and keeps u in registers for
+// the norm.
+template <typename TT>
+__global__ void __launch_bounds__(1024)
 combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_of, int l, int k, float eps,
                     TT *__restrict__ u_out, TT *__restrict__ hs, int64_t ld_hs, int64_t col0)
 {
-    extern __shared__ float u[];   // [l]
     __shared__ int slots[64];
-    __shared__ float red[NT / 32];
+    __shared__ float red[32];
     const int64_t t = blockIdx.x;
-    for (int j = threadIdx.x; j < k; j += NT) slots[j] = slot_of[t * k + j];
+    for (int j = threadIdx.x; j < k; j += blockDim.x) slots[j] = slot_of[t * k + j];
     __syncthreads();
-    float ss = 0.f;
-    for (int c = threadIdx.x; c < l; c += NT) {
-        float acc = 0.f;
+    const int c0 = threadIdx.x * 8;
+    const bool active = c0 < l;
+    float u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) {
         int j = 0;
-        for (; j + 8 <= k; j += 8) {
-            float v[8];
+        for (; j + 4 <= k; j += 4) {
+            float v[4][8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = to_f32(Yp[(int64_t)slots[j + i] * l + c]);
+            for (int q = 0; q < 4; ++q) load8(Yp + (int64_t)slots[j + q] * l + c0, v[q]);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc += v[i];
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) u[i] += v[q][i];
         }
-        for (; j < k; ++j) acc += to_f32(Yp[(int64_t)slots[j] * l + c]);
-        u[c] = acc;
-        u_out[t * l + c] = from_f32<TT>(acc);
-        ss += acc * acc;
+        for (; j < k; ++j) {
+            float v[8];
+            load8(Yp + (int64_t)slots[j] * l + c0, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] += v[i];
+        }
     }
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss += u[i] * u[i];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
     __syncthreads();
     float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) tot += red[w];
+    const int nw = blockDim.x >> 5;
+    for (int w = 0; w < nw; ++w) tot += red[w];
     const float inv = 1.0f / sqrtf(tot / (float)l + eps);
-    for (int c = threadIdx.x; c < l; c += NT) hs[t * ld_hs + col0 + c] = from_f32<TT>(u[c] * inv);
+    if (active) {
+        store8(u_out + t * l + c0, u);
+        float n[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) n[i] = u[i] * inv;
+        store8(hs + t * ld_hs + col0 + c0, n);
+    }
 }
 
 // P[e, 2F, K]: for every block q of ib rows, ib gate rows then the matching ib up rows.
@@ -115,7 +162,7 @@ splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, i
 {
     const int64_t m = blockIdx.y;
     const int nout = (MODE == EPI_GLU) ? N / 2 : N;
-    const int j0 = (blockIdx.x * 256 + threadIdx.x) * 4;
+    const int j0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (j0 >= nout) return;
     const int64_t slab = M * (int64_t)N;
     float r[4];
@@ -173,14 +220,16 @@ cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, in
     if (M == 0) return cudaSuccess;
     if (mode != EPI_SIGMOID && (N % 8 || ldo % 4 || (mode == EPI_GLU && ib % 4))) return cudaErrorInvalidValue;
     const int nout = mode == EPI_GLU ? N / 2 : N;
-    dim3 grid((unsigned)(((nout + 3) / 4 + 255) / 256), (unsigned)M);
+    const int nvec = (nout + 3) / 4;
+    const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
+    dim3 grid((unsigned)((nvec + threads - 1) / threads), (unsigned)M);
     if (mode == EPI_GLU)
-        splitk_reduce_kernel<EPI_GLU><<<grid, 256, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
+        splitk_reduce_kernel<EPI_GLU><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
     else if (mode == EPI_SIGMOID)
-        splitk_reduce_kernel<EPI_SIGMOID><<<grid, 256, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out,
+        splitk_reduce_kernel<EPI_SIGMOID><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out,
                                                                ldo);
     else
-        splitk_reduce_kernel<EPI_STORE><<<grid, 256, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
+        splitk_reduce_kernel<EPI_STORE><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
     return cudaGetLastError();
 }
 
@@ -188,24 +237,14 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s)
 {
     if (T == 0) return cudaSuccess;
-    if (k > 64) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(float) * l;
-    const bool few = T < 296;   // fewer tokens than two per SM: wide blocks
-    if (tok_bf16) {
-        if (few)
-            combine_norm_kernel<bf16, 1024><<<(unsigned)T, 1024, smem, s>>>((const bf16 *)Yp, slot_of, l, k, eps, (bf16 *)u_out,
-                                                                           (bf16 *)hs, ld_hs, col0);
-        else
-            combine_norm_kernel<bf16, 256><<<(unsigned)T, 256, smem, s>>>((const bf16 *)Yp, slot_of, l, k, eps, (bf16 *)u_out,
-                                                                         (bf16 *)hs, ld_hs, col0);
-    } else {
-        if (few)
-            combine_norm_kernel<float, 1024><<<(unsigned)T, 1024, smem, s>>>((const float *)Yp, slot_of, l, k, eps, (float *)u_out,
-                                                                            (float *)hs, ld_hs, col0);
-        else
-            combine_norm_kernel<float, 256><<<(unsigned)T, 256, smem, s>>>((const float *)Yp, slot_of, l, k, eps, (float *)u_out,
-                                                                          (float *)hs, ld_hs, col0);
-    }
+    if (k > 64 || l % 8 || l > 8192 || ld_hs % 8 || col0 % 8) return cudaErrorInvalidValue;
+    const int threads = ((l / 8 + 31) / 32) * 32;
+    if (tok_bf16)
+        combine_norm_kernel<bf16><<<(unsigned)T, threads, 0, s>>>((const bf16 *)Yp, slot_of, l, k, eps, (bf16 *)u_out,
+                                                                    (bf16 *)hs, ld_hs, col0);
+    else
+        combine_norm_kernel<float><<<(unsigned)T, threads, 0, s>>>((const float *)Yp, slot_of, l, k, eps,
+                                                                     (float *)u_out, (float *)hs, ld_hs, col0);
     return cudaGetLastError();
 }
 

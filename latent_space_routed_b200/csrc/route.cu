@@ -10,9 +10,10 @@
 // expert at most once, so the position of (t, j) with e = sel[t, j] is
 //   offsets[e] + #{t' < t : t' selected e}.
 // The top-k kernel (one warp per token) counts each expert's selections per
-// block of ROUTE_TPB tokens, one block scans the counts over blocks and
-// experts (scan kernel), and each block of ROUTE_TPB tokens ranks its tokens
-// within an expert with a bit mask and popcounts (dispatch kernel).
+// block of ROUTE_TPB tokens (expert-major), one block per expert scans its
+// counts over the token blocks (scan kernel), and each block of ROUTE_TPB
+// tokens scans the expert totals into offsets and ranks its tokens within an
+// expert with one bit word per expert and popcounts (dispatch kernel).
 // Integer-only, hence bit-exact and deterministic.
 #include <float.h>
 
@@ -28,7 +29,7 @@ template <typename TO>
 __global__ void __launch_bounds__(TOPK_WARPS * 32)
 topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t T, int E, int k,
             int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
-            int32_t *__restrict__ blockhist)
+            int32_t *__restrict__ blockhist, int nb)
 {
     extern __shared__ float smem[];
     __shared__ int chosen[TOPK_WARPS][KMAX];
@@ -66,84 +67,141 @@ topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t
     }
     float sum = 0.f;   // every lane sums in selection order: identical result
     for (int j = 0; j < k; ++j) sum += rw[chosen[warp][j]];
-    int32_t *hist = blockhist + (t / ROUTE_TPB) * E;
+    const int64_t tb = t / ROUTE_TPB;   // counts are expert-major: blockhist[e][token block]
     for (int j = lane; j < k; j += 32) {
         const int e = chosen[warp][j];
         const float p = rw[e] / sum;
         sel[t * k + j] = e;
         p32[t * k + j] = p;
         p_out[t * k + j] = from_f32<TO>(p);
-        atomicAdd(&hist[e], 1);
+        atomicAdd(&blockhist[(int64_t)e * nb + tb], 1);
     }
 }
 
-// One block: per-expert totals and per-(block, expert) starting positions.
-__global__ void __launch_bounds__(1024)
-scan_kernel(const int32_t *__restrict__ blockhist, int nb, int E, int bm, int32_t *__restrict__ counts,
-            int32_t *__restrict__ offsets, int32_t *__restrict__ base, int32_t *__restrict__ tile_off)
+// Exclusive scan of one int per thread over an NT-thread block; returns this
+// thread's exclusive prefix and the block total in *total.
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, int *s_warp, int *total)
 {
-    __shared__ int s_cnt[1024];
-    __shared__ int s_tiles[1024];
-    const int tid = threadIdx.x;
-    for (int e = tid; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int b = 0; b < nb; ++b) {
-            const int64_t i = (int64_t)b * E + e;
-            const int h = blockhist[i];
-            base[i] = run;
-            run += h;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < NT / 32 ? s_warp[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += o;
         }
-        counts[e] = run;
-        s_cnt[e] = run;
-        s_tiles[e] = (run + bm - 1) / bm;
+        if (lane < NT / 32) s_warp[lane] = w;   // inclusive over warps
     }
     __syncthreads();
-    if (tid == 0) {   // E <= 1024: a serial exclusive scan is a few microseconds at most
-        int acc = 0, tacc = 0;
-        for (int e = 0; e < E; ++e) {
-            offsets[e] = acc;
-            tile_off[e] = tacc;
-            const int c = s_cnt[e], tt = s_tiles[e];
-            s_cnt[e] = acc;
-            acc += c;
-            tacc += tt;
-        }
-        offsets[E] = acc;
-        tile_off[E] = tacc;
-    }
+    const int before = warp ? s_warp[warp - 1] : 0;
+    *total = s_warp[NT / 32 - 1];
     __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        const int off = s_cnt[e];
-        for (int b = 0; b < nb; ++b) base[(int64_t)b * E + e] += off;
-    }
+    return before + incl - v;
 }
 
-constexpr int WORDS = ROUTE_TPB / 32;
+// One block per expert: the expert's per-token-block counts (contiguous,
+// expert-major) are scanned into per-block starting ranks within the expert,
+// and their total is the expert's count.  Chunks of SCAN_NT * 4 token blocks
+// are scanned in order with a running carry.
+constexpr int SCAN_NT = 256;
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(SCAN_NT)
+scan_cols_kernel(const int32_t *__restrict__ blockhist, int nb, int32_t *__restrict__ base,
+                 int32_t *__restrict__ counts)
+{
+    __shared__ int s_warp[SCAN_NT / 32];
+    const int e = blockIdx.x;
+    const int32_t *h = blockhist + (int64_t)e * nb;
+    int32_t *o = base + (int64_t)e * nb;
+    int carry = 0;
+    for (int c0 = 0; c0 < nb; c0 += SCAN_NT * 4) {
+        const int i0 = c0 + threadIdx.x * 4;
+        int v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) v[q] = (i0 + q < nb) ? h[i0 + q] : 0;
+        int total = 0;
+        int run = carry + block_exclusive_scan<SCAN_NT>(v[0] + v[1] + v[2] + v[3], s_warp, &total);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (i0 + q < nb) o[i0 + q] = run;
+            run += v[q];
+        }
+        carry += total;
+    }
+    if (threadIdx.x == 0) counts[e] = carry;
+}
+
+// Dispatch for one block of ROUTE_TPB = 32 tokens.  Every block first scans
+// the expert counts into expert offsets (block 0 also publishes the offsets
+// and the m-tile prefix of the grouped GEMMs), marks which of its tokens chose
+// each expert in one bit word per expert, and places slot (t, j) with
+// e = sel[t, j] at offsets[e] + base[e][block] + #{earlier tokens of this
+// block that chose e}.
+constexpr int DISP_NT = 256;
+
+__global__ void __launch_bounds__(DISP_NT)
 dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, const int32_t *__restrict__ base,
-                int64_t T, int E, int k, int32_t *__restrict__ slot_of, int32_t *__restrict__ perm_tok,
-                float *__restrict__ perm_w)
+                const int32_t *__restrict__ counts, int64_t T, int E, int k, int nb, int bm,
+                int32_t *__restrict__ offsets, int32_t *__restrict__ tile_off, int32_t *__restrict__ slot_of,
+                int32_t *__restrict__ perm_tok, float *__restrict__ perm_w)
 {
-    extern __shared__ uint32_t bits[];   // [E][WORDS]: bit i of expert e = token t_begin+i chose e
+    extern __shared__ int s_dyn[];
+    int *s_off = s_dyn;                             // [E + 1]
+    uint32_t *bits = (uint32_t *)(s_dyn + E + 1);   // [E]
+    __shared__ int s_warp[DISP_NT / 32];
+    {   // expert offsets: E <= 1024 counts, four per thread
+        const int e0 = threadIdx.x * 4;
+        int v[4], tv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            v[q] = (e0 + q < E) ? counts[e0 + q] : 0;
+            tv[q] = (v[q] + bm - 1) / bm;
+        }
+        int total = 0;
+        int run = block_exclusive_scan<DISP_NT>(v[0] + v[1] + v[2] + v[3], s_warp, &total);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (e0 + q < E) s_off[e0 + q] = run;
+            run += v[q];
+        }
+        if (threadIdx.x == 0) s_off[E] = total;
+        if (blockIdx.x == 0) {   // uniform across the block
+            int ttot = 0;
+            int trun = block_exclusive_scan<DISP_NT>(tv[0] + tv[1] + tv[2] + tv[3], s_warp, &ttot);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if (e0 + q < E) tile_off[e0 + q] = trun;
+                trun += tv[q];
+            }
+            if (threadIdx.x == 0) tile_off[E] = ttot;
+        }
+    }
+    for (int i = threadIdx.x; i < E; i += DISP_NT) bits[i] = 0u;
+    __syncthreads();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i <= E; i += DISP_NT) offsets[i] = s_off[i];
     const int64_t t_begin = (int64_t)blockIdx.x * ROUTE_TPB;
     const int ntok = (int)min((int64_t)ROUTE_TPB, T - t_begin);
-    for (int i = threadIdx.x; i < E * WORDS; i += blockDim.x) bits[i] = 0u;
-    __syncthreads();
     const int n = ntok * k;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = threadIdx.x; i < n; i += DISP_NT) {
         const int tl = i / k;
-        const int e = sel[t_begin * k + i];
-        atomicOr(&bits[e * WORDS + (tl >> 5)], 1u << (tl & 31));
+        atomicOr(&bits[sel[t_begin * k + i]], 1u << tl);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    for (int i = threadIdx.x; i < n; i += DISP_NT) {
         const int tl = i / k;
         const int e = sel[t_begin * k + i];
-        const uint32_t *w = bits + e * WORDS;
-        int rank = __popc(w[tl >> 5] & ((1u << (tl & 31)) - 1u));
-        for (int q = 0; q < (tl >> 5); ++q) rank += __popc(w[q]);
-        const int pos = base[(int64_t)blockIdx.x * E + e] + rank;
+        const int rank = __popc(bits[e] & ((1u << tl) - 1u));
+        const int pos = s_off[e] + base[(int64_t)e * nb + blockIdx.x] + rank;
         slot_of[t_begin * k + i] = pos;
         perm_tok[pos] = (int32_t)(t_begin + tl);
         perm_w[pos] = p32[t_begin * k + i];
@@ -241,36 +299,38 @@ cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int
                         void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
 {
     if (k > KMAX) return cudaErrorInvalidValue;
-    const int64_t nhb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
-    cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nhb * E, s);
+    const int64_t nb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
+    cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nb * E, s);
     if (e != cudaSuccess) return e;
-    const unsigned nb = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
+    const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
     const size_t smem = sizeof(float) * 2 * TOPK_WARPS * E;
     if (out_bf16) {
         cudaFuncSetAttribute(topk_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        topk_kernel<bf16><<<nb, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (bf16 *)p_out, blockhist);
+        topk_kernel<bf16><<<nblk, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (bf16 *)p_out, blockhist,
+                                                                (int)nb);
     } else {
         cudaFuncSetAttribute(topk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        topk_kernel<float><<<nb, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (float *)p_out,
-                                                               blockhist);
+        topk_kernel<float><<<nblk, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (float *)p_out,
+                                                                 blockhist, (int)nb);
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int bm, int32_t *counts, int32_t *offsets,
-                        int32_t *base, int32_t *tile_off, cudaStream_t s)
+cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s)
 {
-    if (E > 1024) return cudaErrorInvalidValue;
-    scan_kernel<<<1, 1024, 0, s>>>(blockhist, nb, E, bm, counts, offsets, base, tile_off);
+    scan_cols_kernel<<<E, SCAN_NT, 0, s>>>(blockhist, nb, base, counts);
     return cudaGetLastError();
 }
 
-cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, int64_t T, int E, int k,
-                            int32_t *slot_of, int32_t *perm_tok, float *perm_w, cudaStream_t s)
+cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, const int32_t *counts,
+                            int64_t T, int E, int k, int bm, int32_t *offsets, int32_t *tile_off, int32_t *slot_of,
+                            int32_t *perm_tok, float *perm_w, cudaStream_t s)
 {
+    if (E > 1024) return cudaErrorInvalidValue;
     const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
-    const size_t smem = sizeof(uint32_t) * E * WORDS;
-    dispatch_kernel<<<nb, 256, smem, s>>>(sel, p32, base, T, E, k, slot_of, perm_tok, perm_w);
+    const size_t smem = sizeof(int) * (2 * (size_t)E + 1);
+    dispatch_kernel<<<nb, DISP_NT, smem, s>>>(sel, p32, base, counts, T, E, k, nb, bm, offsets, tile_off, slot_of,
+                                               perm_tok, perm_w);
     return cudaGetLastError();
 }
 
