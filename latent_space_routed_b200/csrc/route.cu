@@ -25,56 +25,95 @@ namespace {
 constexpr int TOPK_WARPS = 8;   // one token per warp, 8 tokens per block
 constexpr int KMAX = 64;
 
-template <typename TO>
+// "a before b": larger biased score first, equal scores to the lower index.
+__device__ __forceinline__ bool ahead(float va, int ia, float vb, int ib)
+{
+    return va > vb || (va == vb && ia < ib);
+}
+
+// Bitonic sort of a lane's N (score, expert) pairs into "ahead" order, in registers.
+template <int N>
+__device__ __forceinline__ void sort_lane(float (&v)[N], int (&ix)[N])
+{
+#pragma unroll
+    for (int kk = 2; kk <= N; kk <<= 1)
+#pragma unroll
+        for (int j = kk >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int m = i ^ j;
+                if (m > i) {
+                    const bool first_ahead = ahead(v[i], ix[i], v[m], ix[m]);
+                    if (((i & kk) == 0) != first_ahead) {
+                        const float tv = v[i]; v[i] = v[m]; v[m] = tv;
+                        const int ti = ix[i]; ix[i] = ix[m]; ix[m] = ti;
+                    }
+                }
+            }
+}
+
+// Top-k for one token per warp.  Lane L holds experts L, L + 32, ... (EPL of
+// them, padded with -inf), sorts them, and the k rounds are a tournament over
+// the 32 lane heads: a butterfly arg-max (ties to the lower index), then the
+// winning lane pops its head.  The raw scores of the chosen experts are
+// normalised by their sum (a fixed butterfly order, so the result does not
+// depend on timing).
+template <typename TO, int EPL>
 __global__ void __launch_bounds__(TOPK_WARPS * 32)
 topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t T, int E, int k,
             int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
             int32_t *__restrict__ blockhist, int nb)
 {
-    extern __shared__ float smem[];
-    __shared__ int chosen[TOPK_WARPS][KMAX];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float *sw = smem + warp * 2 * E;   // biased scores of this warp's token (taken -> -inf)
-    float *rw = sw + E;                // raw scores
     const int64_t t = (int64_t)blockIdx.x * TOPK_WARPS + warp;
     if (t >= T) return;
-    for (int e = lane; e < E; e += 32) {
-        const float rv = r[t * E + e];
-        rw[e] = rv;
-        // NaN / -inf map to -FLT_MAX so that a candidate always exists and
-        // the chosen index stays in range whatever the input holds
-        sw[e] = fmaxf(rv + bias[e], -FLT_MAX);
+    float v[EPL];
+    int ix[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        ix[i] = e;
+        // NaN / -inf map to -FLT_MAX so that a real candidate always beats the padding
+        v[i] = e < E ? fmaxf(r[t * E + e] + bias[e], -FLT_MAX) : -INFINITY;
     }
-    __syncwarp();
+    sort_lane<EPL>(v, ix);
+    int mine0 = 0, mine1 = 0;    // selection j kept by lane j % 32 (slot j / 32)
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int e = lane; e < E; e += 32) {
-            const float v = sw[e];
-            if (v > bv) { bv = v; bi = e; }   // ascending e: strict > keeps the lower index
-        }
+        float bv = v[0];
+        int bi = ix[0];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
             const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            if (ahead(ov, oi, bv, bi)) { bv = ov; bi = oi; }
         }
-        if (lane == 0) {
-            chosen[warp][j] = bi;
-            sw[bi] = -INFINITY;
+        if (lane == (bi & 31)) {            // the winner pops its head
+#pragma unroll
+            for (int i = 0; i + 1 < EPL; ++i) { v[i] = v[i + 1]; ix[i] = ix[i + 1]; }
+            v[EPL - 1] = -INFINITY;
+            ix[EPL - 1] = 0x7fffffff;
         }
-        __syncwarp();
+        if (lane == (j & 31)) {
+            if (j < 32) mine0 = bi; else mine1 = bi;
+        }
     }
-    float sum = 0.f;   // every lane sums in selection order: identical result
-    for (int j = 0; j < k; ++j) sum += rw[chosen[warp][j]];
+    const float r0 = lane < k ? r[t * E + mine0] : 0.f;
+    const float r1 = lane + 32 < k ? r[t * E + mine1] : 0.f;
+    float sum = r0 + r1;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     const int64_t tb = t / ROUTE_TPB;   // counts are expert-major: blockhist[e][token block]
-    for (int j = lane; j < k; j += 32) {
-        const int e = chosen[warp][j];
-        const float p = rw[e] / sum;
-        sel[t * k + j] = e;
-        p32[t * k + j] = p;
-        p_out[t * k + j] = from_f32<TO>(p);
-        atomicAdd(&blockhist[(int64_t)e * nb + tb], 1);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int j = lane + 32 * h;
+        if (j < k) {
+            const int e = h ? mine1 : mine0;
+            const float p = (h ? r1 : r0) / sum;
+            sel[t * k + j] = e;
+            p32[t * k + j] = p;
+            p_out[t * k + j] = from_f32<TO>(p);
+            atomicAdd(&blockhist[(int64_t)e * nb + tb], 1);
+        }
     }
 }
 
@@ -295,25 +334,41 @@ cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp
     return cudaGetLastError();
 }
 
+namespace {
+
+template <typename TO, int EPL>
+cudaError_t run_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32, void *p_out,
+                     int32_t *blockhist, int nb, cudaStream_t s)
+{
+    const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
+    topk_kernel<TO, EPL><<<nblk, TOPK_WARPS * 32, 0, s>>>(r, bias, T, E, k, sel, p32, (TO *)p_out, blockhist, nb);
+    return cudaGetLastError();
+}
+
+template <typename TO>
+cudaError_t run_topk_epl(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
+                         void *p_out, int32_t *blockhist, int nb, cudaStream_t s)
+{
+    const int epl = (E + 31) / 32;
+    if (epl <= 1) return run_topk<TO, 1>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+    if (epl <= 2) return run_topk<TO, 2>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+    if (epl <= 4) return run_topk<TO, 4>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+    if (epl <= 8) return run_topk<TO, 8>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+    if (epl <= 16) return run_topk<TO, 16>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+    return run_topk<TO, 32>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+}
+
+}  // namespace
+
 cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
                         void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
 {
-    if (k > KMAX) return cudaErrorInvalidValue;
+    if (k > KMAX || E > 1024) return cudaErrorInvalidValue;
     const int64_t nb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
     cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nb * E, s);
     if (e != cudaSuccess) return e;
-    const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
-    const size_t smem = sizeof(float) * 2 * TOPK_WARPS * E;
-    if (out_bf16) {
-        cudaFuncSetAttribute(topk_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        topk_kernel<bf16><<<nblk, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (bf16 *)p_out, blockhist,
-                                                                (int)nb);
-    } else {
-        cudaFuncSetAttribute(topk_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        topk_kernel<float><<<nblk, TOPK_WARPS * 32, smem, s>>>(r, bias, T, E, k, sel, p32, (float *)p_out,
-                                                                 blockhist, (int)nb);
-    }
-    return cudaGetLastError();
+    if (out_bf16) return run_topk_epl<bf16>(r, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
+    return run_topk_epl<float>(r, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
 }
 
 cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s)
