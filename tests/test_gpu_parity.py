@@ -95,6 +95,13 @@ def test_bf16_selection_extremes(E, k):
     run_parity(w)
 
 
+def test_bf16_many_rows_per_expert():
+    """About 400 slot rows per expert (the grouped GEMMs' larger-tile regime,
+    with ragged expert ends inside tiles); every row is compared."""
+    w = li.custom("many_rows", 1600, 256, 128, 256, 16, 4, 256, dtype="bf16", seed=24)
+    run_parity(w)
+
+
 def test_fp32_multi_tile_ragged():
     w = li.custom("multi_f32", 333, 256, 128, 128, 24, 5, 192, dtype="f32", seed=23)
     run_parity(w)
