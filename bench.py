@@ -291,7 +291,6 @@ def run_own(args, rank, world, local_rank):
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.fill_(float(i))                      # evict L2 between timed steps (untimed)
-        lm.lmoe_set_stage_events(layer.handle, arrays[i], ns)
         ev_a[i].record(stream)
         layer.forward_into(x, out)
         ev_b[i].record(stream)
@@ -299,14 +298,23 @@ def run_own(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
-    lm.lmoe_set_stage_events(layer.handle, None, 0)
     layer.check_device(T)
-
     step_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
     total_ms = max_over_ranks(sum(step_ms), dev)
+
+    # Per-stage breakdown: the same steps again with stage events set, under
+    # which the library runs every stage on one stream in order (no overlap).
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        lm.lmoe_set_stage_events(layer.handle, arrays[i], ns)
+        layer.forward_into(x, out)
+    torch.cuda.synchronize()
+    lm.lmoe_set_stage_events(layer.handle, None, 0)
+    layer.check_device(T)
     stage_ms = {}
     for si, name in enumerate(lm.STAGE_NAMES):
         stage_ms[name] = sum(ev_stage[i][si].elapsed_time(ev_stage[i][si + 1]) for i in range(args.steps)) / args.steps
+    serial_ms = sum(ev_stage[i][0].elapsed_time(ev_stage[i][ns - 1]) for i in range(args.steps)) / args.steps
 
     graph_ms = None
     if args.graph:
@@ -401,6 +409,8 @@ def run_own(args, rank, world, local_rank):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": roof, "layer_roofline": layer_roof,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "stages_note": "stages timed in a second pass with stage events set (one stream, no overlap)",
+            "serial_ms_per_step": round(serial_ms, 4),
             "cpu_baseline": cpu,
             "e2e": {"value": job_tokens_per_s(world, T, e2e_ms / args.steps), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},

@@ -143,6 +143,12 @@ LMOE_API lmoe_status lmoe_workspace_size(const lmoe_handle *h, int64_t T, size_t
  * Outputs must not overlap x, each other or the workspace.  T = 0 is a no-op.
  * Inputs must be finite.  Overlapping calls on one handle are allowed; calls
  * that share a workspace must be ordered on one stream.
+ * On the tensor-core path, when no stage events are set and the shared GEMM
+ * needs no K split (T >= 256 or so), the shared experts' gate/up GEMM runs on a
+ * stream owned by the handle: forked from `stream` after the down-projection
+ * and joined back into it before the final GEMM.  The call as a whole stays
+ * ordered on `stream` and can be captured into a CUDA graph from it; while such
+ * a capture is open, the handle's other forwards belong in that capture too.
  * INVALID_ARG for null pointers (T > 0) or T < 0; WORKSPACE if ws_bytes is too
  * small or misaligned; CUDA if a launch fails. */
 LMOE_API lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
@@ -181,7 +187,9 @@ LMOE_API lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream)
  * stage i, and events[LMOE_NUM_STAGES] after the last stage, so that the
  * caller can time every kernel with cudaEventElapsedTime.  n must be
  * LMOE_NUM_STAGES + 1, or 0 with events NULL to stop recording.  The array is
- * read at each forward, not copied: the caller keeps it alive. */
+ * read at each forward, not copied: the caller keeps it alive.  While events
+ * are set, every stage runs on the forward's stream in the order listed above
+ * (no side stream), so that each interval times one stage. */
 LMOE_API lmoe_status lmoe_set_stage_events(lmoe_handle *h, void *const *events, int32_t n);
 
 /* Test hooks for failure detection (no counterpart in the pages):

@@ -841,12 +841,14 @@ int tc_num_sms() { return g_num_sms; }
 
 void tc_debug_stall_next() { g_stall_next.store(1); }
 
-cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s, int ksplit)
+cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int cg, int32_t *status, cudaStream_t s, int ksplit)
 {
     GemmArgs r = g;
     r.B = Wr3;
     r.ldb = g.K;
-    return run<1>(ksplit > 1 ? EPI_SIGMOID_PARTIAL : EPI_SIGMOID, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+    const int mode = ksplit > 1 ? EPI_SIGMOID_PARTIAL : EPI_SIGMOID;
+    if (cg == 2) return run<2>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+    return run<1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
 }
 
 }  // namespace lmoe

@@ -30,9 +30,11 @@ int tc_num_sms();
 void tc_debug_stall_next();
 
 // Router r = sigmoid(x W_r^T) from the three-term bf16 split of fp32 W_r
-// (Wr3 = [3, E, d]): the three products accumulate into one fp32 TMEM tile.
-// ksplit > 1: the 3 d/64 k-blocks are split into ksplit ranges whose raw fp32
-// partial tiles go to g.epi.out slabs (launch_splitk_reduce applies sigmoid).
-cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int32_t *status, cudaStream_t s, int ksplit = 1);
+// (Wr3 = [3, E, d]): the three products accumulate into one fp32 TMEM tile,
+// on (128 cg)-row tiles.  ksplit > 1: the 3 d/64 k-blocks are split into
+// ksplit ranges whose raw fp32 partial tiles go to g.epi.out slabs (the top-k
+// kernel sums them and applies the sigmoid).
+cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int cg, int32_t *status, cudaStream_t s,
+                           int ksplit = 1);
 
 }  // namespace lmoe

@@ -14,11 +14,13 @@
 //   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
 //  10 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
 //  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "lmoe_internal.cuh"
@@ -54,7 +56,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
     size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, partial,
-        status;
+        partial_side, status;
     size_t total;
 };
 
@@ -81,6 +83,9 @@ struct lmoe_handle {
     void *Wgu_s;      // [4 f_s, d] interleaved (both shared experts as one of width 2 f_s)
     void *Wcat;       // [d, 2 f_s + l]
     void *const *stage_events;  // caller's cudaEvent_t[LMOE_NUM_STAGES + 1] or NULL
+    cudaStream_t side = nullptr;  // tensor-core path: the shared experts' gate/up runs here, overlapped
+    cudaEvent_t ev_fork = nullptr, ev_z = nullptr, ev_join = nullptr;
+    std::mutex fork_mutex;
 };
 
 namespace {
@@ -93,24 +98,29 @@ namespace {
 constexpr int64_t ROUTER_SMALL_MAX_T = 8;
 constexpr int SPLIT_MAX = 16;
 
-// K splits for a dense GEMM of M rows, N columns (tiles of 128 x 256), nkb
+// K splits for a dense GEMM of M rows, N columns on (128 cg) x 256 tiles, nkb
 // k-blocks of 64.
-int plan_ksplit(const lmoe_handle *h, int64_t M, int64_t N, int64_t nkb, bool any_m = false)
+int plan_ksplit(const lmoe_handle *h, int64_t M, int64_t N, int64_t nkb, bool any_m = false, int cg = 1)
 {
     if (!h->tc) return 1;
     if (!any_m && M >= 256) return 1;   // 256-row pair tiles without a split do better there
     const int sms = tc_num_sms() > 0 ? tc_num_sms() : 148;
-    const int64_t tiles = ((M + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN);
-    if (tiles * 2 >= sms) return 1;
-    int64_t ks = sms / tiles;
+    const int groups = sms / cg;
+    const int64_t tiles = ((M + TC_BM * cg - 1) / (TC_BM * cg)) * ((N + TC_BN - 1) / TC_BN);
+    if (tiles * 2 >= groups) return 1;
+    int64_t ks = groups / tiles;
     if (ks > nkb / 4) ks = nkb / 4;
     if (ks > SPLIT_MAX) ks = SPLIT_MAX;
     return ks >= 2 ? (int)ks : 1;
 }
 
+// Tile rows of the tensor-core router: CTA pairs from 256 tokens on.
+int router_cg(int64_t T) { return T >= 256 ? 2 : 1; }
+
 struct SplitPlan {
     int router, down, shared, final_;
-    size_t partial_floats;   // largest ks * T * N over the split GEMMs
+    size_t partial_floats;        // router and final GEMMs: largest ks * T * N
+    size_t partial_side_floats;   // down and shared gate/up GEMMs (the side stream's)
 };
 
 SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
@@ -118,21 +128,20 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     const lmoe_config &c = h->cfg;
     const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
     SplitPlan sp;
-    sp.router = (h->tc && T > ROUTER_SMALL_MAX_T) ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true) : 1;
+    sp.router = (h->tc && T > ROUTER_SMALL_MAX_T)
+                    ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true, router_cg(T)) : 1;
     sp.down = plan_ksplit(h, T, c.l, c.d / TC_BK);
     sp.shared = plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
     sp.final_ = plan_ksplit(h, T, c.d, ld_hs / TC_BK);
-    size_t m = 0;
-    auto upd = [&](int ks, int64_t n) {
-        if (ks > 1 && (size_t)ks * (size_t)n * (size_t)T > m) m = (size_t)ks * (size_t)n * (size_t)T;
-    };
-    upd(sp.router, c.E);
-    upd(sp.down, c.l);
-    upd(sp.shared, 4 * (int64_t)c.f_shared);
-    upd(sp.final_, c.d);
-    sp.partial_floats = m;
+    auto need = [&](int ks, int64_t n) -> size_t { return ks > 1 ? (size_t)ks * (size_t)n * (size_t)T : 0; };
+    sp.partial_floats = std::max(need(sp.router, c.E), need(sp.final_, c.d));
+    sp.partial_side_floats = std::max(need(sp.down, c.l), need(sp.shared, 4 * (int64_t)c.f_shared));
     return sp;
 }
+
+// The two-stream order: tensor-core path and no stage events (those time the
+// stages one after another on one stream).
+bool use_side_stream(const lmoe_handle *h) { return h->tc && h->side && !h->stage_events; }
 
 Layout plan(const lmoe_handle *h, int64_t T)
 {
@@ -157,7 +166,9 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.H = take(h->tb * S * c.f);
     L.Yp = take(h->tb * S * c.l);
     L.HS = take(h->tb * T * (2 * (int64_t)c.f_shared + c.l));
-    L.partial = take(sizeof(float) * plan_splits(h, T).partial_floats);
+    const SplitPlan sp = plan_splits(h, T);
+    L.partial = take(sizeof(float) * sp.partial_floats);
+    L.partial_side = take(sizeof(float) * sp.partial_side_floats);
     L.status = take(256);
     L.total = o;
     return L;
@@ -194,6 +205,10 @@ void free_handle(lmoe_handle *h)
     void *ptrs[] = {h->Wr, h->Wr3, h->b, h->Wdown, h->Wgu, h->D, h->Wgu_s, h->Wcat};
     for (void *p : ptrs)
         if (p) cudaFree(p);
+    if (h->side) cudaStreamDestroy(h->side);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_z) cudaEventDestroy(h->ev_z);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
     delete h;
 }
 
@@ -241,7 +256,6 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
     }
     cudaStream_t s = (cudaStream_t)stream;
     lmoe_handle *h = new lmoe_handle();
-    memset(h, 0, sizeof *h);
     h->cfg = *cfg;
     cudaGetDevice(&h->device);
     h->tc = tc;
@@ -289,6 +303,10 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
     if (tc) {
         ALLOC(h->Wr3, sizeof(bf16) * 3 * c.E * c.d);
         STEP(launch_split_router(h->Wr, h->Wr3, (int64_t)c.E * c.d, s));
+        STEP(cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+        STEP(cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming));
+        STEP(cudaEventCreateWithFlags(&h->ev_z, cudaEventDisableTiming));
+        STEP(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
     }
     STEP(cudaStreamSynchronize(s));
 #undef ALLOC
@@ -365,12 +383,13 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
     if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
     // status reset, router, histogram reset, top-k, scan, dispatch, down, permute, gate/up,
     // down+combine, norm, shared, final; plus one reduction per split-K GEMM
+    // other than the router's (which the top-k kernel reduces)
     if (T == 0) { *launches = 0; return LMOE_OK; }
     const lmoe_config &c = h->cfg;
     const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
     const SplitPlan sp = plan_splits(h, T);
     (void)ld_hs;
-    *launches = 13 + (sp.router > 1) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
+    *launches = 13 + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
     return LMOE_OK;
 }
 
@@ -429,99 +448,176 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
 
     LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
     const SplitPlan sp = plan_splits(h, T);
-    float *partial = (float *)(ws + L.partial);
-#define STAGE(i)                                                                                 \
-    if (h->stage_events) LMOE_CUDA(cudaEventRecord((cudaEvent_t)h->stage_events[i], s))
+    float *partial = (float *)(ws + L.partial);             // router, final
+    float *partial_side = (float *)(ws + L.partial_side);   // down, shared gate/up
+    const bool router_partial = h->tc && T > ROUTER_SMALL_MAX_T && sp.router > 1;
 
-    // 1 router: r = sigmoid(x W_r^T)
-    STAGE(0);
-    {
+    // ---- the stages, each launched on stream `q`
+    auto st_router = [&](cudaStream_t q) -> lmoe_status {   // r = sigmoid(x W_r^T)
         GemmArgs g = {};
         g.A = x; g.lda = c.d; g.M = (int)T; g.N = c.E; g.K = c.d;
         g.epi.out = r32; g.epi.ldo = c.E;
         if (h->tc && T <= ROUTER_SMALL_MAX_T) {
-            LMOE_CUDA(launch_router_small((const bf16 *)x, h->Wr, T, c.E, c.d, r32, s));
-        } else if (h->tc && sp.router > 1) {
+            LMOE_CUDA(launch_router_small((const bf16 *)x, h->Wr, T, c.E, c.d, r32, q));
+        } else if (router_partial) {
+            // raw logits in split-K slabs; the top-k kernel sums them and applies the sigmoid
             GemmArgs gp = g;
             gp.epi.out = partial;
             gp.epi.ldo = c.E;
-            LMOE_CUDA(tc_gemm_router(h->Wr3, gp, status, s, sp.router));
-            LMOE_CUDA(launch_splitk_reduce(partial, sp.router, T, c.E, EPI_SIGMOID, 0, 0.f, 0.f, 0, r32, c.E, s));
+            LMOE_CUDA(tc_gemm_router(h->Wr3, gp, router_cg(T), status, q, sp.router));
         } else if (h->tc) {
-            LMOE_CUDA(tc_gemm_router(h->Wr3, g, status, s));
+            LMOE_CUDA(tc_gemm_router(h->Wr3, g, router_cg(T), status, q));
         } else {
             g.B = h->Wr; g.ldb = c.d;
-            LMOE_CUDA(launch_simt_gemm(EPI_SIGMOID, tk, 0, 0, g, 0, s));
+            LMOE_CUDA(launch_simt_gemm(EPI_SIGMOID, tk, 0, 0, g, 0, q));
         }
-    }
-    // 2-4 selection and dispatch
-    STAGE(1);
-    LMOE_CUDA(launch_topk(r32, h->b, T, c.E, c.k, selected_experts, p32, mixture_weights, tk, blockhist, s));
-    STAGE(2);
-    LMOE_CUDA(launch_scan(blockhist, nb, c.E, counts, base, s));
-    STAGE(3);
-    LMOE_CUDA(launch_dispatch(selected_experts, p32, base, counts, T, c.E, c.k, bm, offsets, tile_off, slot_of,
-                              perm_tok, perm_w, s));
+        return LMOE_OK;
+    };
+    auto st_topk = [&](cudaStream_t q) -> lmoe_status {
+        LMOE_CUDA(launch_topk(router_partial ? partial : r32, router_partial ? sp.router : 0, r32, h->b, T, c.E, c.k,
+                              selected_experts, p32, mixture_weights, tk, blockhist, q));
+        return LMOE_OK;
+    };
+    auto st_scan = [&](cudaStream_t q) -> lmoe_status {
+        LMOE_CUDA(launch_scan(blockhist, nb, c.E, counts, base, q));
+        return LMOE_OK;
+    };
+    auto st_dispatch = [&](cudaStream_t q) -> lmoe_status {
+        LMOE_CUDA(launch_dispatch(selected_experts, p32, base, counts, T, c.E, c.k, bm, offsets, tile_off, slot_of,
+                                  perm_tok, perm_w, q));
+        return LMOE_OK;
+    };
 
-    // 5 z = x W_down^T, once per token
+    // z = x W_down^T, once per token
     GemmArgs gd = {};
     gd.A = x; gd.lda = c.d; gd.B = h->Wdown; gd.ldb = c.d; gd.M = (int)T; gd.N = c.l; gd.K = c.d;
     gd.epi.out = z; gd.epi.ldo = c.l;
-    // 6 per expert h = act(G z, U z) on the slot rows Zp[m] = z[perm_tok[m]]
+    // per expert h = act(G z, U z) on the slot rows Zp[m] = z[perm_tok[m]]
     GemmArgs gu = {};
     gu.A = Zp; gu.lda = c.l; gu.B = h->Wgu; gu.ldb = c.l; gu.b_group_stride = 2 * (int64_t)c.f * c.l;
     gu.M = (int)S; gu.N = 2 * c.f; gu.K = c.l; gu.offsets = offsets; gu.tile_off = tile_off; gu.E = c.E;
     gu.epi.out = H; gu.epi.ldo = c.f; gu.epi.act = c.act; gu.epi.gate_cap = c.gate_cap; gu.epi.up_cap = c.up_cap;
     gu.epi.ib = h->ib;
-    // 7 per expert Y = p (h D^T)
+    // per expert Y = p (h D^T)
     GemmArgs gc = {};
     gc.A = H; gc.lda = c.f; gc.B = h->D; gc.ldb = c.f; gc.b_group_stride = (int64_t)c.l * c.f;
     gc.M = (int)S; gc.N = c.l; gc.K = c.f; gc.offsets = offsets; gc.tile_off = tile_off; gc.E = c.E;
     gc.epi.out = Yp; gc.epi.ldo = c.l; gc.epi.row_w = perm_w;
-    // 9 shared experts' hidden, both as one expert of width 2 f_s
+    // shared experts' hidden, both as one expert of width 2 f_s
     GemmArgs gs = {};
     gs.A = x; gs.lda = c.d; gs.B = h->Wgu_s; gs.ldb = c.d; gs.M = (int)T; gs.N = 4 * c.f_shared; gs.K = c.d;
     gs.epi.out = HS; gs.epi.ldo = ld_hs; gs.epi.act = c.act; gs.epi.gate_cap = c.gate_cap;
     gs.epi.up_cap = c.up_cap; gs.epi.ib = h->ib;
-    // 10 y = [h_s | n] [D_s1 | D_s2 | W_up]^T
+    // y = [h_s | n] [D_s1 | D_s2 | W_up]^T
     GemmArgs gf = {};
     gf.A = HS; gf.lda = ld_hs; gf.B = h->Wcat; gf.ldb = ld_hs; gf.M = (int)T; gf.N = c.d; gf.K = (int)ld_hs;
     gf.epi.out = output; gf.epi.ldo = c.d;
 
     // Dense tensor-core GEMM, split along K per the plan.
-    auto dense_tc = [&](int mode, const GemmArgs &g, int ks) -> cudaError_t {
-        if (ks <= 1) return tc_gemm(mode, g, 0, cg_dense, status, s);
+    auto dense_tc = [&](int mode, const GemmArgs &g, int ks, float *part, cudaStream_t q) -> cudaError_t {
+        if (ks <= 1) return tc_gemm(mode, g, 0, cg_dense, status, q);
         GemmArgs gp = g;
-        gp.epi.out = partial;
+        gp.epi.out = part;
         gp.epi.ldo = g.N;
-        cudaError_t e = tc_gemm(EPI_STORE_F32, gp, 0, 1, status, s, ks);
+        cudaError_t e = tc_gemm(EPI_STORE_F32, gp, 0, 1, status, q, ks);
         if (e != cudaSuccess) return e;
-        return launch_splitk_reduce(partial, ks, g.M, g.N, mode, g.epi.act, g.epi.gate_cap, g.epi.up_cap, TC_BN / 2,
-                                    g.epi.out, g.epi.ldo, s);
+        return launch_splitk_reduce(part, ks, g.M, g.N, mode, g.epi.act, g.epi.gate_cap, g.epi.up_cap, TC_BN / 2,
+                                    g.epi.out, g.epi.ldo, q);
     };
-    STAGE(4);
-    if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down));
-    else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, s));
-    STAGE(5);
-    LMOE_CUDA(launch_permute_rows(z, perm_tok, Zp, S, c.l, (int)h->tb, s));
-    STAGE(6);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, cg_grouped, status, s));
-    else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, s));
-    STAGE(7);
-    if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, cg_grouped, status, s));
-    else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, tk, gc, max_mtiles, s));
-    // 8 u, RMSNorm(u) into the columns after the shared hidden
-    STAGE(8);
-    LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
-                                  2 * (int64_t)c.f_shared, tk, s));
-    STAGE(9);
-    if (h->tc) LMOE_CUDA(dense_tc(EPI_GLU, gs, sp.shared));
-    else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, s));
-    STAGE(10);
-    if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gf, sp.final_));
-    else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, s));
-    STAGE(LMOE_NUM_STAGES);
+    auto st_down = [&](cudaStream_t q) -> lmoe_status {
+        if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down, partial_side, q));
+        else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, q));
+        return LMOE_OK;
+    };
+    auto st_permute = [&](cudaStream_t q) -> lmoe_status {
+        LMOE_CUDA(launch_permute_rows(z, perm_tok, Zp, S, c.l, (int)h->tb, q));
+        return LMOE_OK;
+    };
+    auto st_gate_up = [&](cudaStream_t q) -> lmoe_status {
+        if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, cg_grouped, status, q));
+        else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, q));
+        return LMOE_OK;
+    };
+    auto st_down_combine = [&](cudaStream_t q) -> lmoe_status {
+        if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, cg_grouped, status, q));
+        else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, tk, gc, max_mtiles, q));
+        return LMOE_OK;
+    };
+    auto st_combine_norm = [&](cudaStream_t q) -> lmoe_status {   // u, RMSNorm(u) after the shared hidden
+        LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
+                                      2 * (int64_t)c.f_shared, tk, q));
+        return LMOE_OK;
+    };
+    auto st_shared = [&](cudaStream_t q) -> lmoe_status {
+        if (h->tc) LMOE_CUDA(dense_tc(EPI_GLU, gs, sp.shared, partial_side, q));
+        else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, q));
+        return LMOE_OK;
+    };
+    auto st_final = [&](cudaStream_t q) -> lmoe_status {
+        if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gf, sp.final_, partial, q));
+        else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, q));
+        return LMOE_OK;
+    };
+#define RUN(call)                                                                                \
+    do {                                                                                         \
+        const lmoe_status st_ = (call);                                                          \
+        if (st_ != LMOE_OK) return st_;                                                          \
+    } while (0)
+
+    if (!use_side_stream(h)) {
+        // One stream, in the order of the stage names; with stage events set,
+        // event i is recorded before stage i and event LMOE_NUM_STAGES after the last.
+#define STAGE(i)                                                                                 \
+    if (h->stage_events) LMOE_CUDA(cudaEventRecord((cudaEvent_t)h->stage_events[i], s))
+        STAGE(0); RUN(st_router(s));
+        STAGE(1); RUN(st_topk(s));
+        STAGE(2); RUN(st_scan(s));
+        STAGE(3); RUN(st_dispatch(s));
+        STAGE(4); RUN(st_down(s));
+        STAGE(5); RUN(st_permute(s));
+        STAGE(6); RUN(st_gate_up(s));
+        STAGE(7); RUN(st_down_combine(s));
+        STAGE(8); RUN(st_combine_norm(s));
+        STAGE(9); RUN(st_shared(s));
+        STAGE(10); RUN(st_final(s));
+        STAGE(LMOE_NUM_STAGES);
 #undef STAGE
+        return LMOE_OK;
+    }
+
+    // Two streams: the down-projection and the shared experts' gate/up GEMM
+    // need only x, so they run on the handle's side stream (the down GEMM
+    // first, beside the router GEMM, neither of which fills the GPU alone)
+    // while the caller's stream does the router and the latency-bound routing
+    // steps (top-k, scan, dispatch, permute), whose blocks fit beside the GEMM
+    // blocks on the same SMs.  The caller's stream waits for z before the
+    // permute, and for the shared GEMM before the routed gate/up GEMM: the
+    // routed GEMMs then start with every SM free, as their static tile
+    // schedule wants.
+    {
+        // record + wait as one step, so that a forward from another host thread
+        // cannot slip its own record in between
+        std::lock_guard<std::mutex> lock(h->fork_mutex);
+        LMOE_CUDA(cudaEventRecord(h->ev_fork, s));
+        LMOE_CUDA(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
+        RUN(st_down(h->side));
+        LMOE_CUDA(cudaEventRecord(h->ev_z, h->side));
+        RUN(st_shared(h->side));
+        LMOE_CUDA(cudaEventRecord(h->ev_join, h->side));
+    }
+    RUN(st_router(s));
+    RUN(st_topk(s));
+    RUN(st_scan(s));
+    RUN(st_dispatch(s));
+    // a later record on the in-order side stream covers this forward's GEMMs too
+    LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_z, 0));
+    RUN(st_permute(s));
+    LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
+    RUN(st_gate_up(s));
+    RUN(st_down_combine(s));
+    RUN(st_combine_norm(s));
+    RUN(st_final(s));
+#undef RUN
     return LMOE_OK;
 }
 

@@ -100,8 +100,11 @@ constexpr int SIMT_BN = 128;
 
 // Router top-k + renormalisation + per-block expert histogram.
 constexpr int ROUTE_TPB = 32;   // tokens per counting block (also the dispatch block)
-cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
-                        void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s);
+// nsplit = 0: r_in is r [T, E]; nsplit > 0: r_in holds nsplit fp32 partial
+// slabs [nsplit, T, E] of the router logits, summed in order, put through the
+// sigmoid and written to r_out [T, E].
+cudaError_t launch_topk(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
+                        int32_t *sel, float *p32, void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s);
 // blockhist is expert-major [E][nb]; base (same layout) gets each block's
 // starting rank within its expert, counts[e] the expert totals.
 cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s);

@@ -52,16 +52,31 @@ __device__ __forceinline__ void sort_lane(float (&v)[N], int (&ix)[N])
             }
 }
 
+// Order-preserving 32-bit key of a score: a > b as floats exactly when
+// key(a) > key(b) as unsigned integers (for -0 and +0 alike only if the caller
+// made -0 into +0, which it does).
+__device__ __forceinline__ uint32_t score_key(float v)
+{
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Top-k for one token per warp.  Lane L holds experts L, L + 32, ... (EPL of
 // them, padded with -inf), sorts them, and the k rounds are a tournament over
-// the 32 lane heads: a butterfly arg-max (ties to the lower index), then the
-// winning lane pops its head.  The raw scores of the chosen experts are
-// normalised by their sum (a fixed butterfly order, so the result does not
-// depend on timing).
+// the 32 lane heads: the largest head score (one warp max-reduction over the
+// score keys), then the lowest expert index among the heads with that score
+// (one min-reduction), so equal scores go to the lower index; the winning lane
+// pops its head.  The raw scores of the chosen experts are normalised by their
+// sum (a fixed butterfly order, so the result does not depend on timing).
+//
+// nsplit = 0: r_in holds the router scores r [T, E].  nsplit > 0: r_in holds
+// nsplit fp32 partial slabs [nsplit, T, E] of the router logits (split-K
+// GEMM); the kernel sums them in slab order, applies the sigmoid and writes r
+// to r_out.
 template <typename TO, int EPL>
 __global__ void __launch_bounds__(TOPK_WARPS * 32)
-topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t T, int E, int k,
-            int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
+topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const float *__restrict__ bias, int64_t T,
+            int E, int k, int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
             int32_t *__restrict__ blockhist, int nb)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -73,20 +88,27 @@ topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t
     for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
         ix[i] = e;
-        // NaN / -inf map to -FLT_MAX so that a real candidate always beats the padding
-        v[i] = e < E ? fmaxf(r[t * E + e] + bias[e], -FLT_MAX) : -INFINITY;
+        float r = 0.f;
+        if (e < E) {
+            if (nsplit == 0) {
+                r = r_in[t * E + e];
+            } else {
+                float a = 0.f;
+                for (int q = 0; q < nsplit; ++q) a += r_in[((int64_t)q * T + t) * E + e];
+                r = sigmoidf_(a);
+                r_out[t * E + e] = r;
+            }
+        }
+        // NaN / -inf map to -FLT_MAX so that a real candidate always beats the
+        // padding; adding +0 turns -0 into +0, so equal scores get equal keys
+        v[i] = e < E ? fmaxf(r + bias[e], -FLT_MAX) + 0.0f : -INFINITY;
     }
     sort_lane<EPL>(v, ix);
     int mine0 = 0, mine1 = 0;    // selection j kept by lane j % 32 (slot j / 32)
     for (int j = 0; j < k; ++j) {
-        float bv = v[0];
-        int bi = ix[0];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ahead(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
+        const uint32_t key = score_key(v[0]);
+        const uint32_t best = __reduce_max_sync(0xffffffffu, key);
+        const int bi = (int)__reduce_min_sync(0xffffffffu, key == best ? (uint32_t)ix[0] : 0xffffffffu);
         if (lane == (bi & 31)) {            // the winner pops its head
 #pragma unroll
             for (int i = 0; i + 1 < EPL; ++i) { v[i] = v[i + 1]; ix[i] = ix[i + 1]; }
@@ -97,8 +119,10 @@ topk_kernel(const float *__restrict__ r, const float *__restrict__ bias, int64_t
             if (j < 32) mine0 = bi; else mine1 = bi;
         }
     }
-    const float r0 = lane < k ? r[t * E + mine0] : 0.f;
-    const float r1 = lane + 32 < k ? r[t * E + mine1] : 0.f;
+    const float *rr = nsplit ? r_out : r_in;
+    if (nsplit) __syncwarp();               // r_out of this token, written by every lane, is visible
+    const float r0 = lane < k ? rr[t * E + mine0] : 0.f;
+    const float r1 = lane + 32 < k ? rr[t * E + mine1] : 0.f;
     float sum = r0 + r1;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -337,38 +361,42 @@ cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp
 namespace {
 
 template <typename TO, int EPL>
-cudaError_t run_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32, void *p_out,
-                     int32_t *blockhist, int nb, cudaStream_t s)
+cudaError_t run_topk(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
+                     int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, cudaStream_t s)
 {
     const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
-    topk_kernel<TO, EPL><<<nblk, TOPK_WARPS * 32, 0, s>>>(r, bias, T, E, k, sel, p32, (TO *)p_out, blockhist, nb);
+    topk_kernel<TO, EPL><<<nblk, TOPK_WARPS * 32, 0, s>>>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, (TO *)p_out,
+                                                         blockhist, nb);
     return cudaGetLastError();
 }
 
 template <typename TO>
-cudaError_t run_topk_epl(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
-                         void *p_out, int32_t *blockhist, int nb, cudaStream_t s)
+cudaError_t run_topk_epl(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
+                         int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, cudaStream_t s)
 {
     const int epl = (E + 31) / 32;
-    if (epl <= 1) return run_topk<TO, 1>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
-    if (epl <= 2) return run_topk<TO, 2>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
-    if (epl <= 4) return run_topk<TO, 4>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
-    if (epl <= 8) return run_topk<TO, 8>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
-    if (epl <= 16) return run_topk<TO, 16>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
-    return run_topk<TO, 32>(r, bias, T, E, k, sel, p32, p_out, blockhist, nb, s);
+#define LMOE_TOPK(N) run_topk<TO, N>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, nb, s)
+    if (epl <= 1) return LMOE_TOPK(1);
+    if (epl <= 2) return LMOE_TOPK(2);
+    if (epl <= 4) return LMOE_TOPK(4);
+    if (epl <= 8) return LMOE_TOPK(8);
+    if (epl <= 16) return LMOE_TOPK(16);
+    return LMOE_TOPK(32);
+#undef LMOE_TOPK
 }
 
 }  // namespace
 
-cudaError_t launch_topk(const float *r, const float *bias, int64_t T, int E, int k, int32_t *sel, float *p32,
-                        void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
+cudaError_t launch_topk(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
+                        int32_t *sel, float *p32, void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
 {
-    if (k > KMAX || E > 1024) return cudaErrorInvalidValue;
+    if (k > KMAX || E > 1024 || nsplit < 0) return cudaErrorInvalidValue;
     const int64_t nb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
     cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nb * E, s);
     if (e != cudaSuccess) return e;
-    if (out_bf16) return run_topk_epl<bf16>(r, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
-    return run_topk_epl<float>(r, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
+    if (out_bf16)
+        return run_topk_epl<bf16>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
+    return run_topk_epl<float>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
 }
 
 cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s)

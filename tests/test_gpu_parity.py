@@ -107,6 +107,39 @@ def test_fp32_multi_tile_ragged():
     run_parity(w)
 
 
+def test_equal_scores_go_to_the_lower_expert_index():
+    """Router rows repeated in groups of four (zero bias) give exactly equal
+    scores inside each group, so every row's top 6 is one whole group plus two
+    experts of the next one: the selection and its order must be the oracle's
+    (score descending, equal scores to the lower index), on rows whose distinct
+    score values near the cut are more than 1e-5 apart (fp32 vs fp64)."""
+    lm = _lm()
+    w = li.custom("ties", 256, 256, 128, 128, 64, 6, 128, dtype="bf16", seed=29)
+    W = dict(li.weights(w))
+    Wr = W["W_r"].clone()
+    for g in range(w.E // 4):
+        Wr[4 * g + 1:4 * g + 4] = Wr[4 * g]
+    W["W_r"] = Wr
+    W["b"] = torch.zeros_like(W["b"])
+    x = li.tokens(w)
+    layer = lm.LatentMoE(lm.config_for(w), {k: v.cuda() for k, v in W.items()})
+    for T in (5, w.T):                       # CUDA-core router, tensor-core router
+        out = layer(x[:T].cuda())
+        torch.cuda.synchronize()
+        ora = oracle.forward(x[:T], W, w.k, eps=w.eps)
+        sel_g = out["selected_experts"].cpu().numpy()
+        checked = 0
+        for t in range(T):
+            vals = np.unique(ora["scores"][t])[::-1][:4]     # distinct group scores, descending
+            if np.min(-np.diff(vals)) <= 1e-5:
+                continue
+            np.testing.assert_array_equal(sel_g[t], ora["selected_experts"][t])
+            assert sel_g[t][4] % 4 == 0 and sel_g[t][5] % 4 == 1   # the next group's two lowest
+            checked += 1
+        assert checked >= 0.9 * T
+    layer.close()
+
+
 # ---------------------------------------------------------------- stages
 def test_router_scores_and_dispatch_are_exact():
     """Scores r match the fp64 oracle to fp32 rounding; counts, offsets, slot
@@ -162,6 +195,54 @@ def test_deterministic_and_host_entry_matches():
     for key in a:
         assert torch.equal(a[key].cpu(), oh[key]), key
     assert layer.launch_count(w.T) > 0
+    layer.close()
+
+
+def test_side_stream_order_and_graph_capture_match_one_stream():
+    """T >= 256 runs the shared gate/up GEMM on the handle's side stream; with
+    stage events set every stage runs on the caller's stream.  Both orders, on
+    the default and on another stream, and a CUDA-graph replay of the forward
+    return the same bits."""
+    import ctypes
+    lm = _lm()
+    w = MULTI
+    x = li.tokens(w).cuda()
+    layer = _layer(w)
+    ref = {k: v.clone() for k, v in layer(x).items()}
+    ns = lm.LMOE_NUM_STAGES + 1
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(ns)]
+    for e in evs:
+        e.record()
+    torch.cuda.synchronize()
+    arr = (ctypes.c_void_p * ns)(*[e.cuda_event for e in evs])
+    lm.lmoe_set_stage_events(layer.handle, arr, ns)
+    one = {k: v.clone() for k, v in layer(x).items()}
+    torch.cuda.synchronize()
+    lm.lmoe_set_stage_events(layer.handle, None, 0)
+    for key in ref:
+        assert torch.equal(ref[key], one[key]), key
+
+    other = torch.cuda.Stream()
+    out = layer.empty_outputs(w.T)
+    layer.workspace(w.T)
+    other.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(other):
+        layer.forward_into(x, out, stream=other)
+    torch.cuda.current_stream().wait_stream(other)
+    torch.cuda.synchronize()
+    for key in ref:
+        assert torch.equal(ref[key], out[key]), key
+
+    gout = layer.empty_outputs(w.T)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.forward_into(x, gout, stream=torch.cuda.current_stream())
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    for key in ref:
+        assert torch.equal(ref[key], gout[key]), key
+    del graph
     layer.close()
 
 
