@@ -55,22 +55,30 @@ constexpr int THREADS = 320;   // 2 role warps + 8 epilogue warps
 constexpr int TMEM_COLS = 2 * BN;
 constexpr long long WAIT_LIMIT_CYCLES = 4000000000ll;   // about 2 s at 2 GHz
 constexpr int MAX_E = 1024;
-// Epilogue staging: one 32 x 32 output chunk (fp32 at most: 4 KB) per epilogue
-// warp, written swizzled and stored to global memory by TMA.
-constexpr int EPI_CHUNK_BYTES = 32 * 32 * 4;
-constexpr int EPI_STAGING = 8 * EPI_CHUNK_BYTES;
-
-template <int CG> struct Cfg {
+template <int CG> struct Tiles {
     static constexpr int A_BYTES = 128 * BK * 2;                // this CTA's 128 A rows
     static constexpr int B_BYTES = (BN / CG) * BK * 2;          // this CTA's share of B rows
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = CG == 2 ? 5 : 3;
     static constexpr int TILE_M = 128 * CG;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_STAGING + 256 +
-                                   2 * sizeof(int) * (MAX_E + 1);
     // kind::f16, D fp32, A and B bf16, both K-major, M = 128 CG, N = BN
     static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                       ((uint32_t)(TILE_M >> 4) << 24);
+};
+
+// Shared memory of one CTA for output elements of OB bytes: the expert tables,
+// one 32 x 32 output chunk of staging per epilogue warp (written swizzled and
+// stored by TMA), and as many operand stages as fit (at most 6): the weight
+// tiles of a grouped GEMM mostly come from HBM, and the ring is what keeps
+// their loads in flight.
+template <int CG, int OB> struct Cfg : Tiles<CG> {
+    static constexpr int EPI_CHUNK = 32 * 32 * OB;
+    static constexpr int EPI_STAGING = 8 * EPI_CHUNK;
+    static constexpr int TABLES = 2 * (int)sizeof(int) * (MAX_E + 1);
+    static constexpr int FIXED = 1024 + EPI_STAGING + 256 + TABLES;
+    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG>::STAGE_BYTES;
+    static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG>::STAGE_BYTES;
+    static_assert(STAGES >= 3, "operand ring too shallow");
 };
 
 // status codes (OR-ed together)
@@ -201,13 +209,13 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Cfg<CG>::IDESC), "r"(accumulate));
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Tiles<CG>::IDESC), "r"(accumulate));
     else
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Cfg<CG>::IDESC), "r"(accumulate));
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Tiles<CG>::IDESC), "r"(accumulate));
 }
 
 // Arrive on `bar` (the same offset in every CTA of the group) once all MMAs
@@ -235,10 +243,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
 }
 
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all_but_one()
-{
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
@@ -375,11 +379,11 @@ __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off,
             const int mid = (lo + hi + 1) >> 1;
             if (s_tile_off[mid] <= mt) lo = mid; else hi = mid - 1;
         }
-        t.row0 = (int64_t)s_offsets[lo] + (int64_t)(mt - s_tile_off[lo]) * Cfg<CG>::TILE_M;
+        t.row0 = (int64_t)s_offsets[lo] + (int64_t)(mt - s_tile_off[lo]) * Tiles<CG>::TILE_M;
         t.row_end = s_offsets[lo + 1];
         t.brow = (int64_t)lo * p.group_rows + t.n0;
     } else {
-        t.row0 = (int64_t)mt * Cfg<CG>::TILE_M;
+        t.row0 = (int64_t)mt * Tiles<CG>::TILE_M;
         t.row_end = p.M;
         t.brow = t.n0;
     }
@@ -391,19 +395,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const TcParams p)
 {
-    using C = Cfg<CG>;
+    using C = Cfg<CG, (int)sizeof(TO)>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;           // 1024-aligned stage ring
     uint8_t *gbase = smem_raw + (sbase - raw);
     const uint32_t epi_base = sbase + (uint32_t)(STAGES * C::STAGE_BYTES);   // 1024-aligned staging
-    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + (size_t)STAGES * C::STAGE_BYTES + EPI_STAGING);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + (size_t)STAGES * C::STAGE_BYTES + C::EPI_STAGING);
     // bars[0..S) full, [S..2S) empty, [2S..2S+2) acc full, [2S+2..2S+4) acc empty
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
     int *abort_flag = reinterpret_cast<int *>(tmem_holder + 1);
     int *drain_counts = abort_flag + 1;                      // [0] loads issued, [1] stages consumed
-    int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * C::STAGE_BYTES + EPI_STAGING + 256);
+    int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * C::STAGE_BYTES + C::EPI_STAGING + 256);
     int *s_offsets = s_tile_off + (MAX_E + 1);                                                 // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -539,8 +543,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // chunks c = 32 h + 64 i, so each warp drains half of its 32 rows' tile.
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
-        const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * EPI_CHUNK_BYTES;
-        uint32_t ebuf_flip = 0;
+        const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * C::EPI_CHUNK;
         int local = 0;
         for (int item = group; item < total; item += ngroups, ++local) {
             const int acc = local & 1;
@@ -567,18 +570,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const bool rows_ok = (p.offsets || p.ksplit > 1) ? (chunk_row + 32 <= t.row_end) : true;
             auto emit = [&](const float *x, int col, int n) {
                 if (p.tma_store && rows_ok && n == 32) {
-                    // bf16 chunks (2 KB) alternate between the two halves of the
-                    // warp's 4 KB buffer, so only the store before last must have
-                    // finished reading; fp32 chunks use the whole buffer
-                    uint32_t buf = ebuf;
-                    if (sizeof(TO) == 2) {
-                        buf += (uint32_t)(ebuf_flip & 1) * 2048u;
-                        ++ebuf_flip;
-                        if (lane == 0) bulk_wait_read_all_but_one();
-                    } else if (lane == 0) {
-                        bulk_wait_read_all();
-                    }
+                    // the warp's previous store must have finished reading its chunk
+                    if (lane == 0) bulk_wait_read_all();
                     __syncwarp();
+                    const uint32_t buf = ebuf;
                     stage_row(buf, lane, x, (TO *)nullptr);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
@@ -704,14 +699,14 @@ cudaError_t group_capacity(int *max_groups)
         return cudaSuccess;
     }
     auto kern = tc_gemm_kernel<MODE, TO, CG>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG>::SMEM);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG, (int)sizeof(TO)>::SMEM);
     if (e != cudaSuccess) return e;
     int groups = g_num_sms / CG;
     if (CG > 1) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(g_num_sms / CG * CG);
         q.blockDim = dim3(THREADS);
-        q.dynamicSmemBytes = Cfg<CG>::SMEM;
+        q.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO)>::SMEM;
         cudaLaunchAttribute qa[1];
         qa[0].id = cudaLaunchAttributeClusterDimension;
         qa[0].val.clusterDim.x = CG;
@@ -741,7 +736,7 @@ cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(groups * CG);
     lc.blockDim = dim3(THREADS);
-    lc.dynamicSmemBytes = Cfg<CG>::SMEM;
+    lc.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO)>::SMEM;
     lc.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -773,7 +768,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.offsets = g.offsets;
     p.tile_off = g.tile_off;
     p.E = g.E;
-    const int mtiles = g.offsets ? max_mtiles : (g.M + Cfg<CG>::TILE_M - 1) / Cfg<CG>::TILE_M;
+    const int mtiles = g.offsets ? max_mtiles : (g.M + Tiles<CG>::TILE_M - 1) / Tiles<CG>::TILE_M;
     p.max_tiles = mtiles * p.ntn;
     p.ksplit = ksplit < 1 ? 1 : ksplit;
     p.split_rows = g.M;
