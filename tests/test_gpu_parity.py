@@ -102,6 +102,19 @@ def test_bf16_many_rows_per_expert():
     run_parity(w)
 
 
+@pytest.mark.parametrize("shape", [
+    (1536, 512, 512, 128, 8, 2, 128),    # K = l = 512: eight A k-blocks, one n-tile per expert
+    (1200, 256, 64, 384, 16, 4, 128),    # K = 64: one A k-block, three n-tiles
+])
+def test_bf16_pair_tiles_edge_shapes(shape):
+    """Enough slot rows per expert for CTA-pair tiles, with the routed GEMMs'
+    K and n-tile counts at their edges (eight k-blocks and one n-tile; one
+    k-block and three n-tiles); every row is compared."""
+    w = li.custom("pair_edges", *shape, dtype="bf16", seed=25)
+    errs, _ = run_parity(w)
+    assert errs["output"] <= TOL["bf16"]
+
+
 def test_fp32_multi_tile_ragged():
     w = li.custom("multi_f32", 333, 256, 128, 128, 24, 5, 192, dtype="f32", seed=23)
     run_parity(w)
