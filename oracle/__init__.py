@@ -16,10 +16,16 @@ page:
 * ``fixed_cutoff_bias`` -- section "Quantile Balancing: measure now, use next
   step": the bias that leaves exactly ``target`` positive margins is minus the
   target-th largest margin (0-based after a descending sort).
+* ``qb_cutoff``, ``qb_margin_histogram``, ``qb_quantile_from_histogram`` --
+  the same section's statistics: the (k+1)-th biased score per token as the
+  cutoff, per-expert margin histograms, and the histogram estimate of the
+  quantile that fixed_cutoff_bias takes exactly.
 
 Pins (tests/test_oracle.py): the worked example and the shape examples of
 "Stable LatentMoE"; routed_example, the norm-order example, the latent_budget
-and fixed_cutoff_bias assertions of the cooking-agi page; brute-force top-k;
+and fixed_cutoff_bias assertions of the cooking-agi page; brute-force top-k
+and cutoffs; margin histograms against a direct count, and their quantile
+estimate within one bin of fixed_cutoff_bias;
 invariants (sum p = 1, k = E, bias shift, D scaling, row permutation,
 stacked shared experts, SiTU -> SwiGLU as the caps grow).  Nothing here is
 "parity unpinned".
@@ -228,6 +234,67 @@ def latent_budget(width, latent, intermediate, experts, top_k, tokens, item_byte
     return {"parameters": experts * expert + proj,
             "mac_per_token": top_k * expert + proj,
             "slot_bytes": 2 * tokens * top_k * latent * item_bytes}
+
+
+def qb_cutoff(s, k: int) -> np.ndarray:
+    """Quantile-Balancing cutoff per token (cooking-agi LatentMoE page, section
+    "Quantile Balancing: measure now, use next step"): the (k+1)-th largest
+    biased score s = r + b of each row of s [T, E]; -inf when k = E (nothing is
+    left unselected).  Works in s's own dtype (the selection is exact)."""
+    s = np.asarray(s)
+    T, E = s.shape
+    if not 1 <= k <= E:
+        raise ValueError("k must satisfy 1 <= k <= E")
+    if k == E:
+        return np.full(T, -np.inf, dtype=s.dtype)
+    return -np.partition(-s, k, axis=1)[:, k]
+
+
+def qb_margin_histogram(s, cutoff, bins: int, lo: float, hi: float) -> np.ndarray:
+    """Per-expert histogram [E, bins] (int64) of the margins m[t, e] = s[t, e] -
+    cutoff[t] (the page: expert-wise score margins against the current cutoff,
+    "global quantiles are approximated with histograms").  Bin j covers
+    [lo + j w, lo + (j + 1) w), w = (hi - lo) / bins; margins below lo count in
+    bin 0 and margins at or above hi in bin bins - 1.  The bin of a margin is
+    floor((m - lo) * (bins / (hi - lo))), each operation rounded in s's dtype
+    (pass fp32 scores to take the decision in fp32)."""
+    s = np.asarray(s)
+    dt = s.dtype.type
+    if bins < 1 or not hi > lo:
+        raise ValueError("need bins >= 1 and hi > lo")
+    T, E = s.shape
+    inv_w = dt(dt(bins) / (dt(hi) - dt(lo)))
+    hist = np.zeros((E, bins), np.int64)
+    for t in range(T):
+        for e in range(E):
+            m = dt(s[t, e] - dt(cutoff[t]))
+            x = dt(dt(m - dt(lo)) * inv_w)
+            j = 0 if x < 0 else (bins - 1 if x >= bins else int(np.floor(x)))
+            hist[e, j] += 1
+    return hist
+
+
+def qb_quantile_from_histogram(hist, target: int, lo: float, hi: float) -> np.ndarray:
+    """Per expert, the histogram estimate of the target-th largest margin
+    (0-based, the value fixed_cutoff_bias takes from sorted margins): scanning
+    bins from the top with C the count in the bins above bin j, the value lies
+    in the bin j with C <= target < C + h_j, and is placed at the upper edge of
+    that bin minus (target - C + 1/2) / h_j of its width (the centre of its
+    rank inside the bin).  Experts whose total count is <= target get lo.  The
+    next step's bias is b - q (fp64)."""
+    hist = np.asarray(hist, dtype=np.int64)
+    E, bins = hist.shape
+    w = (hi - lo) / bins
+    q = np.full(E, float(lo))
+    for e in range(E):
+        above = 0
+        for j in range(bins - 1, -1, -1):
+            h = int(hist[e, j])
+            if above <= target < above + h:
+                q[e] = lo + (j + 1) * w - w * (target - above + 0.5) / h
+                break
+            above += h
+    return q
 
 
 def fixed_cutoff_bias(margins, target):

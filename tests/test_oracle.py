@@ -169,6 +169,91 @@ def test_fixed_cutoff_bias():
         oracle.fixed_cutoff_bias([0.1, float("nan")], 1)
 
 
+# --------------------------------------------------------------------------
+# Quantile Balancing statistics (cooking-agi page, "Quantile Balancing:
+# measure now, use next step")
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("E,k", [(2, 1), (5, 2), (8, 3), (10, 9), (6, 6)])
+def test_qb_cutoff_is_the_next_score_after_the_top_k(E, k):
+    rng = np.random.default_rng(7 * E + k)
+    s = rng.standard_normal((100, E))
+    c = oracle.qb_cutoff(s, k)
+    for t in range(s.shape[0]):
+        ranked = sorted(s[t].tolist(), reverse=True)
+        assert c[t] == (ranked[k] if k < E else -math.inf)
+    # exactly the k selected experts have a positive margin (distinct scores)
+    if k < E:
+        assert np.all(((s - c[:, None]) > 0).sum(axis=1) == k)
+
+
+def test_qb_margin_histogram_matches_a_count_over_bin_intervals():
+    rng = np.random.default_rng(3)
+    T, E, bins, lo, hi = 300, 7, 16, -0.5, 0.5
+    s = rng.uniform(-0.9, 0.9, (T, E))
+    c = rng.uniform(-0.2, 0.2, T)
+    hist = oracle.qb_margin_histogram(s, c, bins, lo, hi)
+    w = (hi - lo) / bins
+    m = s - c[:, None]
+    for e in range(E):
+        for j in range(bins):
+            a, b = lo + j * w, lo + (j + 1) * w
+            inside = (m[:, e] >= a) & (m[:, e] < b)
+            if j == 0:
+                inside |= m[:, e] < lo
+            if j == bins - 1:
+                inside |= m[:, e] >= hi
+            assert hist[e, j] == int(inside.sum())
+    assert np.all(hist.sum(axis=1) == T)
+
+
+def test_qb_histogram_quantile_reproduces_the_fixed_cutoff_example():
+    """The page's margins [0.31, 0.16, 0.07, -0.08, -0.19, -0.34] with target 2:
+    the histogram estimate of the quantile lies within one bin of the exact
+    0.07, and the bias it gives leaves exactly two margins positive, as the
+    page's assertion does."""
+    q = _agi()["fixed_cutoff_bias"]
+    margins, target = q["margins"], q["target"]
+    lo, hi, bins = -1.0, 1.0, 200
+    hist = oracle.qb_margin_histogram(np.asarray(margins)[:, None], np.zeros(len(margins)), bins, lo, hi)
+    est = oracle.qb_quantile_from_histogram(hist, target, lo, hi)[0]
+    exact = -oracle.fixed_cutoff_bias(margins, target)
+    assert abs(est - exact) <= (hi - lo) / bins
+    assert sum(m - est > 0 for m in margins) == q["positive_after_bias"]
+
+
+@pytest.mark.parametrize("target", [0, 1, 17, 250, 499])
+def test_qb_histogram_quantile_within_one_bin_of_the_exact_one(target):
+    rng = np.random.default_rng(11 + target)
+    margins = rng.uniform(-0.8, 0.8, 500)
+    lo, hi, bins = -1.0, 1.0, 64
+    hist = oracle.qb_margin_histogram(margins[:, None], np.zeros(500), bins, lo, hi)
+    est = oracle.qb_quantile_from_histogram(hist, target, lo, hi)[0]
+    exact = sorted(margins.tolist(), reverse=True)[target]
+    assert abs(est - exact) <= (hi - lo) / bins
+
+
+def test_qb_six_tokens_three_experts_top1():
+    """The page's setting: six tokens, three experts, top-1, so six assignments
+    and a target of two per expert.  Per expert, the margins against the
+    current cutoff (the second score of each token) and the fixed-cutoff rule
+    leave exactly two positive margins each; the histogram estimate agrees
+    with it to one bin."""
+    s = np.array([[0.9, 0.2, 0.1], [0.8, 0.3, 0.0], [0.7, 0.6, 0.2],
+                  [0.1, 0.5, 0.4], [0.2, 0.1, 0.65], [0.3, 0.35, 0.05]])
+    k, E = 1, 3
+    target = s.shape[0] * k // E
+    assert target == 2
+    c = oracle.qb_cutoff(s, k)
+    m = s - c[:, None]
+    hist = oracle.qb_margin_histogram(s, c, 400, -1.0, 1.0)
+    est = oracle.qb_quantile_from_histogram(hist, target, -1.0, 1.0)
+    for e in range(E):
+        bias = oracle.fixed_cutoff_bias(m[:, e].tolist(), target)
+        assert int((m[:, e] + bias > 0).sum()) == target
+        assert abs(est[e] + bias) <= 2.0 / 400
+
+
 def test_oracle_parameter_count_matches_budget():
     """Count the weights the oracle consumes for the page's third budget row
     (d=128, l=64, f=256, 16 experts) and compare with the closed form."""
