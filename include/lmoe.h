@@ -175,6 +175,39 @@ LMOE_API lmoe_status lmoe_forward_host(lmoe_handle *h, const void *x_host, int64
  * Balancing", updates it between steps and freezes it for inference). */
 LMOE_API lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream);
 
+/* Quantile-Balancing statistics (cooking-agi LatentMoE page, section
+ * "Quantile Balancing: measure now, use next step": the current (k+1)-th biased
+ * score is the cutoff, expert-wise margins against it estimate the next bias,
+ * which takes effect the next step; global quantiles come from histograms).
+ *
+ * lmoe_qb_histogram: after an lmoe_forward of T tokens with `workspace` on the
+ * same stream, ADD the batch's margin histogram to hist [E, bins] (device
+ * int32, row-major, zeroed by the caller before the first batch; several
+ * batches, or an all-reduce over ranks, accumulate into it).  The margin of
+ * token t for expert e is m = (r[t, e] + b[e]) - cutoff[t] with r the router
+ * scores and cutoff[t] the token's (k+1)-th biased score (workspace region 11);
+ * its bin is computed in fp32 as x = (m - lo) * (bins / (hi - lo)): bin 0 if
+ * x < 0, bins - 1 if x >= bins, floor(x) otherwise.  Reads workspace regions 0
+ * and 11, which the next forward on that workspace overwrites.
+ * INVALID_ARG: NULL pointer, T < 0, bins outside [1, 2^20], lo or hi not
+ * finite, hi <= lo.  T = 0 adds nothing. */
+LMOE_API lmoe_status lmoe_qb_histogram(const lmoe_handle *h, const void *workspace, int64_t T, int32_t bins,
+                                       float lo, float hi, int32_t *hist, void *stream);
+
+/* lmoe_qb_bias_update: the next step's bias from an accumulated histogram, into
+ * bias_out [E] (device fp32; may not alias the handle's bias): per expert, the
+ * target-th largest margin (0-based; the page's fixed-cutoff rule takes it from
+ * sorted margins) is estimated from the histogram -- scanning bins from the
+ * top with C the count above bin j, it lies in the bin with C <= target <
+ * C + h_j, placed at that bin's upper edge minus (target - C + 1/2) / h_j of the
+ * bin width -- and bias_out[e] = b[e] - q_e (lo when the expert has no more
+ * than `target` margins).  Apply it with lmoe_set_bias before the next step.
+ * target is normally the batch's slots per expert, T k / E.
+ * INVALID_ARG: NULL pointer, bins outside [1, 2^20], lo or hi not finite,
+ * hi <= lo, target < 0. */
+LMOE_API lmoe_status lmoe_qb_bias_update(const lmoe_handle *h, const int32_t *hist, int32_t bins, float lo,
+                                         float hi, int64_t target, float *bias_out, void *stream);
+
 /* Stages of one forward, in launch order (for lmoe_set_stage_events):
  *  0 router GEMM, 1 top-k, 2 counting-sort scan, 3 dispatch, 4 down-projection
  *  GEMM, 5 copy of z to the expert-sorted slot rows, 6 routed gate/up GEMM,
@@ -217,7 +250,8 @@ LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t 
  * 4 slot index of (t, j) [T, k] int32; 5 token of each permuted slot [T*k]
  * int32; 6 latent rows z [T, l]; 7 routed hidden H [T*k, f] (slot order);
  * 8 p-weighted expert outputs [T*k, l] (token dtype); 9 [shared hidden | RMSNorm(u)]
- * [T, 2 f_shared + l]; 10 device status word (int32).
+ * [T, 2 f_shared + l]; 10 device status word (int32); 11 Quantile-Balancing
+ * cutoff [T] fp32 (each token's (k+1)-th biased score, -inf when k = E).
  * INVALID_ARG for an unknown region. */
 LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t region, size_t *offset,
                                   size_t *bytes);

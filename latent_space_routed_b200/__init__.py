@@ -30,10 +30,10 @@ STATUS_NAMES = {0: "LMOE_OK", 1: "LMOE_ERR_INVALID_ARG", 2: "LMOE_ERR_UNSUPPORTE
 
 # lmoe_workspace_region ids
 REGION = {"scores": 0, "p32": 1, "counts": 2, "offsets": 3, "slot_of": 4, "perm_tok": 5, "Z": 6, "H": 7,
-          "Y": 8, "HS": 9, "status": 10}
+          "Y": 8, "HS": 9, "status": 10, "cutoff": 11}
 
 EXPORTS = ("lmoe_config_from_base", "lmoe_create", "lmoe_workspace_size", "lmoe_forward", "lmoe_host_workspace_size",
-           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_debug_inject", "lmoe_set_bias", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
+           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_debug_inject", "lmoe_set_bias", "lmoe_qb_histogram", "lmoe_qb_bias_update", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
            "lmoe_last_error", "lmoe_destroy")
 
 
@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "lmoe_forward_noalloc": (I32, [P, P, I64, P, P, P, P, P]),
         "lmoe_debug_inject": (I32, [I32, I32]),
         "lmoe_set_bias": (I32, [P, P, P]),
+        "lmoe_qb_histogram": (I32, [P, P, I64, I32, ctypes.c_float, ctypes.c_float, P, P]),
+        "lmoe_qb_bias_update": (I32, [P, P, I32, ctypes.c_float, ctypes.c_float, I64, P, P]),
         "lmoe_set_stage_events": (I32, [P, P, I32]),
         "lmoe_launch_count": (I32, [P, I64, ctypes.POINTER(I32)]),
         "lmoe_workspace_region": (I32, [P, I64, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
@@ -176,6 +178,14 @@ def lmoe_forward_noalloc(h, x, T, output, selected_experts, mixture_weights, lat
 
 def lmoe_set_bias(h, b, stream=None):
     _check(_lib.lmoe_set_bias(h, _ptr(b), _stream(stream)))
+
+
+def lmoe_qb_histogram(h, workspace, T, bins, lo, hi, hist, stream=None):
+    _check(_lib.lmoe_qb_histogram(h, _ptr(workspace), T, bins, lo, hi, _ptr(hist), _stream(stream)))
+
+
+def lmoe_qb_bias_update(h, hist, bins, lo, hi, target, bias_out, stream=None):
+    _check(_lib.lmoe_qb_bias_update(h, _ptr(hist), bins, lo, hi, target, _ptr(bias_out), _stream(stream)))
 
 
 LMOE_NUM_STAGES = 11
@@ -296,6 +306,21 @@ class LatentMoE:
 
     def launch_count(self, T: int) -> int:
         return lmoe_launch_count(self.handle, T)
+
+    def set_bias(self, b: torch.Tensor, stream=None):
+        """Replace the selection bias with b [E] (device fp32)."""
+        lmoe_set_bias(self.handle, b, stream)
+
+    def qb_histogram(self, T: int, hist: torch.Tensor, bins: int, lo: float, hi: float, stream=None):
+        """Add the last forward's (T tokens) Quantile-Balancing margin histogram to hist [E, bins] int32."""
+        lmoe_qb_histogram(self.handle, self.workspace(T), T, bins, lo, hi, hist, stream)
+        return hist
+
+    def qb_bias_update(self, hist: torch.Tensor, bins: int, lo: float, hi: float, target: int, stream=None):
+        """The next step's bias [E] fp32 from an accumulated histogram (apply with set_bias)."""
+        out = torch.empty(self.cfg.E, dtype=torch.float32, device=self.device)
+        lmoe_qb_bias_update(self.handle, hist, bins, lo, hi, target, out, stream)
+        return out
 
 
 def config_for(workload, gemm: int = 0, act: int = LMOE_ACT_SWIGLU) -> lmoe_config:

@@ -15,6 +15,7 @@
 //  10 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
 //  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -56,7 +57,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
     size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, partial,
-        partial_side, status;
+        partial_side, cutoff, status;
     size_t total;
 };
 
@@ -169,6 +170,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     const SplitPlan sp = plan_splits(h, T);
     L.partial = take(sizeof(float) * sp.partial_floats);
     L.partial_side = take(sizeof(float) * sp.partial_side_floats);
+    L.cutoff = take(sizeof(float) * T);
     L.status = take(256);
     L.total = o;
     return L;
@@ -346,6 +348,7 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 8: *offset = L.Yp; *bytes = h->tb * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
     case 10: *offset = L.status; *bytes = sizeof(int32_t); break;
+    case 11: *offset = L.cutoff; *bytes = sizeof(float) * T; break;
     default: return fail(LMOE_ERR_INVALID_ARG, "unknown region %d", region);
     }
     return LMOE_OK;
@@ -398,6 +401,34 @@ lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream)
     g_err.clear();
     if (!h || !b) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
     LMOE_CUDA(cudaMemcpyAsync(h->b, b, sizeof(float) * h->cfg.E, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_qb_histogram(const lmoe_handle *h, const void *workspace, int64_t T, int32_t bins, float lo, float hi,
+                              int32_t *hist, void *stream)
+{
+    g_err.clear();
+    if (!h || !workspace || !hist) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
+    if (bins < 1 || bins > (1 << 20)) return fail(LMOE_ERR_INVALID_ARG, "bins=%d outside [1, 2^20]", bins);
+    if (!std::isfinite(lo) || !std::isfinite(hi) || !(hi > lo)) return fail(LMOE_ERR_INVALID_ARG, "need finite lo < hi");
+    if (T == 0) return LMOE_OK;
+    const Layout L = plan(h, T);
+    const char *ws = (const char *)workspace;
+    LMOE_CUDA(launch_qb_histogram((const float *)(ws + L.r32), h->b, (const float *)(ws + L.cutoff), T, h->cfg.E,
+                                  bins, lo, hi, hist, (cudaStream_t)stream));
+    return LMOE_OK;
+}
+
+lmoe_status lmoe_qb_bias_update(const lmoe_handle *h, const int32_t *hist, int32_t bins, float lo, float hi,
+                                int64_t target, float *bias_out, void *stream)
+{
+    g_err.clear();
+    if (!h || !hist || !bias_out) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (bins < 1 || bins > (1 << 20)) return fail(LMOE_ERR_INVALID_ARG, "bins=%d outside [1, 2^20]", bins);
+    if (!std::isfinite(lo) || !std::isfinite(hi) || !(hi > lo)) return fail(LMOE_ERR_INVALID_ARG, "need finite lo < hi");
+    if (target < 0) return fail(LMOE_ERR_INVALID_ARG, "target < 0");
+    LMOE_CUDA(launch_qb_bias_update(hist, h->b, h->cfg.E, bins, lo, hi, target, bias_out, (cudaStream_t)stream));
     return LMOE_OK;
 }
 
@@ -475,7 +506,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     };
     auto st_topk = [&](cudaStream_t q) -> lmoe_status {
         LMOE_CUDA(launch_topk(router_partial ? partial : r32, router_partial ? sp.router : 0, r32, h->b, T, c.E, c.k,
-                              selected_experts, p32, mixture_weights, tk, blockhist, q));
+                              selected_experts, p32, mixture_weights, tk, blockhist, (float *)(ws + L.cutoff), q));
         return LMOE_OK;
     };
     auto st_scan = [&](cudaStream_t q) -> lmoe_status {

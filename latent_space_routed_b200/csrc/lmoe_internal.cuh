@@ -102,9 +102,17 @@ constexpr int SIMT_BN = 128;
 constexpr int ROUTE_TPB = 32;   // tokens per counting block (also the dispatch block)
 // nsplit = 0: r_in is r [T, E]; nsplit > 0: r_in holds nsplit fp32 partial
 // slabs [nsplit, T, E] of the router logits, summed in order, put through the
-// sigmoid and written to r_out [T, E].
+// sigmoid and written to r_out [T, E].  cutoff [T] gets each token's (k+1)-th
+// biased score (-inf when k = E).
 cudaError_t launch_topk(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
-                        int32_t *sel, float *p32, void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s);
+                        int32_t *sel, float *p32, void *p_out, int out_bf16, int32_t *blockhist, float *cutoff,
+                        cudaStream_t s);
+// Quantile-Balancing statistics: add the margin histogram of T tokens to hist
+// [E, bins]; and the next bias b - q from an accumulated histogram.
+cudaError_t launch_qb_histogram(const float *r, const float *bias, const float *cutoff, int64_t T, int E, int bins,
+                                float lo, float hi, int32_t *hist, cudaStream_t s);
+cudaError_t launch_qb_bias_update(const int32_t *hist, const float *bias, int E, int bins, float lo, float hi,
+                                  int64_t target, float *bias_out, cudaStream_t s);
 // blockhist is expert-major [E][nb]; base (same layout) gets each block's
 // starting rank within its expert, counts[e] the expert totals.
 cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s);

@@ -77,7 +77,7 @@ template <typename TO, int EPL>
 __global__ void __launch_bounds__(TOPK_WARPS * 32)
 topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const float *__restrict__ bias, int64_t T,
             int E, int k, int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
-            int32_t *__restrict__ blockhist, int nb)
+            int32_t *__restrict__ blockhist, int nb, float *__restrict__ cutoff)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = (int64_t)blockIdx.x * TOPK_WARPS + warp;
@@ -118,6 +118,15 @@ topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const floa
         if (lane == (j & 31)) {
             if (j < 32) mine0 = bi; else mine1 = bi;
         }
+    }
+    // Quantile-Balancing cutoff: the (k+1)-th biased score, one more round
+    // (-inf when k = E leaves nothing unselected)
+    {
+        const uint32_t key = score_key(v[0]);
+        const uint32_t best = __reduce_max_sync(0xffffffffu, key);
+        const int bi = (int)__reduce_min_sync(0xffffffffu, key == best ? (uint32_t)ix[0] : 0xffffffffu);
+        const float cv = __shfl_sync(0xffffffffu, v[0], bi & 31);
+        if (lane == 0) cutoff[t] = k < E ? cv : -INFINITY;
     }
     const float *rr = nsplit ? r_out : r_in;
     if (nsplit) __syncwarp();               // r_out of this token, written by every lane, is visible
@@ -362,20 +371,21 @@ namespace {
 
 template <typename TO, int EPL>
 cudaError_t run_topk(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
-                     int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, cudaStream_t s)
+                     int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, float *cutoff, cudaStream_t s)
 {
     const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
     topk_kernel<TO, EPL><<<nblk, TOPK_WARPS * 32, 0, s>>>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, (TO *)p_out,
-                                                         blockhist, nb);
+                                                         blockhist, nb, cutoff);
     return cudaGetLastError();
 }
 
 template <typename TO>
 cudaError_t run_topk_epl(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
-                         int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, cudaStream_t s)
+                         int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, float *cutoff,
+                         cudaStream_t s)
 {
     const int epl = (E + 31) / 32;
-#define LMOE_TOPK(N) run_topk<TO, N>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, nb, s)
+#define LMOE_TOPK(N) run_topk<TO, N>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, nb, cutoff, s)
     if (epl <= 1) return LMOE_TOPK(1);
     if (epl <= 2) return LMOE_TOPK(2);
     if (epl <= 4) return LMOE_TOPK(4);
@@ -388,15 +398,16 @@ cudaError_t run_topk_epl(const float *r_in, int nsplit, float *r_out, const floa
 }  // namespace
 
 cudaError_t launch_topk(const float *r_in, int nsplit, float *r_out, const float *bias, int64_t T, int E, int k,
-                        int32_t *sel, float *p32, void *p_out, int out_bf16, int32_t *blockhist, cudaStream_t s)
+                        int32_t *sel, float *p32, void *p_out, int out_bf16, int32_t *blockhist, float *cutoff,
+                        cudaStream_t s)
 {
     if (k > KMAX || E > 1024 || nsplit < 0) return cudaErrorInvalidValue;
     const int64_t nb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
     cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nb * E, s);
     if (e != cudaSuccess) return e;
     if (out_bf16)
-        return run_topk_epl<bf16>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
-    return run_topk_epl<float>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, s);
+        return run_topk_epl<bf16>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, cutoff, s);
+    return run_topk_epl<float>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, cutoff, s);
 }
 
 cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s)
