@@ -85,13 +85,16 @@ def peaks():
 
 # ---------------------------------------------------------------- algorithmic model
 def layer_flops(w, T):
-    """2dE + 4dl + 6klf + 12 d f_s per token (router, projections, routed, shared)."""
-    return T * (2 * w.d * w.E + 4 * w.d * w.l + 6 * w.k * w.l * w.f + 12 * w.d * w.f_s)
+    """2dE + 4dl + 6klf + 12 d f_s per token (router, projections, routed, shared);
+    no projection term for the standard MoE (l = d, no W_down / W_up)."""
+    proj = 0 if w.standard else 4 * w.d * w.l
+    return T * (2 * w.d * w.E + proj + 6 * w.k * w.l * w.f + 12 * w.d * w.f_s)
 
 
 def layer_bytes(w, T, touched):
     B = w.item_bytes
-    weights = touched * 3 * w.l * w.f * B + 6 * w.d * w.f_s * B + 2 * w.d * w.l * B + 4 * w.d * w.E
+    proj = 0 if w.standard else 2 * w.d * w.l * B
+    weights = touched * 3 * w.l * w.f * B + 6 * w.d * w.f_s * B + proj + 4 * w.d * w.E
     io = T * w.d * B * 2 + T * w.k * (4 + B) + T * w.l * B
     return weights + io
 
@@ -99,19 +102,20 @@ def layer_bytes(w, T, touched):
 def stage_model(w, T, touched):
     """Per-kernel algorithmic (flops, bytes): operands read once, results written once."""
     B, S = w.item_bytes, T * w.k
+    kf = 2 * w.f_s + (0 if w.standard else w.l)     # final GEMM's K ([h_s | n], or h_s + u added)
     return {
         "router": (2 * T * w.d * w.E, T * w.d * B + 4 * w.d * w.E + 4 * T * w.E),
         "topk": (0, 4 * T * w.E + T * w.k * (8 + B)),
         "scan": (0, 0),
         "dispatch": (0, T * w.k * 16),
-        "down_proj": (2 * T * w.d * w.l, T * w.d * B + w.l * w.d * B + T * w.l * B),
+        "down_proj": (0, 0) if w.standard else (2 * T * w.d * w.l, T * w.d * B + w.l * w.d * B + T * w.l * B),
         "permute": (0, T * w.l * B + S * w.l * B + S * 4),
         "gate_up": (2 * S * 2 * w.f * w.l, touched * 2 * w.f * w.l * B + S * w.l * B + S * w.f * B),
         "down_combine": (2 * S * w.l * w.f, touched * w.l * w.f * B + S * w.f * B + S * w.l * B),
-        "combine_norm": (0, S * w.l * B + 2 * T * w.l * B),
+        "combine_norm": (0, S * w.l * B + (1 if w.standard else 2) * T * w.l * B),
         "shared_gate_up": (2 * T * w.d * 4 * w.f_s, T * w.d * B + 4 * w.f_s * w.d * B + T * 2 * w.f_s * B),
-        "final": (2 * T * w.d * (2 * w.f_s + w.l),
-                  T * (2 * w.f_s + w.l) * B + w.d * (2 * w.f_s + w.l) * B + T * w.d * B),
+        "final": (2 * T * w.d * kf,
+                  T * kf * B + w.d * kf * B + T * w.d * B + (T * w.d * B if w.standard else 0)),
     }
 
 
@@ -192,12 +196,12 @@ def time_oracle(w, x, W, seconds, max_rows=None):
     rng = np.random.default_rng(7)
     n0 = min(cores, T)
     t0 = time.perf_counter()
-    oracle.forward(x, W, w.k, rows=rng.choice(T, n0, replace=False), eps=w.eps)
+    oracle.forward(x, W, w.k, rows=rng.choice(T, n0, replace=False), eps=w.eps, use_norm=not w.standard)
     dt0 = time.perf_counter() - t0
     n = int(max(n0, min(T if max_rows is None else max_rows, n0 * seconds / max(dt0, 1e-6))))
     rows = rng.choice(T, n, replace=False)
     t1 = time.perf_counter()
-    oracle.forward(x, W, w.k, rows=rows, eps=w.eps)
+    oracle.forward(x, W, w.k, rows=rows, eps=w.eps, use_norm=not w.standard)
     dt = time.perf_counter() - t1
     return n / dt, n, dt, cores
 
@@ -218,7 +222,7 @@ def run_reference(args, rank, world):
     for i in range(args.warmup + args.steps):
         rows = rng.choice(T, n, replace=False)
         t0 = time.perf_counter()
-        oracle.forward(x, W, w.k, rows=rows, eps=w.eps)
+        oracle.forward(x, W, w.k, rows=rows, eps=w.eps, use_norm=not w.standard)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     per_step = sum(times) / len(times)

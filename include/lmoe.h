@@ -72,6 +72,13 @@ typedef enum { LMOE_ACT_SWIGLU = 0, LMOE_ACT_SITU = 1 } lmoe_act;
  *  act       lmoe_act; gate_cap / up_cap are the SiTU caps (ignored for SwiGLU)
  *  gemm      0 = tensor cores (tcgen05) for bf16, CUDA cores for fp32;
  *            1 = CUDA cores for every GEMM (a slower cross-check path)
+ *  standard  0 = LatentMoE (above); 1 = the standard MoE it is compared with
+ *            (cooking-agi LatentMoE page: a standard MoE routes and computes its
+ *            experts at the model width; "Does the saving pay for more
+ *            experts?" counts no projections when the latent width equals the
+ *            width): requires l = d, skips W_down, RMSNorm and W_up, so
+ *            y = S1(x) + S2(x) + u with u = sum_j p_j E_j(x) at width d.  The
+ *            router, selection and shared experts are unchanged.
  */
 typedef struct {
     int32_t d, l, f, E, k, f_shared, n_shared;
@@ -80,13 +87,14 @@ typedef struct {
     int32_t act;
     float gate_cap, up_cap;
     int32_t gemm;
+    int32_t standard;
 } lmoe_config;
 
 /* Weights, all device pointers, read only during lmoe_create:
  *  W_r    [E, d]  fp32       router projection
  *  b      [E]     fp32       selection bias
- *  W_down [l, d]             shared down-projection
- *  W_up   [d, l]             up-projection
+ *  W_down [l, d]             shared down-projection (unused, may be NULL, when standard)
+ *  W_up   [d, l]             up-projection (unused, may be NULL, when standard)
  *  G, U   [E, f, l]          routed gate / up projections
  *  D      [E, l, f]          routed down projections
  *  Gs, Us [2, f_shared, d]   shared gate / up projections
@@ -105,9 +113,10 @@ typedef struct lmoe_handle lmoe_handle;
 /* Fill *out from the base-MoE description of the PyPI latent_moe README
  * (LatentMoEConfig: d, m, n_experts N, top_k K, alpha, n_shared, variant) and
  * its variant list: l = d / alpha, E = alpha * N routed experts; "eff" keeps
- * k = K, "acc" takes k = alpha * K; f = f_shared = m.  eps = 1e-6, bf16,
+ * k = K, "acc" takes k = alpha * K; f = f_shared = m.  "std" is the base
+ * standard MoE itself (l = d, E = N, k = K, standard = 1).  eps = 1e-6, bf16,
  * SwiGLU, tensor cores.  INVALID_ARG if a value is not positive, alpha does
- * not divide d, the variant is neither "acc" nor "eff", or k > E. */
+ * not divide d, the variant is not "acc", "eff" or "std", or k > E. */
 LMOE_API lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int32_t K, int32_t alpha,
                                   int32_t n_shared, const char *variant, lmoe_config *out);
 
@@ -117,7 +126,8 @@ LMOE_API lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int3
  * cores).  Work is enqueued on `stream`, which is synchronised before return,
  * so the caller may free its weight copies afterwards.
  * INVALID_ARG: null pointer, non-positive size, l > d, k < 1 or k > E,
- *              n_shared != 2, eps < 0, unknown dtype/act.
+ *              n_shared != 2, eps < 0, unknown dtype/act, standard not 0/1,
+ *              standard with l != d.
  * UNSUPPORTED: d, l, f or f_shared not a multiple of 64, E > 1024, k > 64,
  *              l > 8192, or (bf16
  *              tensor-core path) f or f_shared not a multiple of 128.

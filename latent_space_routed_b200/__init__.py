@@ -47,7 +47,8 @@ class lmoe_config(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("l", ctypes.c_int32), ("f", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("f_shared", ctypes.c_int32), ("n_shared", ctypes.c_int32),
                 ("eps", ctypes.c_float), ("dtype", ctypes.c_int32), ("act", ctypes.c_int32),
-                ("gate_cap", ctypes.c_float), ("up_cap", ctypes.c_float), ("gemm", ctypes.c_int32)]
+                ("gate_cap", ctypes.c_float), ("up_cap", ctypes.c_float), ("gemm", ctypes.c_int32),
+                ("standard", ctypes.c_int32)]
 
 
 class lmoe_weights(ctypes.Structure):
@@ -119,12 +120,12 @@ def lmoe_config_from_base(d, m, N, K, alpha, n_shared, variant) -> lmoe_config:
 
 
 def make_config(d, l, f, E, k, f_shared, n_shared=2, eps=1e-6, dtype=LMOE_BF16, act=LMOE_ACT_SWIGLU,
-                gate_cap=4.0, up_cap=25.0, gemm=0) -> lmoe_config:
-    return lmoe_config(d, l, f, E, k, f_shared, n_shared, eps, dtype, act, gate_cap, up_cap, gemm)
+                gate_cap=4.0, up_cap=25.0, gemm=0, standard=0) -> lmoe_config:
+    return lmoe_config(d, l, f, E, k, f_shared, n_shared, eps, dtype, act, gate_cap, up_cap, gemm, standard)
 
 
 def lmoe_create(cfg: lmoe_config, weights: Dict[str, torch.Tensor], stream=None) -> int:
-    w = lmoe_weights(*[_ptr(weights[n]) for n in ("W_r", "b", "W_down", "W_up", "G", "U", "D", "Gs", "Us", "Ds")])
+    w = lmoe_weights(*[_ptr(weights.get(n)) for n in ("W_r", "b", "W_down", "W_up", "G", "U", "D", "Gs", "Us", "Ds")])
     h = ctypes.c_void_p()
     _check(_lib.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), _stream(stream), ctypes.byref(h)))
     return h.value
@@ -236,6 +237,8 @@ class LatentMoE:
         dev = torch.device("cuda", torch.cuda.current_device())
         w = {}
         for n in ("W_r", "b", "W_down", "W_up", "G", "U", "D", "Gs", "Us", "Ds"):
+            if cfg.standard and n in ("W_down", "W_up"):
+                continue                 # the standard-MoE form has no projections
             want = torch.float32 if n in ("W_r", "b") else self.dtype
             w[n] = weights[n].to(device=dev, dtype=want).contiguous()
         self.handle = lmoe_create(cfg, w, stream)
@@ -327,4 +330,4 @@ def config_for(workload, gemm: int = 0, act: int = LMOE_ACT_SWIGLU) -> lmoe_conf
     """lmoe_config from an lmoe_inputs.Workload."""
     return make_config(workload.d, workload.l, workload.f, workload.E, workload.k, workload.f_s,
                        workload.n_shared, workload.eps, LMOE_F32 if workload.dtype == "f32" else LMOE_BF16, act,
-                       4.0, 25.0, gemm)
+                       4.0, 25.0, gemm, 1 if getattr(workload, "standard", False) else 0)

@@ -608,6 +608,27 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         if (MODE == EPI_SIGMOID) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
+                        } else if (MODE == EPI_STORE && sizeof(TO) == 2) {
+                            if (p.epi.residual && valid) {   // standard MoE: y = shared + u
+                                const bf16 *res = (const bf16 *)p.epi.residual + (slab + row) * p.epi.ldr + col;
+                                if (n == 32 && ((uintptr_t)res & 15u) == 0) {
+#pragma unroll
+                                    for (int q8 = 0; q8 < 4; ++q8) {   // four 16-byte loads
+                                        const uint4 w = *reinterpret_cast<const uint4 *>(res + 8 * q8);
+                                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                        for (int i = 0; i < 4; ++i) {
+                                            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&ws[i]);
+                                            x[8 * q8 + 2 * i] += __low2float(h2);
+                                            x[8 * q8 + 2 * i + 1] += __high2float(h2);
+                                        }
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i)
+                                        if (i < n) x[i] += __bfloat162float(res[i]);
+                                }
+                            }
                         } else if (MODE == EPI_COMBINE) {
                             const float w = valid ? p.epi.row_w[row] : 0.f;   // bf16 rows: p-weighted here
 #pragma unroll

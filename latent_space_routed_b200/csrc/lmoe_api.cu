@@ -14,6 +14,8 @@
 //   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
 //  10 shared gate/up   h_s = act([G_1; G_2] x, [U_1; U_2] x)    [T, 2 f_s]
 //  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
+// The standard-MoE form (config.standard) skips 5, permutes x, skips the norm
+// in 9 and computes y = h_s [D_s1 | D_s2]^T + u in 11.
 #include <algorithm>
 #include <cmath>
 #include <atomic>
@@ -54,6 +56,10 @@ lmoe_status fail(lmoe_status s, const char *fmt, ...)
     } while (0)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Columns of [h_s | RMSNorm(u)], the final GEMM's A (no norm columns in the
+// standard-MoE form, which adds u in the final GEMM's epilogue instead).
+int64_t hs_cols(const lmoe_config &c) { return 2 * (int64_t)c.f_shared + (c.standard ? 0 : c.l); }
 
 struct Layout {
     size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, partial,
@@ -127,11 +133,11 @@ struct SplitPlan {
 SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
 {
     const lmoe_config &c = h->cfg;
-    const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
+    const int64_t ld_hs = hs_cols(c);
     SplitPlan sp;
     sp.router = (h->tc && T > ROUTER_SMALL_MAX_T)
                     ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true, router_cg(T)) : 1;
-    sp.down = plan_ksplit(h, T, c.l, c.d / TC_BK);
+    sp.down = c.standard ? 1 : plan_ksplit(h, T, c.l, c.d / TC_BK);
     sp.shared = plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
     sp.final_ = plan_ksplit(h, T, c.d, ld_hs / TC_BK);
     auto need = [&](int ks, int64_t n) -> size_t { return ks > 1 ? (size_t)ks * (size_t)n * (size_t)T : 0; };
@@ -162,7 +168,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.slot_of = take(sizeof(int32_t) * S);
     L.perm_tok = take(sizeof(int32_t) * S);
     L.perm_w = take(sizeof(float) * S);
-    L.z = take(h->tb * T * c.l);
+    L.z = take(c.standard ? 0 : h->tb * T * c.l);   // the standard form permutes x itself
     L.Zp = take(h->tb * S * c.l);
     L.H = take(h->tb * S * c.f);
     L.Yp = take(h->tb * S * c.l);
@@ -190,6 +196,9 @@ lmoe_status check_config(const lmoe_config *c, bool *tc)
     if (c->act == LMOE_ACT_SITU && !(c->gate_cap > 0.f && c->up_cap > 0.f))
         return fail(LMOE_ERR_INVALID_ARG, "SiTU caps must be positive");
     if (c->gemm != 0 && c->gemm != 1) return fail(LMOE_ERR_INVALID_ARG, "gemm must be 0 or 1");
+    if (c->standard != 0 && c->standard != 1) return fail(LMOE_ERR_INVALID_ARG, "standard must be 0 or 1");
+    if (c->standard && c->l != c->d)
+        return fail(LMOE_ERR_INVALID_ARG, "the standard-MoE form needs l = d (got l=%d, d=%d)", c->l, c->d);
     if (c->E > 1024) return fail(LMOE_ERR_UNSUPPORTED, "E=%d > 1024", c->E);
     if (c->l > 8192) return fail(LMOE_ERR_UNSUPPORTED, "l=%d > 8192", c->l);
     if (c->k > 64) return fail(LMOE_ERR_UNSUPPORTED, "k=%d > 64", c->k);
@@ -229,15 +238,17 @@ lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int32_t K, in
         return fail(LMOE_ERR_INVALID_ARG, "all base values must be positive");
     if (d % alpha) return fail(LMOE_ERR_INVALID_ARG, "alpha=%d does not divide d=%d", alpha, d);
     int k;
-    if (!strcmp(variant, "eff")) k = K;
+    const bool standard = !strcmp(variant, "std");
+    if (!strcmp(variant, "eff") || standard) k = K;
     else if (!strcmp(variant, "acc")) k = alpha * K;
-    else return fail(LMOE_ERR_INVALID_ARG, "variant must be \"acc\" or \"eff\"");
-    const int E = alpha * N;
+    else return fail(LMOE_ERR_INVALID_ARG, "variant must be \"acc\", \"eff\" or \"std\"");
+    const int E = standard ? N : alpha * N;
     if (k > E) return fail(LMOE_ERR_INVALID_ARG, "top-k %d exceeds %d experts", k, E);
     lmoe_config c;
     memset(&c, 0, sizeof c);
-    c.d = d; c.l = d / alpha; c.f = m; c.E = E; c.k = k; c.f_shared = m; c.n_shared = n_shared;
+    c.d = d; c.l = standard ? d : d / alpha; c.f = m; c.E = E; c.k = k; c.f_shared = m; c.n_shared = n_shared;
     c.eps = 1e-6f; c.dtype = LMOE_BF16; c.act = LMOE_ACT_SWIGLU; c.gate_cap = 4.f; c.up_cap = 25.f; c.gemm = 0;
+    c.standard = standard ? 1 : 0;
     *out = c;
     return LMOE_OK;
 }
@@ -250,7 +261,8 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
     bool tc = false;
     lmoe_status st = check_config(cfg, &tc);
     if (st != LMOE_OK) return st;
-    if (!w || !w->W_r || !w->b || !w->W_down || !w->W_up || !w->G || !w->U || !w->D || !w->Gs || !w->Us || !w->Ds)
+    if (!w || !w->W_r || !w->b || !w->G || !w->U || !w->D || !w->Gs || !w->Us || !w->Ds ||
+        (!cfg->standard && (!w->W_down || !w->W_up)))
         return fail(LMOE_ERR_INVALID_ARG, "a weight pointer is NULL");
     if (tc) {
         st = tc_check_device();
@@ -289,19 +301,20 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
 
     ALLOC(h->Wr, sizeof(float) * c.E * c.d);
     ALLOC(h->b, sizeof(float) * c.E);
-    ALLOC(h->Wdown, tb * c.l * c.d);
+    if (!c.standard) ALLOC(h->Wdown, tb * c.l * c.d);
     ALLOC(h->Wgu, tb * (size_t)c.E * 2 * c.f * c.l);
     ALLOC(h->D, tb * (size_t)c.E * c.l * c.f);
     ALLOC(h->Wgu_s, tb * 4 * fs * c.d);
-    ALLOC(h->Wcat, tb * c.d * (2 * fs + c.l));
+    ALLOC(h->Wcat, tb * c.d * hs_cols(c));
     STEP(cudaMemcpyAsync(h->Wr, w->W_r, sizeof(float) * c.E * c.d, cudaMemcpyDeviceToDevice, s));
     STEP(cudaMemcpyAsync(h->b, w->b, sizeof(float) * c.E, cudaMemcpyDeviceToDevice, s));
-    STEP(cudaMemcpyAsync(h->Wdown, w->W_down, tb * c.l * c.d, cudaMemcpyDeviceToDevice, s));
+    if (!c.standard) STEP(cudaMemcpyAsync(h->Wdown, w->W_down, tb * c.l * c.d, cudaMemcpyDeviceToDevice, s));
     STEP(cudaMemcpyAsync(h->D, w->D, tb * (size_t)c.E * c.l * c.f, cudaMemcpyDeviceToDevice, s));
     STEP(launch_pack_glu(w->G, w->U, h->Wgu, c.E, c.f, c.l, h->ib, (int)tb, s));
     // [2, f_s, d] stacks are the rows of one expert of width 2 f_s
     STEP(launch_pack_glu(w->Gs, w->Us, h->Wgu_s, 1, 2 * c.f_shared, c.d, h->ib, (int)tb, s));
-    STEP(launch_pack_cat(w->Ds, w->W_up, h->Wcat, c.d, c.f_shared, c.l, (int)tb, s));
+    // standard: [D_s1 | D_s2] only (u is added in the final GEMM's epilogue)
+    STEP(launch_pack_cat(w->Ds, w->W_up, h->Wcat, c.d, c.f_shared, c.standard ? 0 : c.l, (int)tb, s));
     if (tc) {
         ALLOC(h->Wr3, sizeof(bf16) * 3 * c.E * c.d);
         STEP(launch_split_router(h->Wr, h->Wr3, (int64_t)c.E * c.d, s));
@@ -343,7 +356,7 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 3: *offset = L.offsets; *bytes = sizeof(int32_t) * (c.E + 1); break;
     case 4: *offset = L.slot_of; *bytes = sizeof(int32_t) * S; break;
     case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
-    case 6: *offset = L.z; *bytes = h->tb * T * c.l; break;
+    case 6: *offset = L.z; *bytes = c.standard ? 0 : h->tb * T * c.l; break;
     case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
     case 8: *offset = L.Yp; *bytes = h->tb * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
@@ -389,10 +402,8 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
     // other than the router's (which the top-k kernel reduces)
     if (T == 0) { *launches = 0; return LMOE_OK; }
     const lmoe_config &c = h->cfg;
-    const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
     const SplitPlan sp = plan_splits(h, T);
-    (void)ld_hs;
-    *launches = 13 + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
+    *launches = 13 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
     return LMOE_OK;
 }
 
@@ -469,7 +480,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     const int64_t S = T * c.k;
     const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
     const int tk = c.dtype == LMOE_BF16 ? 1 : 0;
-    const int64_t ld_hs = 2 * (int64_t)c.f_shared + c.l;
+    const int64_t ld_hs = hs_cols(c);
     // Tensor-core tiles: 256-row tiles on CTA pairs where rows are plentiful
     // (grouped: at least ~192 slot rows per expert on average), else 128.
     const int cg_grouped = (h->tc && S >= 192LL * c.E) ? 2 : 1;
@@ -543,6 +554,10 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     GemmArgs gf = {};
     gf.A = HS; gf.lda = ld_hs; gf.B = h->Wcat; gf.ldb = ld_hs; gf.M = (int)T; gf.N = c.d; gf.K = (int)ld_hs;
     gf.epi.out = output; gf.epi.ldo = c.d;
+    if (c.standard) {   // y = [h_s] [D_s1 | D_s2]^T + u
+        gf.epi.residual = latent_routed_aggregate;
+        gf.epi.ldr = c.l;
+    }
 
     // Dense tensor-core GEMM, split along K per the plan.
     auto dense_tc = [&](int mode, const GemmArgs &g, int ks, float *part, cudaStream_t q) -> cudaError_t {
@@ -553,15 +568,16 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
         cudaError_t e = tc_gemm(EPI_STORE_F32, gp, 0, 1, status, q, ks);
         if (e != cudaSuccess) return e;
         return launch_splitk_reduce(part, ks, g.M, g.N, mode, g.epi.act, g.epi.gate_cap, g.epi.up_cap, TC_BN / 2,
-                                    g.epi.out, g.epi.ldo, q);
+                                    g.epi.out, g.epi.ldo, q, g.epi.residual, g.epi.ldr);
     };
     auto st_down = [&](cudaStream_t q) -> lmoe_status {
+        if (c.standard) return LMOE_OK;   // experts read x itself
         if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down, partial_side, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, q));
         return LMOE_OK;
     };
     auto st_permute = [&](cudaStream_t q) -> lmoe_status {
-        LMOE_CUDA(launch_permute_rows(z, perm_tok, Zp, S, c.l, (int)h->tb, q));
+        LMOE_CUDA(launch_permute_rows(c.standard ? x : z, perm_tok, Zp, S, c.l, (int)h->tb, q));
         return LMOE_OK;
     };
     auto st_gate_up = [&](cudaStream_t q) -> lmoe_status {
@@ -575,8 +591,8 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
         return LMOE_OK;
     };
     auto st_combine_norm = [&](cudaStream_t q) -> lmoe_status {   // u, RMSNorm(u) after the shared hidden
-        LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate, HS, ld_hs,
-                                      2 * (int64_t)c.f_shared, tk, q));
+        LMOE_CUDA(launch_combine_norm(Yp, slot_of, T, c.l, c.k, c.eps, latent_routed_aggregate,
+                                      c.standard ? nullptr : HS, ld_hs, 2 * (int64_t)c.f_shared, tk, q));
         return LMOE_OK;
     };
     auto st_shared = [&](cudaStream_t q) -> lmoe_status {

@@ -55,6 +55,8 @@ struct EpiArgs {
     int act;                 // EPI_GLU
     float gate_cap, up_cap;
     int ib;                  // EPI_GLU: gate/up interleave block (columns)
+    const void *residual;    // EPI_STORE: out = C + residual[m, n] (token dtype) when not NULL
+    int64_t ldr;             // row stride of residual, elements
 };
 
 // Write n <= 32 consecutive values v[0..n) of row `row` starting at output column `col`.
@@ -72,8 +74,10 @@ __device__ __forceinline__ void epi_store_chunk(const EpiArgs &e, int64_t row, i
         for (int i = 0; i < 32; ++i) if (i < n) o[i] = from_f32<TO>(w * v[i]);
     } else {
         TO *o = (TO *)e.out + row * e.ldo + col;
+        const TO *res = e.residual ? (const TO *)e.residual + row * e.ldr + col : nullptr;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) if (i < n) o[i] = from_f32<TO>(v[i]);
+        for (int i = 0; i < 32; ++i)
+            if (i < n) o[i] = from_f32<TO>(res ? v[i] + to_f32(res[i]) : v[i]);
     }
 }
 
@@ -123,6 +127,7 @@ cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t 
 cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
                                 cudaStream_t s);
 // Yp in the token dtype.
+// hs = NULL: u only (no RMSNorm; the standard-MoE form).
 cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
                                 void *u_out, void *hs, int64_t ld_hs, int64_t col0, int tok_bf16, cudaStream_t s);
 
@@ -131,7 +136,8 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
 // interleaved in blocks of ib, bf16 out[m, n'] for n' < N / 2) or EPI_SIGMOID
 // (fp32 out[m, n] = sigmoid(sum)).
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
-                                 float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s);
+                                 float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s,
+                                 const void *residual = nullptr, int64_t ldr = 0);
 // Router scores for a few tokens on CUDA cores: r[t, e] = sigmoid(sum_k x[t, k] W[e, k]),
 // x bf16 [T, d], W fp32 [E, d] (fixed summation order, deterministic).
 cudaError_t launch_router_small(const bf16 *x, const float *W, int64_t T, int E, int d, float *r, cudaStream_t s);

@@ -95,10 +95,12 @@ combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_
     const float inv = 1.0f / sqrtf(tot / (float)l + eps);
     if (active) {
         store8(u_out + t * l + c0, u);
-        float n[8];
+        if (hs) {
+            float n[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) n[i] = u[i] * inv;
-        store8(hs + t * ld_hs + col0 + c0, n);
+            for (int i = 0; i < 8; ++i) n[i] = u[i] * inv;
+            store8(hs + t * ld_hs + col0 + c0, n);
+        }
     }
 }
 
@@ -158,7 +160,8 @@ __global__ void split_router_kernel(const float *__restrict__ W, bf16 *__restric
 template <int MODE>
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, int N, int act, float gate_cap,
-                     float up_cap, int ib, void *__restrict__ out_, int64_t ldo)
+                     float up_cap, int ib, void *__restrict__ out_, int64_t ldo,
+                     const bf16 *__restrict__ residual, int64_t ldr)
 {
     const int64_t m = blockIdx.y;
     const int nout = (MODE == EPI_GLU) ? N / 2 : N;
@@ -202,6 +205,10 @@ splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, i
             const float4 a = *reinterpret_cast<const float4 *>(partial + sp * slab + m * N + j0);
             r[0] += a.x; r[1] += a.y; r[2] += a.z; r[3] += a.w;
         }
+        if (residual) {   // standard MoE: y = shared + u
+#pragma unroll
+            for (int i = 0; i < 4; ++i) r[i] += __bfloat162float(residual[m * ldr + j0 + i]);
+        }
     }
     bf16 *out = reinterpret_cast<bf16 *>(out_);
     const __nv_bfloat162 p0 = __floats2bfloat162_rn(r[0], r[1]);
@@ -215,7 +222,8 @@ splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, i
 }  // namespace
 
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
-                                 float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s)
+                                 float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s, const void *residual,
+                                 int64_t ldr)
 {
     if (M == 0) return cudaSuccess;
     if (mode != EPI_SIGMOID && (N % 8 || ldo % 4 || (mode == EPI_GLU && ib % 4))) return cudaErrorInvalidValue;
@@ -224,12 +232,14 @@ cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, in
     const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
     dim3 grid((unsigned)((nvec + threads - 1) / threads), (unsigned)M);
     if (mode == EPI_GLU)
-        splitk_reduce_kernel<EPI_GLU><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
+        splitk_reduce_kernel<EPI_GLU><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo,
+                                                               nullptr, 0);
     else if (mode == EPI_SIGMOID)
         splitk_reduce_kernel<EPI_SIGMOID><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out,
-                                                               ldo);
+                                                                   ldo, nullptr, 0);
     else
-        splitk_reduce_kernel<EPI_STORE><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo);
+        splitk_reduce_kernel<EPI_STORE><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo,
+                                                                 (const bf16 *)residual, ldr);
     return cudaGetLastError();
 }
 

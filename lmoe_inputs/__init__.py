@@ -55,6 +55,7 @@ class Workload:
     n_shared: int = 2
     eps: float = 1e-6
     T_sweep: Sequence[int] = ()
+    standard: bool = False  # the standard MoE (l = d, no projections, no norm)
 
     def with_T(self, T: int) -> "Workload":
         return dataclasses.replace(self, T=T)
@@ -75,13 +76,17 @@ WORKLOADS: Dict[str, Workload] = {
     "large_d4096": Workload("large_d4096", 32768, 4096, 1024, 2688, 512, 24, 2688, "bf16", "uniform", 3),
     "decode_d7168": Workload("decode_d7168", 128, 7168, 1792, 2048, 384, 32, 2048, "bf16", "zero", 4,
                              T_sweep=(1, 8, 32, 128)),
+    # the standard MoE that acc_d2048 is derived from (alpha = 4: 64 experts,
+    # top 6, experts at the model width): the comparison the pages make
+    "std_d2048": Workload("std_d2048", 4096, 2048, 2048, 1408, 64, 6, 1408, "bf16", "uniform", 5,
+                          standard=True),
 }
 
 
 def custom(name: str, T: int, d: int, l: int, f: int, E: int, k: int, f_s: int,
-           dtype: str = "bf16", bias: str = "uniform", seed: int = 100) -> Workload:
+           dtype: str = "bf16", bias: str = "uniform", seed: int = 100, standard: bool = False) -> Workload:
     """A workload with arbitrary sizes (used for multi-tile / ragged tests)."""
-    return Workload(name, T, d, l, f, E, k, f_s, dtype, bias, seed)
+    return Workload(name, T, d, l, f, E, k, f_s, dtype, bias, seed, standard=standard)
 
 
 # Tensor ids: fixed forever so that stored expected values stay valid.
@@ -139,9 +144,22 @@ def weights(w: Workload) -> Dict[str, torch.Tensor]:
     Layout is "out x in" (row-major, as in W @ x):
     W_r [E, d] fp32, b [E] fp32, W_down [l, d], W_up [d, l],
     G, U [E, f, l], D [E, l, f], Gs, Us [2, f_s, d], Ds [2, d, f_s].
+    A standard workload (l = d) carries identity W_down and W_up: the layer
+    formula with identity projections and no norm is the standard MoE, so a
+    reference can run it as is, while the library skips them.
     """
     dt = w.torch_dtype
     s = w.seed
+    if w.standard:
+        if w.l != w.d:
+            raise ValueError("a standard workload needs l = d")
+        eye = torch.eye(w.d, dtype=dt)
+        out = weights(dataclasses.replace(w, standard=False, l=1))
+        out["W_down"], out["W_up"] = eye, eye.clone()
+        out["G"] = _stack(w.E, (w.f, w.l), 1.0 / math.sqrt(w.l), s, _TID["G"], dt)
+        out["U"] = _stack(w.E, (w.f, w.l), 1.0 / math.sqrt(w.l), s, _TID["U"], dt)
+        out["D"] = _stack(w.E, (w.l, w.f), 1.0 / math.sqrt(w.f), s, _TID["D"], dt)
+        return out
     return {
         "W_r": _normal((w.E, w.d), 1.0 / math.sqrt(w.d), _gen(s, _TID["W_r"]), torch.float32),
         "b": bias(w),

@@ -42,6 +42,15 @@ def test_config_from_base_readme_defaults(variant, k):
     assert abs(c.eps - 1e-6) < 1e-12
 
 
+def test_config_from_base_standard_moe():
+    """The base standard MoE the variants are derived from (cooking-agi
+    LatentMoE page: experts at the model width, no projections): l = d,
+    E = N, k = K."""
+    c = lm.lmoe_config_from_base(2048, 1408, 64, 6, 4, 2, "std")
+    assert (c.d, c.l, c.f, c.E, c.k, c.f_shared, c.standard) == (2048, 2048, 1408, 64, 6, 1408, 1)
+    assert lm.lmoe_config_from_base(2048, 1408, 64, 6, 4, 2, "acc").standard == 0
+
+
 @pytest.mark.parametrize("args", [(2048, 1408, 64, 6, 3, 2, "acc"), (2048, 1408, 64, 6, 4, 2, "big"),
                                   (0, 1408, 64, 6, 4, 2, "acc"), (2048, 1408, 2, 3, 1, 2, "eff")])
 def test_config_from_base_rejects(args):
@@ -63,6 +72,7 @@ def _cfg(**kw):
     (dict(dtype=7), lm.LMOE_ERR_INVALID_ARG), (dict(act=5), lm.LMOE_ERR_INVALID_ARG),
     (dict(d=200), lm.LMOE_ERR_UNSUPPORTED), (dict(E=2048, k=4), lm.LMOE_ERR_UNSUPPORTED),
     (dict(k=65, E=100), lm.LMOE_ERR_UNSUPPORTED),
+    (dict(standard=1), lm.LMOE_ERR_INVALID_ARG), (dict(standard=2, l=256), lm.LMOE_ERR_INVALID_ARG),
 ])
 def test_create_validates_before_touching_the_device(kw, status):
     """Constraints of "Stable LatentMoE" (two shared experts, 1 <= k <= E) and

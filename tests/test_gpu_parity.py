@@ -51,11 +51,14 @@ def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0):
         rows = np.sort(rng.choice(T, size=n_rows, replace=False))
         rows[-1] = T - 1   # always include the ragged tail
         rows = np.unique(rows)
-    ora = oracle.forward(x, W, w.k, act=act, rows=rows, eps=w.eps)
+    # a standard workload carries identity projections: with no norm, the
+    # oracle's layer formula is then the standard MoE
+    norm = not w.standard
+    ora = oracle.forward(x, W, w.k, act=act, rows=rows, eps=w.eps, use_norm=norm)
 
     def rerun(idx, sel):
         r = idx if rows is None else rows[idx]
-        return oracle.forward(x, W, w.k, act=act, rows=r, sel=sel, eps=w.eps)
+        return oracle.forward(x, W, w.k, act=act, rows=r, sel=sel, eps=w.eps, use_norm=norm)
 
     errs = compare({k: v.cpu() for k, v in out.items()}, ora, W["b"].numpy(), TOL[w.dtype], rerun, rows)
     layer.close()
@@ -113,6 +116,24 @@ def test_bf16_pair_tiles_edge_shapes(shape):
     w = li.custom("pair_edges", *shape, dtype="bf16", seed=25)
     errs, _ = run_parity(w)
     assert errs["output"] <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype,gemm", [("bf16", 0), ("bf16", 1), ("f32", 0)])
+def test_standard_moe_form(dtype, gemm):
+    """config.standard: experts at the model width on x itself, no projections
+    or norm, y = shared + sum_j p_j E_j(x) (the final GEMM adds u in its
+    epilogue); every row against the oracle run with identity projections and
+    no norm."""
+    w = li.custom("standard", 600, 256, 256, 256, 16, 3, 256, dtype=dtype, seed=27, standard=True)
+    run_parity(w, gemm=gemm)
+
+
+@pytest.mark.parametrize("T", [5, 100])
+def test_standard_moe_form_few_tokens(T):
+    """Few tokens: CUDA-core router and split-K final GEMM, whose reduction
+    adds u."""
+    w = li.custom("standard_few", T, 512, 512, 256, 32, 4, 256, dtype="bf16", seed=28, standard=True)
+    run_parity(w)
 
 
 def test_fp32_multi_tile_ragged():
@@ -281,7 +302,7 @@ def test_zero_tokens_is_a_noop_and_errors_are_reported():
 
 
 # ---------------------------------------------------------------- full-size workloads, sampled rows
-@pytest.mark.parametrize("name,n_rows", [("acc_d2048", 64), ("eff_zipf_d2048", 64)])
+@pytest.mark.parametrize("name,n_rows", [("acc_d2048", 64), ("eff_zipf_d2048", 64), ("std_d2048", 48)])
 def test_full_size_sampled_rows(name, n_rows):
     errs, _ = run_parity(li.WORKLOADS[name], n_rows=n_rows)
     print(name, errs)
