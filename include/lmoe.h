@@ -286,7 +286,7 @@ LMOE_API lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspac
  * until the process exits.  Nothing is allocated by the call.
  *  - If lmoe_workspace_size(h, T) exceeds the area, it returns
  *    LMOE_ERR_WORKSPACE and launches nothing (the area covers, for example,
- *    up to 105 tokens of a d = 7168, l = 1792, f = 2048, k = 32, E = 384
+ *    up to 132 tokens of a d = 7168, l = 1792, f = 2048, k = 32, E = 384
  *    layer on a 148-SM B200).
  *  - The first call on a device looks up the area's device address with that
  *    device current; make it before any stream capture.
