@@ -136,6 +136,15 @@ def test_standard_moe_form_few_tokens(T):
     run_parity(w)
 
 
+@pytest.mark.parametrize("bias", ["zipf", "uniform"])
+def test_bf16_pair_tiles_skewed_expert_loads(bias):
+    """CTA-pair tiles for the grouped GEMMs; a Zipf bias gives experts from a
+    handful of slot rows to thousands (empty and ragged m-tiles next to long
+    runs of full ones); every row compared."""
+    w = li.custom("skew_" + bias, 1500, 256, 256, 256, 16, 4, 256, dtype="bf16", bias=bias, seed=26)
+    run_parity(w)
+
+
 def test_fp32_multi_tile_ragged():
     w = li.custom("multi_f32", 333, 256, 128, 128, 24, 5, 192, dtype="f32", seed=23)
     run_parity(w)
