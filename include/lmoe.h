@@ -171,8 +171,14 @@ LMOE_API lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, s
 
 /* lmoe_forward on HOST buffers (same shapes and dtypes as lmoe_forward; use
  * pinned memory for asynchronous copies): copies x to the device, runs the
- * forward, and copies the four outputs back, all enqueued on `stream`.  The
- * host outputs are valid once the stream has been synchronised.
+ * forward, and copies the four outputs back.  The host outputs are valid once
+ * `stream` has been synchronised.  From 2 x max(2048, 192 E / k) tokens on, the
+ * call cuts the batch into up to 8 chunks of whole rows and pipelines them:
+ * chunk j's input crosses on a copy stream the handle owns while chunk j - 1
+ * computes on `stream`, and its outputs return on a second one while chunk
+ * j + 1 computes; `stream` waits for the last copy.  Rows are independent, so
+ * every row's result is that of lmoe_forward on the chunk that holds it.  The
+ * device status word (lmoe_check_device) covers the whole call.
  * Errors as lmoe_forward. */
 LMOE_API lmoe_status lmoe_forward_host(lmoe_handle *h, const void *x_host, int64_t T, void *output_host,
                               int32_t *selected_experts_host, void *mixture_weights_host,

@@ -93,6 +93,10 @@ struct lmoe_handle {
     cudaStream_t side = nullptr;  // tensor-core path: the shared experts' gate/up runs here, overlapped
     cudaEvent_t ev_fork = nullptr, ev_z = nullptr, ev_join = nullptr;
     std::mutex fork_mutex;
+    // lmoe_forward_host: copy streams and events of its chunk pipeline
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t ev_host[2 + 2 * 8] = {};
+    std::mutex host_mutex;
 };
 
 namespace {
@@ -150,6 +154,26 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
 // stages one after another on one stream).
 bool use_side_stream(const lmoe_handle *h) { return h->tc && h->side && !h->stage_events; }
 
+// Chunks of a host-buffer forward (lmoe_forward_host): the copies of chunk
+// j + 1 in and chunk j - 1 out overlap the compute of chunk j.  Rows are
+// independent, so chunking changes no row's arithmetic (only how a batch is
+// cut into launches); each chunk keeps at least 2048 tokens and enough slot
+// rows per expert (192 E / k tokens) for CTA-pair tiles.
+constexpr int HOST_MAX_CHUNKS = 8;
+int host_chunks(const lmoe_config &c, int64_t T, int64_t *Tc)
+{
+    int64_t minc = (192LL * c.E + c.k - 1) / c.k;
+    if (minc < 2048) minc = 2048;
+    int64_t nc = T / minc;
+    if (nc > HOST_MAX_CHUNKS) nc = HOST_MAX_CHUNKS;
+    if (nc < 2) {
+        *Tc = T;
+        return 1;
+    }
+    *Tc = (T + nc - 1) / nc;
+    return (int)nc;
+}
+
 Layout plan(const lmoe_handle *h, int64_t T)
 {
     const lmoe_config &c = h->cfg;
@@ -158,6 +182,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     Layout L;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
+    L.status = take(256);   // first: the same offset for every T (chunked host forwards share it)
     L.r32 = take(sizeof(float) * T * c.E);
     L.p32 = take(sizeof(float) * S);
     L.blockhist = take(sizeof(int32_t) * nb * c.E);
@@ -177,7 +202,6 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.partial = take(sizeof(float) * sp.partial_floats);
     L.partial_side = take(sizeof(float) * sp.partial_side_floats);
     L.cutoff = take(sizeof(float) * T);
-    L.status = take(256);
     L.total = o;
     return L;
 }
@@ -219,6 +243,10 @@ void free_handle(lmoe_handle *h)
     if (h->side) cudaStreamDestroy(h->side);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_z) cudaEventDestroy(h->ev_z);
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
+    for (cudaEvent_t e : h->ev_host)
+        if (e) cudaEventDestroy(e);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
     delete h;
 }
@@ -323,6 +351,9 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
         STEP(cudaEventCreateWithFlags(&h->ev_z, cudaEventDisableTiming));
         STEP(cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming));
     }
+    STEP(cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking));
+    STEP(cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking));
+    for (cudaEvent_t &e : h->ev_host) STEP(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
     STEP(cudaStreamSynchronize(s));
 #undef ALLOC
 #undef STEP
@@ -443,11 +474,12 @@ lmoe_status lmoe_qb_bias_update(const lmoe_handle *h, const int32_t *hist, int32
     return LMOE_OK;
 }
 
-lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
-                         void *mixture_weights, void *latent_routed_aggregate, void *workspace, size_t ws_bytes,
-                         void *stream)
+// The forward of lmoe_forward; reset_status = false keeps the device status
+// word as it is (the chunks of one lmoe_forward_host call after the first).
+static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
+                                void *mixture_weights, void *latent_routed_aggregate, void *workspace,
+                                size_t ws_bytes, void *stream, bool reset_status)
 {
-    g_err.clear();
     if (!h) return fail(LMOE_ERR_INVALID_ARG, "handle is NULL");
     if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
     if (T == 0) return LMOE_OK;
@@ -488,7 +520,7 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     const int bm = h->tc ? TC_BM * cg_grouped : SIMT_BM;
     const int max_mtiles = (int)((S + bm - 1) / bm + c.E);
 
-    LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    if (reset_status) LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
     const SplitPlan sp = plan_splits(h, T);
     float *partial = (float *)(ws + L.partial);             // router, final
     float *partial_side = (float *)(ws + L.partial_side);   // down, shared gate/up
@@ -668,6 +700,15 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
     return LMOE_OK;
 }
 
+lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
+                         void *mixture_weights, void *latent_routed_aggregate, void *workspace, size_t ws_bytes,
+                         void *stream)
+{
+    g_err.clear();
+    return forward_body(h, x, T, output, selected_experts, mixture_weights, latent_routed_aggregate, workspace,
+                        ws_bytes, stream, true);
+}
+
 lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes)
 {
     g_err.clear();
@@ -681,7 +722,11 @@ lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *by
     o = align_up(o + sizeof(int32_t) * T * c.k, 256);
     o = align_up(o + h->tb * T * c.k, 256);
     o = align_up(o + h->tb * T * c.l, 256);
-    *bytes = o + plan(h, T).total;
+    int64_t Tc = T;
+    const int nc = host_chunks(c, T, &Tc);
+    size_t fw = plan(h, Tc).total;                       // the chunks' forward workspace
+    if (nc > 1) fw = std::max(fw, plan(h, T - (int64_t)(nc - 1) * Tc).total);
+    *bytes = o + fw;
     return LMOE_OK;
 }
 
@@ -710,13 +755,53 @@ lmoe_status lmoe_forward_host(lmoe_handle *h, const void *x_host, int64_t T, voi
     char *dsel = ws + o; o = align_up(o + bs, 256);
     char *dp = ws + o; o = align_up(o + bp, 256);
     char *du = ws + o; o = align_up(o + bu, 256);
-    LMOE_CUDA(cudaMemcpyAsync(dx, x_host, bx, cudaMemcpyHostToDevice, s));
-    lmoe_status st = lmoe_forward(h, dx, T, dy, (int32_t *)dsel, dp, du, ws + o, ws_bytes - o, stream);
-    if (st != LMOE_OK) return st;
-    LMOE_CUDA(cudaMemcpyAsync(output_host, dy, bx, cudaMemcpyDeviceToHost, s));
-    LMOE_CUDA(cudaMemcpyAsync(selected_experts_host, dsel, bs, cudaMemcpyDeviceToHost, s));
-    LMOE_CUDA(cudaMemcpyAsync(mixture_weights_host, dp, bp, cudaMemcpyDeviceToHost, s));
-    LMOE_CUDA(cudaMemcpyAsync(latent_routed_aggregate_host, du, bu, cudaMemcpyDeviceToHost, s));
+    char *fws = ws + o;
+    const size_t fbytes = ws_bytes - o;
+    int64_t Tc = T;
+    const int nc = host_chunks(c, T, &Tc);
+    if (nc == 1) {
+        LMOE_CUDA(cudaMemcpyAsync(dx, x_host, bx, cudaMemcpyHostToDevice, s));
+        lmoe_status st = forward_body(h, dx, T, dy, (int32_t *)dsel, dp, du, fws, fbytes, stream, true);
+        if (st != LMOE_OK) return st;
+        LMOE_CUDA(cudaMemcpyAsync(output_host, dy, bx, cudaMemcpyDeviceToHost, s));
+        LMOE_CUDA(cudaMemcpyAsync(selected_experts_host, dsel, bs, cudaMemcpyDeviceToHost, s));
+        LMOE_CUDA(cudaMemcpyAsync(mixture_weights_host, dp, bp, cudaMemcpyDeviceToHost, s));
+        LMOE_CUDA(cudaMemcpyAsync(latent_routed_aggregate_host, du, bu, cudaMemcpyDeviceToHost, s));
+        return LMOE_OK;
+    }
+    // Pipeline: chunk j's input on copy_in, its forward on `stream` (after its
+    // input), its outputs on copy_out (after its forward); the caller's stream
+    // waits for the last copy.  One status word for the whole call.
+    std::lock_guard<std::mutex> lock(h->host_mutex);
+    cudaEvent_t *ev = h->ev_host;   // [0] start, [1] all out, [2 + j] chunk j in, [2 + 8 + j] chunk j done
+    const size_t rx = h->tb * c.d, rs = sizeof(int32_t) * c.k, rp = h->tb * c.k, ru = h->tb * c.l;
+    LMOE_CUDA(cudaMemsetAsync(fws + plan(h, Tc).status, 0, sizeof(int32_t), s));
+    LMOE_CUDA(cudaEventRecord(ev[0], s));
+    LMOE_CUDA(cudaStreamWaitEvent(h->copy_in, ev[0], 0));
+    LMOE_CUDA(cudaStreamWaitEvent(h->copy_out, ev[0], 0));
+    for (int j = 0; j < nc; ++j) {
+        const int64_t t0 = (int64_t)j * Tc;
+        const int64_t tj = std::min(Tc, T - t0);
+        LMOE_CUDA(cudaMemcpyAsync(dx + t0 * rx, (const char *)x_host + t0 * rx, tj * rx, cudaMemcpyHostToDevice,
+                                  h->copy_in));
+        LMOE_CUDA(cudaEventRecord(ev[2 + j], h->copy_in));
+        LMOE_CUDA(cudaStreamWaitEvent(s, ev[2 + j], 0));
+        const lmoe_status st = forward_body(h, dx + t0 * rx, tj, dy + t0 * rx, (int32_t *)(dsel + t0 * rs),
+                                            dp + t0 * rp, du + t0 * ru, fws, fbytes, stream, false);
+        if (st != LMOE_OK) return st;
+        LMOE_CUDA(cudaEventRecord(ev[2 + HOST_MAX_CHUNKS + j], s));
+        LMOE_CUDA(cudaStreamWaitEvent(h->copy_out, ev[2 + HOST_MAX_CHUNKS + j], 0));
+        LMOE_CUDA(cudaMemcpyAsync((char *)output_host + t0 * rx, dy + t0 * rx, tj * rx, cudaMemcpyDeviceToHost,
+                                  h->copy_out));
+        LMOE_CUDA(cudaMemcpyAsync((char *)selected_experts_host + t0 * rs, dsel + t0 * rs, tj * rs,
+                                  cudaMemcpyDeviceToHost, h->copy_out));
+        LMOE_CUDA(cudaMemcpyAsync((char *)mixture_weights_host + t0 * rp, dp + t0 * rp, tj * rp,
+                                  cudaMemcpyDeviceToHost, h->copy_out));
+        LMOE_CUDA(cudaMemcpyAsync((char *)latent_routed_aggregate_host + t0 * ru, du + t0 * ru, tj * ru,
+                                  cudaMemcpyDeviceToHost, h->copy_out));
+    }
+    LMOE_CUDA(cudaEventRecord(ev[1], h->copy_out));
+    LMOE_CUDA(cudaStreamWaitEvent(s, ev[1], 0));
     return LMOE_OK;
 }
 

@@ -289,6 +289,31 @@ def test_side_stream_order_and_graph_capture_match_one_stream():
     layer.close()
 
 
+def test_host_entry_pipelines_chunks():
+    """Enough tokens for lmoe_forward_host to cut the batch into chunks whose
+    copies overlap the compute: each row equals lmoe_forward on the chunk that
+    holds it, bit for bit, and the whole batch matches the oracle."""
+    lm = _lm()
+    w = li.custom("host_chunks", 4200, 256, 128, 256, 16, 6, 256, dtype="bf16", seed=44)
+    x = li.tokens(w)
+    layer = _layer(w)
+    xh = x.pin_memory()
+    oh = layer.empty_outputs(w.T, device="cpu", pin=True)
+    layer.forward_host(xh, oh)
+    torch.cuda.synchronize()
+    layer.check_device(w.T)
+    Tc = (w.T + 1) // 2                      # max(2048, 192 E / k) = 2048 -> two chunks
+    for t0 in (0, Tc):
+        part = layer(x[t0:t0 + Tc].cuda())
+        torch.cuda.synchronize()
+        for key in part:
+            assert torch.equal(part[key].cpu(), oh[key][t0:t0 + Tc]), key
+    ora = oracle.forward(x, _weights(w), w.k, eps=w.eps)
+    compare(oh, ora, _weights(w)["b"].numpy(), TOL["bf16"],
+            lambda idx, sel: oracle.forward(x, _weights(w), w.k, rows=idx, sel=sel, eps=w.eps))
+    layer.close()
+
+
 def test_zero_tokens_is_a_noop_and_errors_are_reported():
     lm = _lm()
     w = MULTI
