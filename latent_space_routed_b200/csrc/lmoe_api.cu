@@ -141,9 +141,10 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     SplitPlan sp;
     sp.router = (h->tc && T > ROUTER_SMALL_MAX_T)
                     ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true, router_cg(T)) : 1;
-    sp.down = c.standard ? 1 : plan_ksplit(h, T, c.l, c.d / TC_BK);
-    sp.shared = plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
-    sp.final_ = plan_ksplit(h, T, c.d, ld_hs / TC_BK);
+    const bool gemv = h->tc && T <= GEMV_MAX_T;   // few tokens: dense GEMMs as weight-streaming GEMVs
+    sp.down = (c.standard || gemv) ? 1 : plan_ksplit(h, T, c.l, c.d / TC_BK);
+    sp.shared = gemv ? 1 : plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
+    sp.final_ = gemv ? 1 : plan_ksplit(h, T, c.d, ld_hs / TC_BK);
     auto need = [&](int ks, int64_t n) -> size_t { return ks > 1 ? (size_t)ks * (size_t)n * (size_t)T : 0; };
     sp.partial_floats = std::max(need(sp.router, c.E), need(sp.final_, c.d));
     sp.partial_side_floats = std::max(need(sp.down, c.l), need(sp.shared, 4 * (int64_t)c.f_shared));
@@ -604,7 +605,8 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     };
     auto st_down = [&](cudaStream_t q) -> lmoe_status {
         if (c.standard) return LMOE_OK;   // experts read x itself
-        if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down, partial_side, q));
+        if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_STORE, gd, q));
+        else if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down, partial_side, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, q));
         return LMOE_OK;
     };
@@ -628,12 +630,14 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         return LMOE_OK;
     };
     auto st_shared = [&](cudaStream_t q) -> lmoe_status {
-        if (h->tc) LMOE_CUDA(dense_tc(EPI_GLU, gs, sp.shared, partial_side, q));
+        if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_GLU, gs, q));
+        else if (h->tc) LMOE_CUDA(dense_tc(EPI_GLU, gs, sp.shared, partial_side, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, q));
         return LMOE_OK;
     };
     auto st_final = [&](cudaStream_t q) -> lmoe_status {
-        if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gf, sp.final_, partial, q));
+        if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_STORE, gf, q));
+        else if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gf, sp.final_, partial, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, q));
         return LMOE_OK;
     };

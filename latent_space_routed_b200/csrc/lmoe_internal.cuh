@@ -138,6 +138,11 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
                                  float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s,
                                  const void *residual = nullptr, int64_t ldr = 0);
+// Dense bf16 GEMM of a few tokens (g.M = T <= GEMV_MAX_T, rows of A and B
+// contiguous, K a multiple of 8) on CUDA cores, streaming B: EPI_STORE (with
+// the optional residual) or EPI_GLU (gate/up rows interleaved in blocks of ib).
+constexpr int GEMV_MAX_T = 2;
+cudaError_t launch_gemv(int mode, const GemmArgs &g, cudaStream_t s);
 // Router scores for a few tokens on CUDA cores: r[t, e] = sigmoid(sum_k x[t, k] W[e, k]),
 // x bf16 [T, d], W fp32 [E, d] (fixed summation order, deterministic).
 cudaError_t launch_router_small(const bf16 *x, const float *W, int64_t T, int E, int d, float *r, cudaStream_t s);

@@ -87,8 +87,10 @@ def test_bf16_situ_tensor_cores():
     run_parity(MULTI, act="situ")
 
 
-@pytest.mark.parametrize("T", [1, 2, 127, 129, 333])
+@pytest.mark.parametrize("T", [1, 2, 3, 6, 8, 9, 127, 129, 333])
 def test_bf16_token_counts(T):
+    """Token counts across the few-token plans (CUDA-core router and dense
+    GEMVs up to 8 tokens, split-K tensor-core GEMMs above) and ragged tiles."""
     run_parity(MULTI, T=T)
 
 
