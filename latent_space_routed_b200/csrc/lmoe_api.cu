@@ -75,6 +75,10 @@ lmoe_status lmoe::report_error(lmoe_status s, const char *msg)
     return s;
 }
 
+namespace {
+constexpr int HOST_MAX_CHUNKS = 8;   // chunks of one lmoe_forward_host call
+}  // namespace
+
 struct lmoe_handle {
     lmoe_config cfg;
     int device;
@@ -95,7 +99,7 @@ struct lmoe_handle {
     std::mutex fork_mutex;
     // lmoe_forward_host: copy streams and events of its chunk pipeline
     cudaStream_t copy_in = nullptr, copy_out = nullptr;
-    cudaEvent_t ev_host[2 + 2 * 8] = {};
+    cudaEvent_t ev_host[2 + 2 * HOST_MAX_CHUNKS] = {};
     std::mutex host_mutex;
 };
 
@@ -160,7 +164,6 @@ bool use_side_stream(const lmoe_handle *h) { return h->tc && h->side && !h->stag
 // independent, so chunking changes no row's arithmetic (only how a batch is
 // cut into launches); each chunk keeps at least 2048 tokens and enough slot
 // rows per expert (192 E / k tokens) for CTA-pair tiles.
-constexpr int HOST_MAX_CHUNKS = 8;
 int host_chunks(const lmoe_config &c, int64_t T, int64_t *Tc)
 {
     int64_t minc = (192LL * c.E + c.k - 1) / c.k;
