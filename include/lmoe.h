@@ -256,7 +256,8 @@ LMOE_API lmoe_status lmoe_set_stage_events(lmoe_handle *h, void *const *events, 
 #define LMOE_INJECT_FAIL_ALLOC 2
 LMOE_API lmoe_status lmoe_debug_inject(int32_t what, int32_t arg);
 
-/* Number of kernel launches one lmoe_forward of T tokens makes. */
+/* Number of kernels one lmoe_forward of T tokens launches (its two memsets,
+ * of the status word and of the per-block expert counts, are not counted). */
 LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches);
 
 /* Byte offset and size of one intermediate inside the forward workspace, so

@@ -432,13 +432,14 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
 {
     g_err.clear();
     if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
-    // status reset, router, histogram reset, top-k, scan, dispatch, down, permute, gate/up,
-    // down+combine, norm, shared, final; plus one reduction per split-K GEMM
-    // other than the router's (which the top-k kernel reduces)
+    // kernels: router, top-k, scan, dispatch, down (none in the standard form), permute,
+    // gate/up, down+combine, norm, shared, final; plus one reduction per split-K GEMM
+    // other than the router's (which the top-k kernel reduces).  The two memsets
+    // (status word, per-block expert counts) are not kernels and are not counted.
     if (T == 0) { *launches = 0; return LMOE_OK; }
     const lmoe_config &c = h->cfg;
     const SplitPlan sp = plan_splits(h, T);
-    *launches = 13 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
+    *launches = 11 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
     return LMOE_OK;
 }
 

@@ -316,6 +316,28 @@ def test_host_entry_pipelines_chunks():
     layer.close()
 
 
+def test_launch_count_matches_the_kernels_launched():
+    """lmoe_launch_count (the bench's gpu_launches) against the library
+    kernels a CUDA activity trace sees in one forward, for the one-or-two-token
+    plan and for the two-stream plan."""
+    from torch.profiler import profile, ProfilerActivity
+    w = MULTI
+    x = li.tokens(w).cuda()
+    layer = _layer(w)
+    layer(x)
+    torch.cuda.synchronize()
+    for T in (2, w.T):
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            layer(x[:T])
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if str(e.device_type).endswith("CUDA")]
+        if not names:
+            pytest.skip("no CUDA activity trace on this machine")
+        ours = [n for n in names if "lmoe" in n]
+        assert len(ours) == layer.launch_count(T), sorted(set(ours))
+    layer.close()
+
+
 def test_zero_tokens_is_a_noop_and_errors_are_reported():
     lm = _lm()
     w = MULTI
