@@ -395,6 +395,14 @@ def run_own(args, rank, world, local_rank):
                   "bound": "tensor" if Lf / (tf_burst * 1e12) >= Lb / (hbm * 1e9) else "hbm",
                   "achieved_tflops": Lf / (ms / 1e3) / 1e12, "achieved_gbs": Lb / (ms / 1e3) / 1e9,
                   "frac_of_sustained_tensor": (Lf / (tf_sus * 1e12)) / (ms / 1e3) if tf_sus else None}
+    # the two routed expert GEMMs together: the touched experts' weights (the
+    # decode workload's figure of merit) and all their algorithmic bytes
+    r_ms = stage_ms["gate_up"] + stage_ms["down_combine"]
+    r_weights = touched * 3 * w.l * w.f * w.item_bytes
+    r_bytes = model["gate_up"][1] + model["down_combine"][1]
+    routed = {"ms": r_ms, "touched_experts": touched, "weight_bytes": r_weights, "bytes": r_bytes,
+              "weight_gbs": r_weights / (r_ms / 1e3) / 1e9, "all_gbs": r_bytes / (r_ms / 1e3) / 1e9,
+              "weight_frac_of_hbm": r_weights / (r_ms / 1e3) / 1e9 / hbm}
 
     cpu = None
     if not args.no_cpu_baseline and world == 1:
@@ -411,7 +419,7 @@ def run_own(args, rank, world, local_rank):
                        "gemm": "tcgen05" if (args.gemm == 0 and w.dtype == "bf16") else "cuda-cores",
                        "l2": "flushed between timed steps (256 MiB write, untimed)",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-            "roofline": roof, "layer_roofline": layer_roof,
+            "roofline": roof, "layer_roofline": layer_roof, "routed": routed,
             "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "stages_note": "stages timed in a second pass with stage events set (one stream, no overlap)",
             "serial_ms_per_step": round(serial_ms, 4),
