@@ -153,12 +153,13 @@ LMOE_API lmoe_status lmoe_workspace_size(const lmoe_handle *h, int64_t T, size_t
  * Outputs must not overlap x, each other or the workspace.  T = 0 is a no-op.
  * Inputs must be finite.  Overlapping calls on one handle are allowed; calls
  * that share a workspace must be ordered on one stream.
- * On the tensor-core path, when no stage events are set and the shared GEMM
- * needs no K split (T >= 256 or so), the shared experts' gate/up GEMM runs on a
- * stream owned by the handle: forked from `stream` after the down-projection
- * and joined back into it before the final GEMM.  The call as a whole stays
- * ordered on `stream` and can be captured into a CUDA graph from it; while such
- * a capture is open, the handle's other forwards belong in that capture too.
+ * On the tensor-core path, when no stage events are set, the down-projection
+ * and the shared experts' gate/up GEMM run on a stream owned by the handle,
+ * forked from `stream` at the start of the call; `stream` waits for z before
+ * the permute and for the shared hidden before the routed gate/up GEMM.  The
+ * call as a whole stays ordered on `stream` and can be captured into a CUDA
+ * graph from it; while such a capture is open, the handle's other forwards
+ * belong in that capture too.
  * INVALID_ARG for null pointers (T > 0) or T < 0; WORKSPACE if ws_bytes is too
  * small or misaligned; CUDA if a launch fails. */
 LMOE_API lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output, int32_t *selected_experts,
@@ -265,9 +266,10 @@ LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t 
  * region: 0 router scores r [T, E] fp32; 1 mixture weights fp32 [T, k];
  * 2 per-expert counts [E] int32; 3 expert offsets [E+1] int32;
  * 4 slot index of (t, j) [T, k] int32; 5 token of each permuted slot [T*k]
- * int32; 6 latent rows z [T, l]; 7 routed hidden H [T*k, f] (slot order);
- * 8 p-weighted expert outputs [T*k, l] (token dtype); 9 [shared hidden | RMSNorm(u)]
- * [T, 2 f_shared + l]; 10 device status word (int32); 11 Quantile-Balancing
+ * int32; 6 latent rows z [T, l] (0 bytes in the standard form); 7 routed
+ * hidden H [T*k, f] (slot order); 8 p-weighted expert outputs [T*k, l] (token
+ * dtype); 9 [shared hidden | RMSNorm(u)] [T, 2 f_shared + l] (no RMSNorm
+ * columns in the standard form); 10 device status word (int32); 11 Quantile-Balancing
  * cutoff [T] fp32 (each token's (k+1)-th biased score, -inf when k = E).
  * INVALID_ARG for an unknown region. */
 LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t region, size_t *offset,
@@ -278,6 +280,10 @@ LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int3
  * LMOE_ERR_DEVICE_TIMEOUT if a bounded wait gave up (its outputs are then
  * invalid).  `workspace` is the one passed to lmoe_forward. */
 LMOE_API lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream);
+
+/* lmoe_check_device for the workspace of an lmoe_forward_host call of T
+ * tokens (its status word covers every chunk of the call). */
+LMOE_API lmoe_status lmoe_check_device_host(lmoe_handle *h, int64_t T, void *workspace, void *stream);
 
 /* Size of the scratch area built into the library for lmoe_forward_noalloc. */
 #define LMOE_NOALLOC_WORKSPACE_BYTES ((size_t)64 << 20)

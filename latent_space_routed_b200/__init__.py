@@ -33,7 +33,7 @@ REGION = {"scores": 0, "p32": 1, "counts": 2, "offsets": 3, "slot_of": 4, "perm_
           "Y": 8, "HS": 9, "status": 10, "cutoff": 11}
 
 EXPORTS = ("lmoe_config_from_base", "lmoe_create", "lmoe_workspace_size", "lmoe_forward", "lmoe_host_workspace_size",
-           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_debug_inject", "lmoe_set_bias", "lmoe_qb_histogram", "lmoe_qb_bias_update", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device",
+           "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_debug_inject", "lmoe_set_bias", "lmoe_qb_histogram", "lmoe_qb_bias_update", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device", "lmoe_check_device_host",
            "lmoe_last_error", "lmoe_destroy")
 
 
@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "lmoe_launch_count": (I32, [P, I64, ctypes.POINTER(I32)]),
         "lmoe_workspace_region": (I32, [P, I64, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)]),
         "lmoe_check_device": (I32, [P, I64, P, P]),
+        "lmoe_check_device_host": (I32, [P, I64, P, P]),
         "lmoe_last_error": (ctypes.c_char_p, []),
         "lmoe_destroy": (None, [P]),
     }
@@ -216,6 +217,10 @@ def lmoe_check_device(h, T, workspace, stream=None):
     _check(_lib.lmoe_check_device(h, T, _ptr(workspace), _stream(stream)))
 
 
+def lmoe_check_device_host(h, T, workspace, stream=None):
+    _check(_lib.lmoe_check_device_host(h, T, _ptr(workspace), _stream(stream)))
+
+
 # ------------------------------------------------------------------ convenience wrapper
 _TORCH_DT = {LMOE_F32: torch.float32, LMOE_BF16: torch.bfloat16}
 
@@ -306,6 +311,10 @@ class LatentMoE:
 
     def check_device(self, T: int, stream=None):
         lmoe_check_device(self.handle, T, self.workspace(T), stream)
+
+    def check_device_host(self, T: int, stream=None):
+        """lmoe_check_device after forward_host of T tokens."""
+        lmoe_check_device_host(self.handle, T, self.workspace(T, host=True), stream)
 
     def launch_count(self, T: int) -> int:
         return lmoe_launch_count(self.handle, T)

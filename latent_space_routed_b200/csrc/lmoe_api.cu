@@ -717,12 +717,10 @@ lmoe_status lmoe_forward(lmoe_handle *h, const void *x, int64_t T, void *output,
                         ws_bytes, stream, true);
 }
 
-lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes)
+// Bytes of the device staging of x and the four outputs in front of the
+// forward workspace inside an lmoe_forward_host workspace.
+static size_t host_staging_bytes(const lmoe_handle *h, int64_t T)
 {
-    g_err.clear();
-    if (!h || !bytes) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
-    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
-    if (T == 0) { *bytes = 0; return LMOE_OK; }
     const lmoe_config &c = h->cfg;
     size_t o = 0;
     o = align_up(o + h->tb * T * c.d, 256);          // x
@@ -730,6 +728,17 @@ lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *by
     o = align_up(o + sizeof(int32_t) * T * c.k, 256);
     o = align_up(o + h->tb * T * c.k, 256);
     o = align_up(o + h->tb * T * c.l, 256);
+    return o;
+}
+
+lmoe_status lmoe_host_workspace_size(const lmoe_handle *h, int64_t T, size_t *bytes)
+{
+    g_err.clear();
+    if (!h || !bytes) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
+    if (T == 0) { *bytes = 0; return LMOE_OK; }
+    const lmoe_config &c = h->cfg;
+    const size_t o = host_staging_bytes(h, T);
     int64_t Tc = T;
     const int nc = host_chunks(c, T, &Tc);
     size_t fw = plan(h, Tc).total;                       // the chunks' forward workspace
@@ -813,22 +822,37 @@ lmoe_status lmoe_forward_host(lmoe_handle *h, const void *x_host, int64_t T, voi
     return LMOE_OK;
 }
 
+// Read and clear the device status word at `word`.
+static lmoe_status check_status_word(char *word, cudaStream_t s)
+{
+    int32_t v = 0;
+    LMOE_CUDA(cudaMemcpyAsync(&v, word, sizeof v, cudaMemcpyDeviceToHost, s));
+    LMOE_CUDA(cudaStreamSynchronize(s));
+    if (v != 0) {
+        LMOE_CUDA(cudaMemsetAsync(word, 0, sizeof(int32_t), s));
+        LMOE_CUDA(cudaStreamSynchronize(s));
+        return fail(LMOE_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait gave up (status word 0x%x)", v);
+    }
+    return LMOE_OK;
+}
+
 lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream)
 {
     g_err.clear();
     if (!h || !workspace) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
     if (T < 1) return LMOE_OK;
-    const Layout L = plan(h, T);
-    int32_t v = 0;
-    cudaStream_t s = (cudaStream_t)stream;
-    LMOE_CUDA(cudaMemcpyAsync(&v, (char *)workspace + L.status, sizeof v, cudaMemcpyDeviceToHost, s));
-    LMOE_CUDA(cudaStreamSynchronize(s));
-    if (v != 0) {
-        LMOE_CUDA(cudaMemsetAsync((char *)workspace + L.status, 0, sizeof(int32_t), s));
-        LMOE_CUDA(cudaStreamSynchronize(s));
-        return fail(LMOE_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait gave up (status word 0x%x)", v);
-    }
-    return LMOE_OK;
+    return check_status_word((char *)workspace + plan(h, T).status, (cudaStream_t)stream);
+}
+
+lmoe_status lmoe_check_device_host(lmoe_handle *h, int64_t T, void *workspace, void *stream)
+{
+    g_err.clear();
+    if (!h || !workspace) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (T < 1) return LMOE_OK;
+    // the forward workspace follows the staging of x and the four outputs; its
+    // status word is first in every chunk's layout
+    return check_status_word((char *)workspace + host_staging_bytes(h, T) + plan(h, 1).status,
+                             (cudaStream_t)stream);
 }
 
 }  // extern "C"

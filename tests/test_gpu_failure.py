@@ -42,6 +42,35 @@ def test_bounded_wait_runs_out_and_is_reported():
     layer.close()
 
 
+@pytest.mark.parametrize("T", [256, 4200])
+def test_bounded_wait_is_reported_through_the_host_entry(T):
+    """lmoe_forward_host (at 4200 tokens cut into two pipelined chunks): a wait
+    that runs out in the first chunk stays in the status word through the
+    later chunks, and lmoe_check_device_host reports it."""
+    import latent_space_routed_b200 as lm
+    w = li.custom("failure_host", T, 256, 128, 256, 16, 6, 256, dtype="bf16", seed=42)
+    layer = lm.LatentMoE(lm.config_for(w), {k: v.cuda() for k, v in li.weights(w).items()})
+    xh = li.tokens(w).pin_memory()
+    ref = layer.empty_outputs(T, device="cpu", pin=True)
+    layer.forward_host(xh, ref)
+    torch.cuda.synchronize()
+    layer.check_device_host(T)
+
+    lm.lmoe_debug_inject(lm.LMOE_INJECT_STALL_NEXT_GEMM)
+    out = layer.empty_outputs(T, device="cpu", pin=True)
+    layer.forward_host(xh, out)
+    with pytest.raises(lm.LmoeError) as ei:
+        layer.check_device_host(T)
+    assert ei.value.status == lm.LMOE_ERR_DEVICE_TIMEOUT
+
+    layer.forward_host(xh, out)                  # the context is still usable
+    torch.cuda.synchronize()
+    layer.check_device_host(T)
+    for key in ref:
+        assert torch.equal(out[key], ref[key]), key
+    layer.close()
+
+
 @pytest.mark.parametrize("which", [1, 3, 7])
 def test_injected_allocation_failure(which):
     import latent_space_routed_b200 as lm

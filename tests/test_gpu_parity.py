@@ -303,7 +303,7 @@ def test_host_entry_pipelines_chunks():
     oh = layer.empty_outputs(w.T, device="cpu", pin=True)
     layer.forward_host(xh, oh)
     torch.cuda.synchronize()
-    layer.check_device(w.T)
+    layer.check_device_host(w.T)
     Tc = (w.T + 1) // 2                      # max(2048, 192 E / k) = 2048 -> two chunks
     for t0 in (0, Tc):
         part = layer(x[t0:t0 + Tc].cuda())
