@@ -130,7 +130,7 @@ def test_standard_moe_form(dtype, gemm):
     run_parity(w, gemm=gemm)
 
 
-@pytest.mark.parametrize("T", [5, 100])
+@pytest.mark.parametrize("T", [2, 5, 100])
 def test_standard_moe_form_few_tokens(T):
     """Few tokens: CUDA-core router and split-K final GEMM, whose reduction
     adds u."""
