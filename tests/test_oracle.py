@@ -323,6 +323,41 @@ def test_single_expert_is_a_dense_swiglu_mlp_between_two_linear_maps():
     np.testing.assert_array_equal(out["mixture_weights"], 1.0)
 
 
+def test_identity_projections_without_norm_are_the_standard_moe():
+    """The standard-MoE form the library offers (cooking-agi page: a standard
+    MoE routes and computes its experts at the model width) is the oracle's
+    layer with W_down = W_up = I and no norm.  Checked against torch's topk,
+    linear and silu at width d: r = sigmoid(W_r x), the top k of r + b,
+    p = r_sel / sum r_sel, y = sum_j p_j E_j(x) + S_1(x) + S_2(x)."""
+    rng = np.random.default_rng(8)
+    d, f, fs, E, k, T = 6, 5, 3, 5, 2, 9
+    F = torch.nn.functional
+    Wr, b = rng.standard_normal((E, d)), rng.uniform(-0.05, 0.05, E)
+    G, U, D = rng.standard_normal((E, f, d)), rng.standard_normal((E, f, d)), rng.standard_normal((E, d, f))
+    Gs, Us, Ds = rng.standard_normal((2, fs, d)), rng.standard_normal((2, fs, d)), rng.standard_normal((2, d, fs))
+    x = rng.standard_normal((T, d))
+    w = _weights(W_r=Wr, b=b, W_down=np.eye(d), W_up=np.eye(d), G=G, U=U, D=D, Gs=Gs, Us=Us, Ds=Ds)
+    out = oracle.forward(_f32(x), w, k, use_norm=False)
+    t = lambda a: torch.tensor(_f32(a), dtype=torch.float64)
+    X = t(x)
+    r = torch.sigmoid(F.linear(X, t(Wr)))
+    sel = torch.topk(r + t(b), k, dim=1).indices
+    y = torch.zeros(T, d, dtype=torch.float64)
+    u = torch.zeros(T, d, dtype=torch.float64)
+    for i in range(T):
+        rs = r[i, sel[i]]
+        for j in range(k):
+            e = int(sel[i, j])
+            h = F.silu(F.linear(X[i], t(G)[e])) * F.linear(X[i], t(U)[e])
+            u[i] += rs[j] / rs.sum() * F.linear(h, t(D)[e])
+    y += u
+    for j in range(2):
+        y = y + F.linear(F.silu(F.linear(X, t(Gs)[j])) * F.linear(X, t(Us)[j]), t(Ds)[j])
+    np.testing.assert_array_equal(out["selected_experts"], sel.numpy())
+    np.testing.assert_allclose(out["latent_routed_aggregate"], u.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(out["output"], y.numpy(), rtol=1e-12, atol=1e-12)
+
+
 def test_shared_only_is_two_swiglu_mlps():
     """Routed path zeroed (D = 0, so u = 0 and RMSNorm(0) = 0): y is the sum of
     the two shared SwiGLU experts, each on the full-width x (Hint 2)."""
