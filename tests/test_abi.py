@@ -96,3 +96,29 @@ def test_null_arguments():
     assert lib.lmoe_create(ctypes.byref(cfg), None, None, ctypes.byref(h)) == lm.LMOE_ERR_INVALID_ARG
     assert lib.lmoe_create(None, None, None, ctypes.byref(h)) == lm.LMOE_ERR_INVALID_ARG
     lib.lmoe_destroy(None)   # ignored
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the built library the package refuses to import (no fallback)."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "latent_space_routed_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(os.path.dirname(lm.__file__), "__init__.py"), pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import latent_space_routed_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0
+    assert "liblmoe.so is missing" in r.stderr
+
+
+def test_product_never_reaches_the_oracle():
+    """The package and its sources name neither the oracle nor a CPU path for the layer."""
+    root = os.path.dirname(lm.__file__)
+    for dirpath, _, files in os.walk(root):
+        for name in files:
+            if name.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, name)).read()
+                assert "import oracle" not in text and "from oracle" not in text, name
+                assert "lmoe_oracle" not in text, name
+
