@@ -147,6 +147,14 @@ def test_bf16_pair_tiles_skewed_expert_loads(bias):
     run_parity(w)
 
 
+@pytest.mark.parametrize("T", [2, 4])
+def test_bf16_few_slot_rows_per_expert(T):
+    """Fewer slot rows than experts (S <= E, the decode regime at a small
+    size): single-CTA tiles with one or two real rows each; every row compared."""
+    w = li.custom("grouped_split", 4, 512, 512, 512, 64, 4, 256, dtype="bf16", seed=45)
+    run_parity(w, T=T)
+
+
 def test_fp32_multi_tile_ragged():
     w = li.custom("multi_f32", 333, 256, 128, 128, 24, 5, 192, dtype="f32", seed=23)
     run_parity(w)
