@@ -1,18 +1,26 @@
 #!/usr/bin/env python
 """LatentMoE layer-forward benchmark on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--T T]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME [--T T]]
     python bench.py --impl reference ...
 
 One step = one whole layer forward (router, top-k, dispatch, down-projection,
 routed experts, combine, RMSNorm, shared experts, up-projection) over the
 workload's batch, inputs resident in HBM.  Prints one JSON line (rank 0).
 
-N > 1 (launched with torch.distributed.run) runs N independent replicas, one
-per GPU, each on its own batch: the layer's rows are independent and there is
-no exchange step, so there is no data-path collective (weak scaling).  The
-NCCL process group is used only for the barrier and the max over ranks of the
-timed region.
+With no --workload the headline is large_d4096 (T 32768, d 4096, 512 experts,
+top 24), the largest single-GPU workload; the same run also measures
+acc_d2048, eff_zipf_d2048, std_d2048 and the decode_d7168 sweep (T = 1, 8,
+32, 128, also replayed from a CUDA graph) and reports them under
+``workloads``.  ``--save DIR`` writes each workload's full line to
+DIR/bench_<workload>[_T<T>].json.
+
+N > 1 runs N independent replicas, one per GPU, each on its own batch: the
+layer's rows are independent and there is no exchange step, so there is no
+data-path collective (weak scaling).  The process group is used only for the
+barrier and the max over ranks of the timed region.  Launched without
+torch.distributed.run (no WORLD_SIZE in the environment), ``--gpus N`` starts
+the N ranks itself through torch.distributed.run on 127.0.0.1.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference this
 layer has) on the host cores, each step a bounded sample of token rows.
@@ -24,6 +32,7 @@ import ctypes
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -35,41 +44,55 @@ sys.path.insert(0, ROOT)
 METRIC = "LatentMoE layer fwd tokens/s on 1 B200; % of tensor-core or HBM roofline"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+HEADLINE = "large_d4096"
+OTHERS = (("acc_d2048", None), ("eff_zipf_d2048", None), ("std_d2048", None),
+          ("decode_d7168", 1), ("decode_d7168", 8), ("decode_d7168", 32), ("decode_d7168", 128))
+# B200 datasheet figures (dense bf16 tensor, HBM3e), beside the measured peaks
+SPEC_TFLOPS, SPEC_GBS = 2250.0, 7700.0
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
-    ap.add_argument("--workload", default="acc_d2048")
+    ap.add_argument("--workload", default=None, help="one workload only (default: the headline and the others)")
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--gemm", type=int, default=0, help="0 tensor cores, 1 CUDA cores")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--graph", action="store_true", help="also time the forward replayed from a CUDA graph")
-    return ap.parse_args()
+    ap.add_argument("--save", default=None, help="directory for one JSON file per workload line")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="CPU only: start the ranks, time a trivial step per rank over gloo and print the line "
+                         "(checks the multi-rank launch and aggregation without a GPU)")
+    return ap.parse_args(argv)
 
 
-def measured_traffic(workload, T, kernel):
-    """DRAM bytes per launch of `kernel` from a committed ncu summary under
-    profiles/, or None when none matches or the kernel sources changed since."""
-    import glob
+def source_hash():
+    """Hash of the GEMM and planner sources a traffic capture was taken from."""
     import hashlib
-    import re
     h = hashlib.sha256()
     for f in ("latent_space_routed_b200/csrc/gemm_tc.cu", "latent_space_routed_b200/csrc/lmoe_api.cu"):
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    sha = h.hexdigest()[:16]
-    pat = re.compile(r"^traffic: workload=(\S+) T=(\d+) kernel=(\S+) bytes=(\d+) sources=(\w+)")
-    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
-        with open(path) as fh:
-            for line in fh:
-                m = pat.match(line.strip())
-                if m and m.group(1) == workload and int(m.group(2)) == T and m.group(3) == kernel:
-                    return int(m.group(4)) if m.group(5) == sha else None
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, T, kernel):
+    """DRAM bytes per launch of `kernel` at T tokens from profiles/traffic.json
+    (ncu dram__bytes_read.sum + dram__bytes_write.sum), or None when no entry
+    matches or the kernel sources changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as fh:
+            entries = json.load(fh)["entries"]
+    except (OSError, ValueError, KeyError):
+        return None
+    sha = source_hash()
+    for e in entries:
+        if e["workload"] == workload and e["T"] == T and e["kernel"] == kernel:
+            return int(e["bytes_per_launch"]) if e["sources"] == sha else None
     return None
 
 
@@ -142,6 +165,18 @@ def replica_seed(w, rank: int) -> int:
     return w.seed + 1000 * rank
 
 
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launcher_cmd(argv, gpus: int, port: int):
+    """torch.distributed.run command that starts `gpus` ranks of this script."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
 # ---------------------------------------------------------------- clocks
 class Clocks:
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -210,7 +245,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     import lmoe_inputs as li
-    w = li.WORKLOADS[args.workload]
+    w = li.WORKLOADS[args.workload or HEADLINE]
     T = args.T or w.T
     x, W = li.tokens(w, T), li.weights(w)
     # one step = the oracle on a bounded sample of rows, sized to ~4 s
@@ -239,20 +274,24 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------- own arm
-def run_own(args, rank, world, local_rank):
-    import numpy as np
+def _roofline(fl, by, ms, hbm, tf):
+    """Roofline object of `ms` per launch for fl FLOPs and by bytes."""
+    t_s = ms / 1e3
+    if fl / (tf * 1e12) >= by / (hbm * 1e9):
+        r = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": tf, "unit": "TFLOP/s",
+             "frac_of_spec": fl / t_s / 1e12 / SPEC_TFLOPS}
+    else:
+        r = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": hbm, "unit": "GB/s",
+             "frac_of_spec": by / t_s / 1e9 / SPEC_GBS}
+    r["frac"] = r["achieved"] / r["peak"]
+    return r
+
+
+def measure(args, w, T, layer, x_cpu, W, rank, world, dev, *, headline):
+    """Time one workload at T tokens on an existing layer; returns the full line."""
     import torch
-    import lmoe_inputs as li
     import latent_space_routed_b200 as lm
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = li.WORKLOADS[args.workload]
-    T = args.T or w.T
-    W = li.weights(w)
-    x_cpu = li.tokens(w, T, seed=replica_seed(w, rank))
-    layer = lm.LatentMoE(lm.config_for(w, gemm=args.gemm), {k: v.to(dev) for k, v in W.items()})
-    torch.cuda.empty_cache()   # the caller-side weight copies are no longer needed (the handle repacked them)
     x = x_cpu.to(dev)
     out = layer.empty_outputs(T)
     stream = torch.cuda.current_stream()
@@ -283,11 +322,10 @@ def run_own(args, rank, world, local_rank):
     ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
 
-    gpu_id = 0
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
-        gpu_id = local_rank
+        gpu_id = dev.index
     clocks = Clocks(gpu_id)
     time.sleep(0.5)
     if world > 1:
@@ -321,7 +359,7 @@ def run_own(args, rank, world, local_rank):
     serial_ms = sum(ev_stage[i][0].elapsed_time(ev_stage[i][ns - 1]) for i in range(args.steps)) / args.steps
 
     graph_ms = None
-    if args.graph:
+    if args.graph or T <= 128:
         # the same forward captured once into a CUDA graph and replayed (no host launch gaps)
         layer.workspace(T)
         side = torch.cuda.Stream()
@@ -338,13 +376,15 @@ def run_own(args, rank, world, local_rank):
         torch.cuda.synchronize()
         g_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         g_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
         for i in range(args.steps):
             flush.fill_(float(i))
             g_a[i].record(stream)
             graph.replay()
             g_b[i].record(stream)
         torch.cuda.synchronize()
-        graph_ms = sum(a.elapsed_time(b) for a, b in zip(g_a, g_b)) / args.steps
+        graph_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(g_a, g_b)), dev) / args.steps
         del graph
         layer.check_device(T)
 
@@ -364,14 +404,15 @@ def run_own(args, rank, world, local_rank):
         layer.forward_host(x_host, out_host)
         e_b[i].record(stream)
     torch.cuda.synchronize()
+    layer.check_device_host(T)
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_a, e_b)), dev)
     B = w.item_bytes
     h2d = T * w.d * B
     d2h = T * w.d * B + T * w.k * 4 + T * w.k * B + T * w.l * B
+    del x, out, flush, x_host, out_host
 
     if rank != 0:
-        layer.close()
-        return
+        return None
 
     hbm, tf_burst, tf_sus, peak_src = peaks()
     ms = total_ms / args.steps
@@ -379,22 +420,19 @@ def run_own(args, rank, world, local_rank):
     model = stage_model(w, T, touched)
     dom = max(stage_ms, key=lambda k: stage_ms[k])
     fl, by = model[dom]
-    t_s = stage_ms[dom] / 1e3
-    if fl / (tf_burst * 1e12) >= by / (hbm * 1e9):
-        roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": tf_burst, "unit": "TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": hbm, "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof = _roofline(fl, by, stage_ms[dom], hbm, tf_burst)
     roof["traffic"] = measured_traffic(w.name, T, dom)
     roof["kernel"] = dom
     roof["per_launch"] = {"flops": fl, "bytes": by, "ms": stage_ms[dom]}
-    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst bf16 / copy bandwidth)"
+    roof["peak_source"] = (f"{peak_src} (MEASURED_PEAKS.json burst bf16 / copy bandwidth); "
+                           f"frac_of_spec against the B200 datasheet {SPEC_TFLOPS:.0f} TFLOP/s / {SPEC_GBS:.0f} GB/s")
     Lf, Lb = layer_flops(w, T), layer_bytes(w, T, touched)
     t_roof = max(Lf / (tf_burst * 1e12), Lb / (hbm * 1e9))
+    bound = "tensor" if Lf / (tf_burst * 1e12) >= Lb / (hbm * 1e9) else "hbm"
     layer_roof = {"flops": Lf, "bytes": Lb, "roofline_ms": t_roof * 1e3, "frac": t_roof / (ms / 1e3),
-                  "bound": "tensor" if Lf / (tf_burst * 1e12) >= Lb / (hbm * 1e9) else "hbm",
-                  "achieved_tflops": Lf / (ms / 1e3) / 1e12, "achieved_gbs": Lb / (ms / 1e3) / 1e9,
-                  "frac_of_sustained_tensor": (Lf / (tf_sus * 1e12)) / (ms / 1e3) if tf_sus else None}
+                  "bound": bound, "achieved_tflops": Lf / (ms / 1e3) / 1e12, "achieved_gbs": Lb / (ms / 1e3) / 1e9,
+                  "frac_of_sustained_tensor": (Lf / (tf_sus * 1e12)) / (ms / 1e3) if tf_sus else None,
+                  "frac_of_spec": max(Lf / (SPEC_TFLOPS * 1e12), Lb / (SPEC_GBS * 1e9)) / (ms / 1e3)}
     # the two routed expert GEMMs together: the touched experts' weights (the
     # decode workload's figure of merit) and all their algorithmic bytes
     r_ms = stage_ms["gate_up"] + stage_ms["down_combine"]
@@ -405,7 +443,7 @@ def run_own(args, rank, world, local_rank):
               "weight_frac_of_hbm": r_weights / (r_ms / 1e3) / 1e9 / hbm}
 
     cpu = None
-    if not args.no_cpu_baseline and world == 1:
+    if headline and not args.no_cpu_baseline and world == 1:
         v, n, dt, cores = time_oracle(w, x_cpu, W, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} seeded token rows of the {T}-token batch in {dt:.1f} s (fp64 C oracle)"}
@@ -431,15 +469,119 @@ def run_own(args, rank, world, local_rank):
     if graph_ms is not None:
         line["graph"] = {"ms_per_step": graph_ms, "value": world * T / (graph_ms / 1e3), "unit": UNIT,
                          "layer_frac": t_roof / (graph_ms / 1e3)}
-    print(json.dumps(line), flush=True)
-    layer.close()
+    return line
 
 
-def main():
-    args = parse()
+def summary(line):
+    """The per-workload entry of the headline line's `workloads` object."""
+    s = {"T": line["config"]["T"], "ms_per_step": line["ms_per_step"], "tokens_per_s": line["value"],
+         "layer_frac": line["layer_roofline"]["frac"], "layer_bound": line["layer_roofline"]["bound"],
+         "dominant_kernel": line["roofline"]["kernel"], "dominant_kernel_frac": line["roofline"]["frac"],
+         "routed_weight_gbs": line["routed"]["weight_gbs"],
+         "routed_weight_frac_of_hbm": line["routed"]["weight_frac_of_hbm"],
+         "e2e_tokens_per_s": line["e2e"]["value"], "clocks": line["clocks"]}
+    if "graph" in line:
+        s["graph_ms_per_step"] = line["graph"]["ms_per_step"]
+        s["graph_layer_frac"] = line["graph"]["layer_frac"]
+    return s
+
+
+def _save(args, line):
+    if not args.save:
+        return
+    os.makedirs(args.save, exist_ok=True)
+    c = line["config"]
+    name = f"bench_{c['workload']}" + (f"_T{c['T']}" if c["workload"] == "decode_d7168" else "") + ".json"
+    with open(os.path.join(args.save, name), "w") as fh:
+        json.dump(line, fh, indent=1)
+
+
+def run_own(args, rank, world, local_rank):
+    import torch
+    import lmoe_inputs as li
+    import latent_space_routed_b200 as lm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if args.workload:
+        plan = [(args.workload, [args.T])]
+        headline = args.workload
+    else:
+        plan = [(HEADLINE, [None])]
+        for name, T in OTHERS:
+            if plan[-1][0] == name:
+                plan[-1][1].append(T)
+            else:
+                plan.append((name, [T]))
+        headline = HEADLINE
+    lines = []
+    for name, Ts in plan:
+        w = li.WORKLOADS[name]
+        W = li.weights(w)
+        layer = lm.LatentMoE(lm.config_for(w, gemm=args.gemm), {k: v.to(dev) for k, v in W.items()})
+        torch.cuda.empty_cache()   # the caller-side weight copies are no longer needed (the handle repacked them)
+        for T in Ts:
+            T = T or w.T
+            x_cpu = li.tokens(w, T, seed=replica_seed(w, rank))
+            line = measure(args, w, T, layer, x_cpu, W, rank, world, dev, headline=(name == headline and not lines))
+            if line is not None:
+                _save(args, line)
+                lines.append(line)
+        layer.close()
+        del layer, W
+        torch.cuda.empty_cache()
+    if rank != 0:
+        return
+    head = lines[0]
+    if len(lines) > 1:
+        head["workloads"] = {}
+        for ln in lines[1:]:
+            c = ln["config"]
+            key = c["workload"] + (f"_T{c['T']}" if c["workload"] == "decode_d7168" else "")
+            head["workloads"][key] = summary(ln)
+    print(json.dumps(head), flush=True)
+
+
+def run_launch_check(args, rank, world):
+    """The multi-rank plumbing on CPU ranks over gloo: barrier, a trivial timed
+    step per rank, max over ranks, the whole-job aggregate."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        T = 1024
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        a = torch.ones(256, 256)
+        for _ in range(args.steps):
+            a = a @ a * 1e-3
+        per_rank_ms = (time.perf_counter() - t0) * 1e3 + 5.0 * rank
+        job_ms = max_over_ranks(per_rank_ms, "cpu")
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "launch_check": True, "n_gpus": world, "rank_ms": per_rank_ms,
+                              "job_ms": job_ms, "value": job_tokens_per_s(world, T, job_ms / args.steps),
+                              "unit": UNIT, "steps": args.steps, "warmup": args.warmup}), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse(argv)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # started as a plain script with --gpus N: start the N ranks here
+        r = subprocess.run(launcher_cmd(argv, args.gpus, _free_port()))
+        sys.exit(r.returncode)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.launch_check:
+        run_launch_check(args, rank, world)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

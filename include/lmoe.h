@@ -205,8 +205,9 @@ LMOE_API lmoe_status lmoe_set_bias(lmoe_handle *h, const float *b, void *stream)
  * scores and cutoff[t] the token's (k+1)-th biased score (workspace region 11);
  * its bin is computed in fp32 as x = (m - lo) * (bins / (hi - lo)): bin 0 if
  * x < 0, bins - 1 if x >= bins, floor(x) otherwise.  Reads workspace regions 0
- * and 11, which the next forward on that workspace overwrites.
- * INVALID_ARG: NULL pointer, T < 0, bins outside [1, 2^20], lo or hi not
+ * and 11, which the next forward on that workspace overwrites.  workspace
+ * NULL reads the built-in area of lmoe_forward_noalloc (handle's device current).
+ * INVALID_ARG: NULL handle or hist, T < 0, bins outside [1, 2^20], lo or hi not
  * finite, hi <= lo.  T = 0 adds nothing. */
 LMOE_API lmoe_status lmoe_qb_histogram(const lmoe_handle *h, const void *workspace, int64_t T, int32_t bins,
                                        float lo, float hi, int32_t *hist, void *stream);
@@ -278,7 +279,9 @@ LMOE_API lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int3
 /* Synchronise `stream`, then read and clear the device status word that the
  * kernels of the last forward on this workspace wrote: LMOE_OK, or
  * LMOE_ERR_DEVICE_TIMEOUT if a bounded wait gave up (its outputs are then
- * invalid).  `workspace` is the one passed to lmoe_forward. */
+ * invalid).  `workspace` is the one passed to lmoe_forward, or NULL for the
+ * built-in area of lmoe_forward_noalloc (the handle's device must then be
+ * current; INVALID_ARG otherwise). */
 LMOE_API lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream);
 
 /* lmoe_check_device for the workspace of an lmoe_forward_host call of T
@@ -306,6 +309,11 @@ LMOE_API lmoe_status lmoe_check_device_host(lmoe_handle *h, int64_t T, void *wor
  *  - All calls on a device share the area and find the previous call's data
  *    in it (the forward resets what must start at zero itself).  Calls that
  *    overlap on the GPU race on it: order them on one stream.
+ *  - The device the handle was created on must be current: INVALID_ARG
+ *    otherwise.
+ *  - lmoe_check_device (and lmoe_qb_histogram) with workspace NULL read this
+ *    area: the status word of the last call, LMOE_ERR_DEVICE_TIMEOUT if one of
+ *    its bounded waits gave up.
  * Errors as lmoe_forward. */
 LMOE_API lmoe_status lmoe_forward_noalloc(lmoe_handle *h, const void *x, int64_t T, void *output,
                                           int32_t *selected_experts, void *mixture_weights,

@@ -103,6 +103,8 @@ struct lmoe_handle {
     std::mutex host_mutex;
 };
 
+int lmoe::handle_device(const lmoe_handle *h) { return h->device; }
+
 namespace {
 
 // Few-token plans.  The router runs on CUDA cores for a handful of tokens;
@@ -455,7 +457,15 @@ lmoe_status lmoe_qb_histogram(const lmoe_handle *h, const void *workspace, int64
                               int32_t *hist, void *stream)
 {
     g_err.clear();
-    if (!h || !workspace || !hist) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (!h || !hist) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (!workspace && T > 0) {   // the built-in area of lmoe_forward_noalloc
+        void *area = nullptr;
+        size_t area_bytes = 0;
+        const lmoe_status st = noalloc_area_for(h, &area, &area_bytes);
+        if (st != LMOE_OK) return st;
+        if (plan(h, T).total > area_bytes) return fail(LMOE_ERR_WORKSPACE, "T exceeds the built-in area");
+        workspace = area;
+    }
     if (T < 0) return fail(LMOE_ERR_INVALID_ARG, "T < 0");
     if (bins < 1 || bins > (1 << 20)) return fail(LMOE_ERR_INVALID_ARG, "bins=%d outside [1, 2^20]", bins);
     if (!std::isfinite(lo) || !std::isfinite(hi) || !(hi > lo)) return fail(LMOE_ERR_INVALID_ARG, "need finite lo < hi");
@@ -839,8 +849,13 @@ static lmoe_status check_status_word(char *word, cudaStream_t s)
 lmoe_status lmoe_check_device(lmoe_handle *h, int64_t T, void *workspace, void *stream)
 {
     g_err.clear();
-    if (!h || !workspace) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
+    if (!h) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
     if (T < 1) return LMOE_OK;
+    if (!workspace) {   // the built-in area of lmoe_forward_noalloc
+        size_t area_bytes = 0;
+        const lmoe_status st = noalloc_area_for(h, &workspace, &area_bytes);
+        if (st != LMOE_OK) return st;
+    }
     return check_status_word((char *)workspace + plan(h, T).status, (cudaStream_t)stream);
 }
 

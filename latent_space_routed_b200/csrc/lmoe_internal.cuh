@@ -14,6 +14,14 @@ typedef __nv_bfloat16 bf16;
 // Record `msg` as the calling thread's lmoe_last_error() and return `s`.
 lmoe_status report_error(lmoe_status s, const char *msg);
 
+// Device the handle was created on (its weights live there).
+int handle_device(const lmoe_handle *h);
+
+// Device address of the library's built-in scratch area (lmoe_forward_noalloc)
+// on the handle's device, which must be current: LMOE_ERR_INVALID_ARG when it
+// is not, LMOE_ERR_CUDA when the address lookup fails.  *bytes gets its size.
+lmoe_status noalloc_area_for(const lmoe_handle *h, void **area, size_t *bytes);
+
 // ---------------------------------------------------------------- conversions
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }

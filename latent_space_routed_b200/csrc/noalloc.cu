@@ -22,6 +22,11 @@
 //    start at zero (its status word and per-block expert counts) itself.
 //    Calls that overlap on the GPU (different streams, or different handles on
 //    the same device without ordering) race on the area: order them.
+//  - The handle's device must be current (the area of another device would
+//    hold none of its data); otherwise the call returns LMOE_ERR_INVALID_ARG.
+//  - lmoe_check_device and lmoe_qb_histogram given a NULL workspace read the
+//    area, so the status word and the router statistics of this entry point
+//    stay reachable.
 //  - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 #include <mutex>
 
@@ -61,6 +66,23 @@ lmoe_status noalloc_area(void **out)
 
 }  // namespace
 
+lmoe_status lmoe::noalloc_area_for(const lmoe_handle *h, void **area, size_t *bytes)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return lmoe::report_error(LMOE_ERR_CUDA, "cudaGetDevice failed");
+    }
+    if (dev != lmoe::handle_device(h))
+        return lmoe::report_error(LMOE_ERR_INVALID_ARG,
+                                  "the current device is not the one the handle was created on: make the "
+                                  "handle's device current before using the built-in scratch area");
+    const lmoe_status st = noalloc_area(area);
+    if (st != LMOE_OK) return lmoe::report_error(st, "cudaGetSymbolAddress of the built-in scratch area failed");
+    *bytes = kNoallocBytes;
+    return LMOE_OK;
+}
+
 extern "C" lmoe_status lmoe_forward_noalloc(lmoe_handle *h, const void *x, int64_t T, void *output,
                                             int32_t *selected_experts, void *mixture_weights,
                                             void *latent_routed_aggregate, void *stream)
@@ -76,8 +98,9 @@ extern "C" lmoe_status lmoe_forward_noalloc(lmoe_handle *h, const void *x, int64
                                   "T tokens need more scratch than the built-in area of LMOE_NOALLOC_WORKSPACE_BYTES "
                                   "(64 MiB): use lmoe_forward with a caller workspace, or fewer tokens per call");
     void *area = nullptr;
-    st = noalloc_area(&area);
-    if (st != LMOE_OK) return lmoe::report_error(st, "cudaGetSymbolAddress of the built-in scratch area failed");
+    size_t area_bytes = 0;
+    st = lmoe::noalloc_area_for(h, &area, &area_bytes);
+    if (st != LMOE_OK) return st;
     return lmoe_forward(h, x, T, output, selected_experts, mixture_weights, latent_routed_aggregate, area,
                         kNoallocBytes, stream);
 }

@@ -108,9 +108,27 @@ def _normal(shape, std: float, g: torch.Generator, dtype: torch.dtype) -> torch.
 
 
 def _stack(n: int, shape, std: float, seed: int, tid: int, dtype: torch.dtype) -> torch.Tensor:
+    """n slices, each from its own generator; slices are drawn on a thread pool
+    (torch releases the GIL), which leaves every value unchanged."""
+    import concurrent.futures as cf
+    import os
+
     out = torch.empty((n,) + tuple(shape), dtype=dtype)
-    for i in range(n):
+
+    def one(i):
         out[i] = _normal(shape, std, _gen(seed, tid, i), dtype)
+
+    def worker(i):
+        torch.set_num_threads(1)      # in the worker thread: no nested intra-op pools
+        one(i)
+
+    workers = min(n, len(os.sched_getaffinity(0)), 32)
+    if workers <= 1 or n * math.prod(shape) < (1 << 22):
+        for i in range(n):
+            one(i)
+        return out
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(worker, range(n)))
     return out
 
 

@@ -36,7 +36,10 @@ def _layer(w, gemm=0, act=0):
     return lm.LatentMoE(lm.config_for(w, gemm=gemm, act=act), {k: v.cuda() for k, v in W.items()})
 
 
-def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0):
+def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0, expert_tails=False):
+    """Whole batch on the GPU; oracle on every row, or on n_rows seeded rows
+    (always with the last row, and with expert_tails also every token that
+    holds an expert's last slot row, where a tile's ragged edge falls)."""
     lm = _lm()
     T = w.T if T is None else T
     W = _weights(w)
@@ -50,6 +53,11 @@ def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0):
         rng = np.random.default_rng(1234 + seed)
         rows = np.sort(rng.choice(T, size=n_rows, replace=False))
         rows[-1] = T - 1   # always include the ragged tail
+        if expert_tails:
+            offsets = layer.region(T, "offsets", torch.int32, (w.E + 1,)).cpu().numpy().astype(np.int64)
+            perm = layer.region(T, "perm_tok", torch.int32, (T * w.k,)).cpu().numpy()
+            last = offsets[1:][offsets[1:] > offsets[:-1]] - 1      # each non-empty expert's last slot row
+            rows = np.concatenate([rows, perm[last]])
         rows = np.unique(rows)
     # a standard workload carries identity projections: with no norm, the
     # oracle's layer formula is then the standard MoE
@@ -367,20 +375,33 @@ def test_zero_tokens_is_a_noop_and_errors_are_reported():
     layer.close()
 
 
-# ---------------------------------------------------------------- full-size workloads, sampled rows
-@pytest.mark.parametrize("name,n_rows", [("acc_d2048", 64), ("eff_zipf_d2048", 64), ("std_d2048", 48)])
-def test_full_size_sampled_rows(name, n_rows):
-    errs, _ = run_parity(li.WORKLOADS[name], n_rows=n_rows)
+# ---------------------------------------------------------------- full-size workloads
+@pytest.mark.parametrize("name", ["acc_d2048", "eff_zipf_d2048"])
+def test_full_size_every_row(name):
+    """The whole batch in the benchmark's launch configuration, every row
+    against the oracle."""
+    errs, _ = run_parity(li.WORKLOADS[name])
+    assert errs["rows_compared"] == li.WORKLOADS[name].T
     print(name, errs)
+
+
+def test_standard_full_size_sampled_rows():
+    errs, _ = run_parity(li.WORKLOADS["std_d2048"], n_rows=256, expert_tails=True)
+    print("std_d2048", errs)
 
 
 @pytest.mark.parametrize("T", [1, 8, 32, 128])
 def test_decode_sweep(T):
+    """Every row of each decode batch."""
     w = li.WORKLOADS["decode_d7168"]
-    errs, _ = run_parity(w, T=T, n_rows=min(T, 16))
+    errs, _ = run_parity(w, T=T)
+    assert errs["rows_compared"] == T
     print("decode", T, errs)
 
 
 def test_large_sampled_rows():
-    errs, _ = run_parity(li.WORKLOADS["large_d4096"], n_rows=24)
+    """512 seeded rows plus every token holding an expert's last slot row (the
+    grouped GEMMs' ragged tile edges): about a thousand rows of 32768."""
+    errs, _ = run_parity(li.WORKLOADS["large_d4096"], n_rows=512, expert_tails=True)
+    assert errs["rows_compared"] >= 512
     print("large", errs)

@@ -59,3 +59,23 @@ def test_single_process_needs_no_group():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(3.5, "cpu") == 3.5
+
+
+def test_bench_gpus_flag_starts_the_ranks_itself():
+    """`bench.py --gpus 2` run as a plain script (no WORLD_SIZE) starts two
+    ranks through torch.distributed.run; with --launch-check each rank times a
+    trivial CPU step over gloo, and rank 0's line reports both ranks, the max
+    over ranks (rank 1 adds 5 ms) and the whole-job aggregate."""
+    import json
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--launch-check",
+                        "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(s) for s in r.stdout.splitlines() if s.startswith("{")]
+    assert len(lines) == 1, r.stdout                 # rank 0 alone prints
+    line = lines[0]
+    assert line["launch_check"] and line["n_gpus"] == 2
+    assert line["job_ms"] >= line["rank_ms"]                  # the max over ranks
+    assert line["value"] == pytest.approx(2 * 1024 / (line["job_ms"] / 3 / 1e3))
