@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "LMOE_OK", 1: "LMOE_ERR_INVALID_ARG", 2: "LMOE_ERR_UNSUPPORTE
 
 # lmoe_workspace_region ids
 REGION = {"scores": 0, "p32": 1, "counts": 2, "offsets": 3, "slot_of": 4, "perm_tok": 5, "Z": 6, "H": 7,
-          "Y": 8, "HS": 9, "status": 10, "cutoff": 11}
+          "Y": 8, "HS": 9, "status": 10, "cutoff": 11, "Zp": 12}
 
 EXPORTS = ("lmoe_config_from_base", "lmoe_create", "lmoe_workspace_size", "lmoe_forward", "lmoe_host_workspace_size",
            "lmoe_forward_host", "lmoe_forward_noalloc", "lmoe_debug_inject", "lmoe_set_bias", "lmoe_qb_histogram", "lmoe_qb_bias_update", "lmoe_set_stage_events", "lmoe_launch_count", "lmoe_workspace_region", "lmoe_check_device", "lmoe_check_device_host",

@@ -46,6 +46,7 @@
 #include <cudaTypedefs.h>
 
 #include "gemm_tc.cuh"
+#include "topk.cuh"
 
 namespace lmoe {
 namespace {
@@ -55,11 +56,19 @@ constexpr int THREADS = 320;   // 2 role warps + 8 epilogue warps
 constexpr int TMEM_COLS = 2 * BN;
 constexpr long long WAIT_LIMIT_CYCLES = 4000000000ll;   // about 2 s at 2 GHz
 constexpr int MAX_E = 1024;
-template <int CG> struct Tiles {
+// NH: 256-column halves per output tile.  NH = 1: (128 CG) x 256 tiles in two
+// double-buffered 256-column accumulators.  NH = 2 (CTA pairs): 256 x 512
+// tiles in one 512-column accumulator of two halves, each filled by its own
+// M = 256, N = 256 MMAs from the same A stage, so every operand byte a CTA
+// moves feeds a third more MMA work (48 KB per k-step for 128 x 512 outputs
+// instead of 32 KB for 128 x 256).
+template <int CG, int NH = 1> struct Tiles {
     static constexpr int A_BYTES = 128 * BK * 2;                // this CTA's 128 A rows
-    static constexpr int B_BYTES = (BN / CG) * BK * 2;          // this CTA's share of B rows
+    static constexpr int B_HALF_BYTES = (BN / CG) * BK * 2;     // this CTA's share of one half's B rows
+    static constexpr int B_BYTES = NH * B_HALF_BYTES;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TILE_M = 128 * CG;
+    static constexpr int TILE_N = BN * NH;
     // kind::f16, D fp32, A and B bf16, both K-major, M = 128 CG, N = BN
     static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                       ((uint32_t)(TILE_M >> 4) << 24);
@@ -70,14 +79,14 @@ template <int CG> struct Tiles {
 // stored by TMA), and as many operand stages as fit (at most 6): the weight
 // tiles of a grouped GEMM mostly come from HBM, and the ring is what keeps
 // their loads in flight.
-template <int CG, int OB> struct Cfg : Tiles<CG> {
+template <int CG, int OB, int NH = 1> struct Cfg : Tiles<CG, NH> {
     static constexpr int EPI_CHUNK = 32 * 32 * OB;
     static constexpr int EPI_STAGING = 8 * EPI_CHUNK;
     static constexpr int TABLES = 2 * (int)sizeof(int) * (MAX_E + 1);
     static constexpr int FIXED = 1024 + EPI_STAGING + 256 + TABLES;
-    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG>::STAGE_BYTES;
+    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG, NH>::STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG>::STAGE_BYTES;
+    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG, NH>::STAGE_BYTES;
     static_assert(STAGES >= 3, "operand ring too shallow");
 };
 
@@ -367,12 +376,12 @@ struct Tile {
 
 // Grouped mode reads the expert row offsets and m-tile prefix from shared
 // memory (staged once per CTA), so decoding a tile costs no global round trip.
-template <int CG>
+template <int CG, int NH>
 __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off, const int *s_offsets, int tile)
 {
     Tile t;
     const int mt = tile / p.ntn, nt = tile % p.ntn;
-    t.n0 = nt * BN;
+    t.n0 = nt * BN * NH;
     if (p.offsets) {
         int lo = 0, hi = p.E - 1;  // last e with tile_off[e] <= mt
         while (lo < hi) {
@@ -390,12 +399,12 @@ __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off,
     return t;
 }
 
-template <int MODE, typename TO, int CG>
+template <int MODE, typename TO, int CG, int NH>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const TcParams p)
 {
-    using C = Cfg<CG, (int)sizeof(TO)>;
+    using C = Cfg<CG, (int)sizeof(TO), NH>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -436,12 +445,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
     }
-    if (p.offsets) {
-        for (int i = threadIdx.x; i <= p.E; i += THREADS) {
-            s_tile_off[i] = p.tile_off[i];
-            s_offsets[i] = p.offsets[i];
-        }
-    }
     if (warp == 1) {
         if (CG == 2) {
             asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -451,6 +454,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                          ::"r"(smem_u32(tmem_holder)), "r"(TMEM_COLS) : "memory");
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
+    }
+    // the prologue above overlaps the previous kernel's tail; from here on this
+    // kernel reads its inputs (A rows, expert tables) and writes its outputs
+    griddep_wait();
+    griddep_launch_dependents();
+    if (p.offsets) {
+        for (int i = threadIdx.x; i <= p.E; i += THREADS) {
+            s_tile_off[i] = p.tile_off[i];
+            s_offsets[i] = p.offsets[i];
         }
     }
     tc_fence_before();
@@ -468,7 +481,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             int it = 0;
             bool ok = true;
             for (int item = group; item < total && ok; item += ngroups) {
-                const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
+                const Tile t = decode<CG, NH>(p, s_tile_off, s_offsets, item / p.ksplit);
+                const int nh = (NH == 2 && p.N - t.n0 > BN) ? 2 : 1;   // halves with columns in this tile
                 const int split = item % p.ksplit;
                 const int kb_end = (split + 1) * nkb_total / p.ksplit;
                 for (int kb = split * nkb_total / p.ksplit; kb < kb_end; ++kb, ++it) {
@@ -483,10 +497,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
                     const uint32_t fb = CG == 2 ? map_to_rank(full_bar(s), 0) : full_bar(s);
-                    if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
+                    if (leader) mbar_expect_tx(full_bar(s), CG * (C::A_BYTES + nh * C::B_HALF_BYTES));
                     tma_load_2d<CG>(sa, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
-                    tma_load_2d<CG>(sa + C::A_BYTES, &tmB, fb, kk,
-                                    (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
+                    for (int h = 0; h < nh; ++h)
+                        tma_load_2d<CG>(sa + C::A_BYTES + h * C::B_HALF_BYTES, &tmB, fb, kk,
+                                        (int)(t.brow + h * BN + (BN / CG) * rank + term * p.term_rows));
                     drain_counts[0] = it + 1;
                 }
             }
@@ -495,10 +510,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (lane == 0 && leader) {
             // ---------------------------------------------------- MMA issuer (leader CTA)
             int it = 0, local = 0;
+            int uses[2] = {0, 0};       // NH = 2: tiles that have used each half so far
             bool ok = true;
             for (int item = group; item < total && ok; item += ngroups, ++local) {
-                const int acc = local & 1;
-                const uint32_t aph = (uint32_t)(local >> 1) & 1u;
+                // NH = 1: this tile's accumulator alternates; NH = 2: halves 0 and 1
+                const int acc = NH == 1 ? (local & 1) : 0;
+                const uint32_t aph = NH == 1 ? ((uint32_t)(local >> 1) & 1u) : ((uint32_t)uses[0] & 1u);
+                int nh = 1;
+                if (NH == 2) {
+                    const Tile t = decode<CG, NH>(p, s_tile_off, s_offsets, item / p.ksplit);
+                    nh = p.N - t.n0 > BN ? 2 : 1;
+                }
                 const int split = item % p.ksplit;
                 const int kb_begin = split * nkb_total / p.ksplit, kb_end = (split + 1) * nkb_total / p.ksplit;
                 if (!mbar_wait(acce_bar(acc), aph ^ 1u)) {
@@ -525,16 +547,40 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                     tc_fence_after();
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
+                    for (int h = 0; h < nh; ++h) {
+                        // NH = 2: the first k-step's MMAs into half 1 wait until the
+                        // epilogue has read the previous tile's half 1 (half 0's
+                        // MMAs already run meanwhile)
+                        if (NH == 2 && h == 1 && kb == kb_begin) {
+                            if (!mbar_wait(acce_bar(1), ((uint32_t)uses[1] & 1u) ^ 1u)) {
+                                atomicOr(p.status, ST_MMA);
+                                *(volatile int *)abort_flag = 1;
+                                ok = false;
+                                break;        // half 0's MMAs of this stage are committed below
+                            }
+                            tc_fence_after();
+                        }
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = sdesc_sw128(sa + 32u * k);
-                        const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + 32u * k);
-                        umma_bf16<CG>(dt, ad, bd, (kb > kb_begin || k > 0) ? 1u : 0u);
+                        for (int k = 0; k < BK / 16; ++k) {
+                            const uint64_t ad = sdesc_sw128(sa + 32u * k);
+                            const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + h * C::B_HALF_BYTES + 32u * k);
+                            umma_bf16<CG>(dt + (uint32_t)(h * BN), ad, bd, (kb > kb_begin || k > 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit<CG>(empty_bar(s));
                     drain_counts[1] = it + 1;
+                    if (!ok) break;
                 }
-                if (ok) umma_commit<CG>(accf_bar(acc));
+                if (ok) {
+                    if (NH == 2) {
+                        for (int h = 0; h < nh; ++h) {
+                            umma_commit<CG>(accf_bar(h));
+                            ++uses[h];
+                        }
+                    } else {
+                        umma_commit<CG>(accf_bar(acc));
+                    }
+                }
             }
         }
     } else {
@@ -545,24 +591,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
         const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * C::EPI_CHUNK;
         int local = 0;
-        for (int item = group; item < total; item += ngroups, ++local) {
-            const int acc = local & 1;
-            const uint32_t aph = (uint32_t)(local >> 1) & 1u;
-            const bool got = mbar_wait(accf_bar(acc), aph);
-            if (!got || *(volatile int *)abort_flag) {
-                if (lane == 0) {
-                    atomicOr(p.status, ST_EPILOGUE);
-                    *(volatile int *)abort_flag = 1;
-                }
-                break;
-            }
-            tc_fence_after();
-            const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
+        int uses[2] = {0, 0};           // NH = 2: tiles that have used each half so far
+        bool stop = false;
+        for (int item = group; item < total && !stop; item += ngroups, ++local) {
+            const Tile t = decode<CG, NH>(p, s_tile_off, s_offsets, item / p.ksplit);
+            const int nh = (NH == 2 && p.N - t.n0 > BN) ? 2 : 1;
             const int64_t slab = (int64_t)(item % p.ksplit) * p.split_rows;   // 0 unless split K
             const int64_t row = t.row0 + 128 * rank + 32 * q + lane;
             const bool valid = row < t.row_end;
-            const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
-            float v[32], u[32];
             // Emit 32 output columns [col, col + n) of this warp's 32 rows: whole
             // chunks go through the staging buffer and one TMA store; chunks that
             // straddle an expert's last row (or a ragged column edge) store per lane.
@@ -582,65 +618,116 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     store_n((TO *)p.epi.out + (slab + row) * p.epi.ldo + col, x, n);
                 }
             };
-            if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
-                const int half = BN / 2;
-#pragma unroll 1
-                for (int c = 32 * hset; c < half; c += 64) {
-                    __syncwarp();
-                    tmem_ld32_pair(tq + c, tq + half + c, v, u);   // gate and up columns, one wait
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
-                                                                                       p.epi.up_cap);
-                    emit(v, t.n0 / 2 + c, 32);
+            // one 256-column accumulator at a time: NH = 1 the tile's (alternating
+            // between two), NH = 2 each half of the tile in turn
+            for (int hu = 0; hu < nh; ++hu) {
+                const int acc = NH == 1 ? (local & 1) : hu;
+                const uint32_t aph = NH == 1 ? ((uint32_t)(local >> 1) & 1u) : ((uint32_t)uses[hu] & 1u);
+                const bool got = mbar_wait(accf_bar(acc), aph);
+                if (!got || *(volatile int *)abort_flag) {
+                    if (lane == 0) {
+                        atomicOr(p.status, ST_EPILOGUE);
+                        *(volatile int *)abort_flag = 1;
+                    }
+                    stop = true;
+                    break;
                 }
-            } else {
+                tc_fence_after();
+                const int n0 = t.n0 + (NH == 2 ? hu * BN : 0);      // first GEMM column of this accumulator
+                const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
+                float v[32], u[32];
+                if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
+                    const int half = BN / 2;
 #pragma unroll 1
-                for (int c = 32 * hset; c < BN; c += 128) {
-                    __syncwarp();
-                    tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // warp-collective: every lane
+                    for (int c = 32 * hset; c < half; c += 64) {
+                        __syncwarp();
+                        tmem_ld32_pair(tq + c, tq + half + c, v, u);   // gate and up columns, one wait
 #pragma unroll
-                    for (int part = 0; part < 2; ++part) {
-                        float *x = part ? u : v;
-                        const int col = t.n0 + c + 64 * part;
-                        int n = p.N - col;
-                        if (n > 32) n = 32;
-                        if (n <= 0) continue;             // uniform across the warp
-                        if (MODE == EPI_SIGMOID) {
+                        for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
+                                                                                           p.epi.up_cap);
+                        emit(v, n0 / 2 + c, 32);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int c = 32 * hset; c < BN; c += 128) {
+                        __syncwarp();
+                        tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // warp-collective: every lane
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
-                        } else if (MODE == EPI_STORE && sizeof(TO) == 2) {
-                            if (p.epi.residual && valid) {   // standard MoE: y = shared + u
-                                const bf16 *res = (const bf16 *)p.epi.residual + (slab + row) * p.epi.ldr + col;
-                                if (n == 32 && ((uintptr_t)res & 15u) == 0) {
+                        for (int part = 0; part < 2; ++part) {
+                            float *x = part ? u : v;
+                            const int col = n0 + c + 64 * part;
+                            int n = p.N - col;
+                            if (n > 32) n = 32;
+                            if (n <= 0) continue;             // uniform across the warp
+                            if (MODE == EPI_SIGMOID) {
 #pragma unroll
-                                    for (int q8 = 0; q8 < 4; ++q8) {   // four 16-byte loads
-                                        const uint4 w = *reinterpret_cast<const uint4 *>(res + 8 * q8);
-                                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                                for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
+                            } else if (MODE == EPI_STORE && sizeof(TO) == 2) {
+                                if (p.epi.residual && valid) {   // standard MoE: y = shared + u
+                                    const bf16 *res = (const bf16 *)p.epi.residual + (slab + row) * p.epi.ldr + col;
+                                    if (n == 32 && ((uintptr_t)res & 15u) == 0) {
 #pragma unroll
-                                        for (int i = 0; i < 4; ++i) {
-                                            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&ws[i]);
-                                            x[8 * q8 + 2 * i] += __low2float(h2);
-                                            x[8 * q8 + 2 * i + 1] += __high2float(h2);
+                                        for (int q8 = 0; q8 < 4; ++q8) {   // four 16-byte loads
+                                            const uint4 w = *reinterpret_cast<const uint4 *>(res + 8 * q8);
+                                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                                            for (int i = 0; i < 4; ++i) {
+                                                const __nv_bfloat162 h2 =
+                                                    *reinterpret_cast<const __nv_bfloat162 *>(&ws[i]);
+                                                x[8 * q8 + 2 * i] += __low2float(h2);
+                                                x[8 * q8 + 2 * i + 1] += __high2float(h2);
+                                            }
                                         }
+                                    } else {
+#pragma unroll
+                                        for (int i = 0; i < 32; ++i)
+                                            if (i < n) x[i] += __bfloat162float(res[i]);
                                     }
-                                } else {
-#pragma unroll
-                                    for (int i = 0; i < 32; ++i)
-                                        if (i < n) x[i] += __bfloat162float(res[i]);
                                 }
-                            }
-                        } else if (MODE == EPI_COMBINE) {
-                            const float w = valid ? p.epi.row_w[row] : 0.f;   // bf16 rows: p-weighted here
+                            } else if (MODE == EPI_COMBINE) {
+                                const float w = valid ? p.epi.row_w[row] : 0.f;   // bf16 rows: p-weighted here
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) x[i] *= w;
+                                for (int i = 0; i < 32; ++i) x[i] *= w;
+                            }
+                            if (MODE == EPI_SCATTER) {
+                                // the token's latent row goes straight to its k slot rows
+                                if (valid) {
+                                    const int32_t *so = p.epi.slot_of + row * p.epi.kslots;
+                                    if (n == 32) {
+                                        uint4 w4[4];
+#pragma unroll
+                                        for (int q4 = 0; q4 < 4; ++q4) {
+                                            uint32_t w[4];
+#pragma unroll
+                                            for (int i = 0; i < 4; ++i) {
+                                                const __nv_bfloat162 pr =
+                                                    __floats2bfloat162_rn(x[q4 * 8 + 2 * i], x[q4 * 8 + 2 * i + 1]);
+                                                w[i] = *reinterpret_cast<const uint32_t *>(&pr);
+                                            }
+                                            w4[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+                                        }
+                                        for (int j = 0; j < p.epi.kslots; ++j) {
+                                            uint4 *d4 = reinterpret_cast<uint4 *>((bf16 *)p.epi.out +
+                                                                                 (int64_t)so[j] * p.epi.ldo + col);
+#pragma unroll
+                                            for (int q4 = 0; q4 < 4; ++q4) d4[q4] = w4[q4];
+                                        }
+                                    } else {
+                                        for (int j = 0; j < p.epi.kslots; ++j)
+                                            store_n((bf16 *)p.epi.out + (int64_t)so[j] * p.epi.ldo + col, x, n);
+                                    }
+                                }
+                            } else {
+                                emit(x, col, n);
+                            }
                         }
-                        emit(x, col, n);
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(CG == 2 ? map_to_rank(acce_bar(acc), 0) : acce_bar(acc));
+                if (NH == 2) ++uses[hu];
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(CG == 2 ? map_to_rank(acce_bar(acc), 0) : acce_bar(acc));
         }
         if (lane == 0) bulk_wait_all();             // this warp's TMA stores are complete
     }
@@ -708,7 +795,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
 // CTA pairs, how many pairs fit at once), done on first use and cached.
 constexpr int MAX_DEVICES = 64;
 
-template <int MODE, typename TO, int CG>
+template <int MODE, typename TO, int CG, int NH>
 cudaError_t group_capacity(int *max_groups)
 {
     static std::atomic<int> cached[MAX_DEVICES];   // 0 = not yet known
@@ -719,15 +806,15 @@ cudaError_t group_capacity(int *max_groups)
         *max_groups = cached[dev];
         return cudaSuccess;
     }
-    auto kern = tc_gemm_kernel<MODE, TO, CG>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG, (int)sizeof(TO)>::SMEM);
+    auto kern = tc_gemm_kernel<MODE, TO, CG, NH>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG, (int)sizeof(TO), NH>::SMEM);
     if (e != cudaSuccess) return e;
     int groups = g_num_sms / CG;
     if (CG > 1) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(g_num_sms / CG * CG);
         q.blockDim = dim3(THREADS);
-        q.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO)>::SMEM;
+        q.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO), NH>::SMEM;
         cudaLaunchAttribute qa[1];
         qa[0].id = cudaLaunchAttributeClusterDimension;
         qa[0].val.clusterDim.x = CG;
@@ -745,34 +832,37 @@ cudaError_t group_capacity(int *max_groups)
 }
 
 // Persistent grid: min(work items, CTA groups that can be resident at once).
-template <int MODE, typename TO, int CG>
+template <int MODE, typename TO, int CG, int NH>
 cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const TcParams &p, cudaStream_t s)
 {
-    auto kern = tc_gemm_kernel<MODE, TO, CG>;
+    auto kern = tc_gemm_kernel<MODE, TO, CG, NH>;
     int max_groups = 0;
-    const cudaError_t e = group_capacity<MODE, TO, CG>(&max_groups);
+    const cudaError_t e = group_capacity<MODE, TO, CG, NH>(&max_groups);
     if (e != cudaSuccess) return e;
     const int items = p.max_tiles * p.ksplit;
     const int groups = items < max_groups ? items : max_groups;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(groups * CG);
     lc.blockDim = dim3(THREADS);
-    lc.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO)>::SMEM;
+    lc.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO), NH>::SMEM;
     lc.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CG;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
-    lc.numAttrs = 1;
+    lc.numAttrs = 2;
     return cudaLaunchKernelEx(&lc, kern, a, b, c, p);
 }
 
-template <int CG>
+template <int CG, int NH>
 cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t term_rows, int64_t b_rows_total,
                 int ksplit, int32_t *status, cudaStream_t s)
 {
+    static_assert(NH == 1 || CG == 2, "512-column tiles are for CTA pairs");
     if (!g_encode) return cudaErrorInitializationError;
     if (g.K % BK) return cudaErrorInvalidValue;
     if (((uintptr_t)g.A | (uintptr_t)g.B) & 15u) return cudaErrorMisalignedAddress;
@@ -784,17 +874,21 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.nkb = g.K / BK;
     p.nterms = nterms;
     p.term_rows = term_rows;
-    p.ntn = (mode == EPI_GLU) ? g.N / BN : (g.N + BN - 1) / BN;   // GLU: N = 2F, F % (BN/2) == 0
+    // GLU: N = 2F, F % (BN/2) == 0, so every 256-column half holds whole gate/up pairs
+    p.ntn = (g.N + BN * NH - 1) / (BN * NH);
     p.group_rows = g.offsets ? g.b_group_stride / g.ldb : 0;
     p.offsets = g.offsets;
     p.tile_off = g.tile_off;
     p.E = g.E;
-    const int mtiles = g.offsets ? max_mtiles : (g.M + Tiles<CG>::TILE_M - 1) / Tiles<CG>::TILE_M;
+    const int mtiles = g.offsets ? max_mtiles : (g.M + Tiles<CG, NH>::TILE_M - 1) / Tiles<CG, NH>::TILE_M;
     p.max_tiles = mtiles * p.ntn;
     p.ksplit = ksplit < 1 ? 1 : ksplit;
     p.split_rows = g.M;
     if (p.ksplit > 1 && (g.offsets || (mode != EPI_STORE_F32 && mode != EPI_SIGMOID_PARTIAL) ||
                          p.ksplit > p.nkb * nterms))
+        return cudaErrorInvalidValue;
+    if (NH == 2 && (p.ksplit > 1 || nterms > 1 || mode == EPI_SIGMOID || mode == EPI_STORE_F32 ||
+                    mode == EPI_SIGMOID_PARTIAL))
         return cudaErrorInvalidValue;
     p.epi = g.epi;
     p.status = status;
@@ -811,18 +905,344 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     memset(&tc, 0, sizeof tc);
     p.tma_store = make_out_map(&tc, g.epi.out, out_f32, (uint64_t)p.out_cols, (uint64_t)g.M * p.ksplit,
                                (uint64_t)g.epi.ldo * (out_f32 ? 4 : 2)) ? 1 : 0;
+    if (NH == 2) {
+        switch (mode) {
+        case EPI_GLU:
+            if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG, NH>(ta, tb, tc, p, s);
+            return launch<EPI_GLU, bf16, CG, NH>(ta, tb, tc, p, s);
+        case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG, NH>(ta, tb, tc, p, s);
+        case EPI_STORE: return launch<EPI_STORE, bf16, CG, NH>(ta, tb, tc, p, s);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     switch (mode) {
-    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG>(ta, tb, tc, p, s);
+    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG, 1>(ta, tb, tc, p, s);
     case EPI_GLU:
-        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG>(ta, tb, tc, p, s);
-        return launch<EPI_GLU, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_STORE_F32: return launch<EPI_STORE, float, CG>(ta, tb, tc, p, s);
+        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG, 1>(ta, tb, tc, p, s);
+        return launch<EPI_GLU, bf16, CG, 1>(ta, tb, tc, p, s);
+    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG, 1>(ta, tb, tc, p, s);
+    case EPI_STORE: return launch<EPI_STORE, bf16, CG, 1>(ta, tb, tc, p, s);
+    case EPI_SCATTER: return launch<EPI_SCATTER, bf16, CG, 1>(ta, tb, tc, p, s);
+    case EPI_STORE_F32: return launch<EPI_STORE, float, CG, 1>(ta, tb, tc, p, s);
     default: return cudaErrorInvalidValue;
     }
 }
 
+
+// ------------------------------------------------------------------ router + top-k
+// Router scores, biased top-k and renormalisation in one launch ("Stable
+// LatentMoE", equations for r, T_k(x) and p_i), for E <= 512 experts.
+//
+// A cluster of KS CTAs takes one 128-token tile: CTA `rank` runs the k-blocks
+// [rank, rank + 1) * NKB / KS of the three bf16 terms of the fp32 router
+// weight (hi + mid + lo; with bf16 tokens every product is exact in fp32)
+// through tcgen05.mma into one fp32 TMEM accumulator of E columns (two
+// 256-column halves for E = 512).  Its eight epilogue warps write the partial
+// logits to L2 (KS > 1; in rank slabs) or, for KS = 1, r = sigmoid(logit)
+// directly.  After a cluster barrier each CTA owns 128 / KS tokens of the
+// tile: one warp per token sums the KS partial logits in rank order (fixed
+// order, deterministic), applies the sigmoid and writes r, runs the warp
+// tournament on r + b (warp_topk: equal scores to the lower index), and writes
+// the selection, p from the raw scores, the Quantile-Balancing cutoff and the
+// per-32-token expert counts that the counting sort scans.
+struct RtParams {
+    int T, E, k;
+    int nkb;                 // k-blocks of 64 per term (d / 64)
+    int ks;                  // CTAs per cluster (split of the 3 nkb k-blocks)
+    int halves, n_half;      // MMA column halves (1 or 2) and columns per half
+    uint32_t idesc;          // kind::f16, M = 128, N = n_half
+    int stages, stage_bytes, tmem_cols;
+    const float *bias;
+    float *partial;          // [ks][T][E] partial logits (ks > 1)
+    float *r;                // [T][E]
+    int32_t *sel;
+    float *p32;
+    void *p_out;
+    float *cutoff;
+    int32_t *blockhist;
+    int nb;
+    int stall_test;
+    int32_t *status;
+};
+
+template <typename TO, int EPL>
+__global__ void __launch_bounds__(THREADS, 1)
+router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const RtParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t *gbase = smem_raw + (sbase - raw);
+    const int STAGES = p.stages;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(gbase + (size_t)STAGES * p.stage_bytes);
+    // bars[0..S) full, [S..2S) empty, [2S] accumulator full
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 1);
+    int *abort_flag = reinterpret_cast<int *>(tmem_holder + 1);
+    int *drain_counts = abort_flag + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)(blockIdx.x % p.ks);
+    const int64_t row0 = (int64_t)(blockIdx.x / p.ks) * 128;
+    const int nkb_total = 3 * p.nkb;
+    const int kb_begin = rank * nkb_total / p.ks, kb_end = (rank + 1) * nkb_total / p.ks;
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    const uint32_t accf = bar0 + 8u * (2 * STAGES);
+    const int a_bytes = 128 * BK * 2, bh_bytes = p.n_half * BK * 2;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(accf, 1);
+        *abort_flag = 0;
+        drain_counts[0] = drain_counts[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_holder)), "r"(p.tmem_cols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    griddep_wait();
+    griddep_launch_dependents();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {   // ------------------------------------------------ TMA producer
+            int it = 0;
+            for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
+                    atomicOr(p.status, ST_PRODUCER);
+                    *(volatile int *)abort_flag = 1;
+                    break;
+                }
+                const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
+                const uint32_t sa = sbase + (uint32_t)s * p.stage_bytes;
+                mbar_expect_tx(full_bar(s), a_bytes + p.halves * bh_bytes);
+                tma_load_2d<1>(sa, &tmA, full_bar(s), kk, (int)row0);
+                for (int h = 0; h < p.halves; ++h)
+                    tma_load_2d<1>(sa + a_bytes + h * bh_bytes, &tmB, full_bar(s), kk,
+                                   term * p.E + h * p.n_half);
+                drain_counts[0] = it + 1;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {   // ------------------------------------------------ MMA issuer
+            int it = 0;
+            bool ok = true;
+            if (p.stall_test && !mbar_wait(accf, 0u)) {
+                // only this thread commits that barrier: the wait runs out by design
+                atomicOr(p.status, ST_MMA);
+                *(volatile int *)abort_flag = 1;
+                ok = false;
+            }
+            for (int kb = kb_begin; kb < kb_end && ok; ++kb, ++it) {
+                const int s = it % STAGES;
+                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                if (!mbar_wait(full_bar(s), ph) || *(volatile int *)abort_flag) {
+                    atomicOr(p.status, ST_MMA);
+                    *(volatile int *)abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = sbase + (uint32_t)s * p.stage_bytes;
+                for (int h = 0; h < p.halves; ++h) {
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = sdesc_sw128(sa + 32u * k);
+                        const uint64_t bd = sdesc_sw128(sa + a_bytes + h * bh_bytes + 32u * k);
+                        const uint32_t acc = (kb > kb_begin || k > 0) ? 1u : 0u;
+                        asm volatile(
+                            "{\n\t.reg .pred q;\n\t"
+                            "setp.ne.b32 q, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n\t}"
+                            ::"r"(tmem_base + (uint32_t)(h * 256)), "l"(ad), "l"(bd), "r"(p.idesc), "r"(acc));
+                    }
+                }
+                umma_commit<1>(empty_bar(s));
+                drain_counts[1] = it + 1;
+            }
+            if (ok) umma_commit<1>(accf);
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue warps 2..9
+        const int q = warp & 3, hset = (warp - 2) >> 2;
+        const bool got = mbar_wait(accf, 0u);
+        if (!got || *(volatile int *)abort_flag) {
+            if (lane == 0) {
+                atomicOr(p.status, ST_EPILOGUE);
+                *(volatile int *)abort_flag = 1;
+            }
+        } else {
+            tc_fence_after();
+            const int64_t row = row0 + 32 * q + lane;
+            const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
+            float *dst = p.ks > 1 ? p.partial + ((int64_t)rank * p.T + row) * p.E : p.r + row * p.E;
+            for (int c = 32 * hset; c < p.E; c += 64) {
+                uint32_t v[32];
+                asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                             "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                             "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                               "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+                               "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+                               "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+                               "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+                               "=r"(v[31])
+                             : "r"(tq + (uint32_t)c));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (row < p.T) {
+                    float f[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        f[i] = __uint_as_float(v[i]);
+                        if (p.ks == 1) f[i] = sigmoidf_(f[i]);
+                    }
+                    store32(dst + c, f);
+                }
+            }
+        }
+    }
+    // every CTA of the cluster passes exactly these barriers, whatever happened above
+    __syncwarp();
+    __threadfence();
+    tc_fence_before();
+    __syncthreads();
+    if (p.ks > 1) cluster_sync();     // every rank's partial logits are written and visible
+
+    // ---------------------------------------------------------------- top-k, one warp per token
+    if (!*(volatile int *)abort_flag) {
+        const int own = 128 / p.ks;
+        const int64_t t0 = row0 + (int64_t)rank * own;
+        for (int i = warp; i < own; i += THREADS / 32) {
+            const int64_t t = t0 + i;
+            if (t >= p.T) break;
+            float v[EPL];
+            int ix[EPL];
+#pragma unroll
+            for (int j = 0; j < EPL; ++j) {
+                const int e = lane + 32 * j;
+                ix[j] = e;
+                float r = 0.f;
+                if (e < p.E) {
+                    if (p.ks == 1) {
+                        r = p.r[t * p.E + e];
+                    } else {
+                        float a = 0.f;
+                        for (int qq = 0; qq < p.ks; ++qq) a += __ldcg(p.partial + ((int64_t)qq * p.T + t) * p.E + e);
+                        r = sigmoidf_(a);
+                        p.r[t * p.E + e] = r;
+                    }
+                }
+                v[j] = e < p.E ? biased_key(r, p.bias[e]) : -INFINITY;
+            }
+            int mine0, mine1;
+            float cv;
+            warp_topk<EPL>(v, ix, p.k, p.E, lane, &mine0, &mine1, &cv);
+            if (lane == 0) p.cutoff[t] = cv;
+            __syncwarp();                 // this token's r, written by every lane, is visible
+            const float r0 = lane < p.k ? p.r[t * p.E + mine0] : 0.f;
+            const float r1 = lane + 32 < p.k ? p.r[t * p.E + mine1] : 0.f;
+            float sum = r0 + r1;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            const int64_t tb = t / ROUTE_TPB;   // per-block counts, expert-major
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int j = lane + 32 * h;
+                if (j < p.k) {
+                    const int e = h ? mine1 : mine0;
+                    const float pv = (h ? r1 : r0) / sum;
+                    p.sel[t * p.k + j] = e;
+                    p.p32[t * p.k + j] = pv;
+                    ((TO *)p.p_out)[t * p.k + j] = from_f32<TO>(pv);
+                    atomicAdd(&p.blockhist[(int64_t)e * p.nb + tb], 1);
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (*(volatile int *)abort_flag && threadIdx.x == 0) {
+        // Drain: loads issued but never consumed, then the MMAs behind the last commit.
+        const int issued = drain_counts[0], consumed = drain_counts[1];
+        bool ok = true;
+        for (int i = consumed; i < issued; ++i)
+            ok &= mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
+        if (consumed > 0) {
+            const int i = consumed - 1;
+            ok &= mbar_wait(empty_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
+        }
+        if (!ok) atomicOr(p.status, ST_DRAIN);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(p.tmem_cols)
+                     : "memory");
+}
+
+constexpr int RT_SMEM_FIXED = 1024 + 256;   // alignment slack, barriers and flags
+
+// Stages and bytes of the router + top-k kernel for E experts.
+void rt_shape(int E, int *halves, int *n_half, int *stages, int *stage_bytes, int *tmem_cols)
+{
+    *halves = E > 256 ? 2 : 1;
+    *n_half = E > 256 ? 256 : E;
+    *stage_bytes = 128 * BK * 2 + *halves * *n_half * BK * 2;
+    int st = (232448 - RT_SMEM_FIXED) / *stage_bytes;
+    *stages = st > 6 ? 6 : st;
+    int cols = 32;
+    while (cols < E) cols *= 2;
+    *tmem_cols = cols;
+}
+
+template <typename TO, int EPL>
+cudaError_t launch_rt(const CUtensorMap &a, const CUtensorMap &b, const RtParams &p, int tiles, cudaStream_t s)
+{
+    auto kern = router_topk_kernel<TO, EPL>;
+    const size_t smem = RT_SMEM_FIXED + (size_t)p.stages * p.stage_bytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)(tiles * p.ks));
+    lc.blockDim = dim3(THREADS);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 2;
+    return cudaLaunchKernelEx(&lc, kern, a, b, p);
+}
+
+template <typename TO>
+cudaError_t launch_rt_epl(const CUtensorMap &a, const CUtensorMap &b, const RtParams &p, int tiles, cudaStream_t s)
+{
+    const int epl = (p.E + 31) / 32;
+    if (epl <= 1) return launch_rt<TO, 1>(a, b, p, tiles, s);
+    if (epl <= 2) return launch_rt<TO, 2>(a, b, p, tiles, s);
+    if (epl <= 4) return launch_rt<TO, 4>(a, b, p, tiles, s);
+    if (epl <= 8) return launch_rt<TO, 8>(a, b, p, tiles, s);
+    return launch_rt<TO, 16>(a, b, p, tiles, s);
+}
 }  // namespace
 
 lmoe_status tc_check_device()
@@ -849,8 +1269,17 @@ cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t
 {
     // B rows: dense N; grouped E * (rows per expert)
     const int64_t b_rows = g.offsets ? (int64_t)g.E * (g.b_group_stride / g.ldb) : g.N;
-    if (cg == 2) return run<2>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
-    return run<1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
+    if (cg == 2 && ksplit <= 1 && mode != EPI_SIGMOID && mode != EPI_STORE_F32 && mode != EPI_SCATTER) {
+        // 256 x 512 tiles where they still make many waves of CTA pairs (a
+        // handful of waves would lose more to the last one's idle pairs than
+        // the wider tile saves)
+        const int64_t mt = g.offsets ? (int64_t)max_mtiles : ((int64_t)g.M + 255) / 256;
+        const int64_t wide_tiles = mt * (((int64_t)g.N + 2 * BN - 1) / (2 * BN));
+        const int pairs = (g_num_sms > 0 ? g_num_sms : 148) / 2;
+        if (wide_tiles >= 6 * (int64_t)pairs) return run<2, 2>(mode, g, max_mtiles, 1, 0, b_rows, 1, status, s);
+    }
+    if (cg == 2) return run<2, 1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
+    return run<1, 1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
 }
 
 int tc_num_sms() { return g_num_sms; }
@@ -863,8 +1292,59 @@ cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int cg, int32_t *
     r.B = Wr3;
     r.ldb = g.K;
     const int mode = ksplit > 1 ? EPI_SIGMOID_PARTIAL : EPI_SIGMOID;
-    if (cg == 2) return run<2>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
-    return run<1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+    if (cg == 2) return run<2, 1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+    return run<1, 1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+}
+
+}  // namespace lmoe
+
+namespace lmoe {
+
+int tc_router_topk_splits(int64_t T, int E, int d)
+{
+    if (T <= 0 || E > 512 || E % 32 || (E > 256 && E != 512) || d % BK) return 0;
+    const int sms = g_num_sms > 0 ? g_num_sms : 148;
+    const int64_t tiles = (T + 127) / 128;
+    const int nkb_total = 3 * (d / BK);
+    int ks = 1;
+    while (ks < 8 && tiles * ks * 2 <= sms && 2 * ks * 2 <= nkb_total) ks *= 2;
+    return ks;
+}
+
+cudaError_t tc_router_topk(const bf16 *x, const bf16 *Wr3, const float *bias, int64_t T, int E, int d, int k,
+                           float *partial, float *r, int32_t *sel, float *p32, void *p_out, int out_bf16,
+                           float *cutoff, int32_t *blockhist, int32_t *status, cudaStream_t s)
+{
+    const int ks = tc_router_topk_splits(T, E, d);
+    if (!ks || k < 1 || k > 64 || k > E) return cudaErrorInvalidValue;
+    if (!g_encode) return cudaErrorInitializationError;
+    if (((uintptr_t)x | (uintptr_t)Wr3) & 15u) return cudaErrorMisalignedAddress;
+    RtParams p = {};
+    p.T = (int)T;
+    p.E = E;
+    p.k = k;
+    p.nkb = d / BK;
+    p.ks = ks;
+    rt_shape(E, &p.halves, &p.n_half, &p.stages, &p.stage_bytes, &p.tmem_cols);
+    p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.n_half >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    p.bias = bias;
+    p.partial = partial;
+    p.r = r;
+    p.sel = sel;
+    p.p32 = p32;
+    p.p_out = p_out;
+    p.cutoff = cutoff;
+    p.blockhist = blockhist;
+    p.nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
+    p.stall_test = g_stall_next.exchange(0);
+    p.status = status;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, x, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&tb, Wr3, (uint64_t)d, (uint64_t)3 * E, (uint64_t)d * 2, (uint32_t)p.n_half))
+        return cudaErrorInvalidValue;
+    const int tiles = (int)((T + 127) / 128);
+    if (out_bf16) return launch_rt_epl<bf16>(ta, tb, p, tiles, s);
+    return launch_rt_epl<float>(ta, tb, p, tiles, s);
 }
 
 }  // namespace lmoe

@@ -37,4 +37,17 @@ void tc_debug_stall_next();
 cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int cg, int32_t *status, cudaStream_t s,
                            int ksplit = 1);
 
+// Router scores, biased top-k and renormalisation in one launch (tensor
+// cores, fp32 router through its three-term bf16 split Wr3 = [3, E, d]) for
+// T tokens of x [T, d]: r [T, E] fp32, sel / p32 / p_out (token dtype) [T, k],
+// the Quantile-Balancing cutoff [T] and the per-32-token expert counts added
+// into blockhist [E][ceil(T / 32)] (zeroed by the caller).  partial holds
+// splits * T * E floats when tc_router_topk_splits() > 1.
+// tc_router_topk_splits: CTAs per 128-token tile (a cluster), or 0 when this
+// path does not apply (E > 512, E not a multiple of 32, 256 < E < 512).
+int tc_router_topk_splits(int64_t T, int E, int d);
+cudaError_t tc_router_topk(const bf16 *x, const bf16 *Wr3, const float *bias, int64_t T, int E, int d, int k,
+                           float *partial, float *r, int32_t *sel, float *p32, void *p_out, int out_bf16,
+                           float *cutoff, int32_t *blockhist, int32_t *status, cudaStream_t s);
+
 }  // namespace lmoe

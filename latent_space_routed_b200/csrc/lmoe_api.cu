@@ -7,8 +7,9 @@
 //   2 top-k            sel, p (fp32 and token dtype), per-block expert counts
 //   3 scan             counts, offsets, per-block bases, m-tile prefix
 //   4 dispatch         slot_of[t, j], token and weight of every slot row
-//   5 down GEMM        z = x W_down^T                           [T, l]
-//   6 permute          Zp[m] = z[token of slot m]               [S, l]
+//   5 down GEMM        z = x W_down^T, written to the token's k slot rows of
+//                      Zp (one tensor-core GEMM), or to z [T, l] (split-K, GEMV)
+//   6 permute          Zp[m] = z[token of slot m] [S, l] (only with z [T, l])
 //   7 gate/up GEMM     per expert: h = act(G z, U z)            [S, f]
 //   8 down GEMM        per expert: Y = p * (h D^T)              [S, l] token dtype
 //   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
@@ -16,6 +17,14 @@
 //  11 final GEMM       y = [h_s | n] [D_s1 | D_s2 | W_up]^T     [T, d]
 // The standard-MoE form (config.standard) skips 5, permutes x, skips the norm
 // in 9 and computes y = h_s [D_s1 | D_s2]^T + u in 11.
+//
+// Tensor-core path: for E <= 512 (a multiple of 32, not between 256 and 512)
+// stages 1 and 2 are one launch (tc_router_topk: router GEMM, sigmoid, top-k,
+// p, cutoff, per-block counts).  Few tokens: up to ROUTE_SMALL_MAX_T tokens,
+// stages 1-4 are one launch (route_small_kernel); up to GEMV_MAX_T tokens the
+// dense GEMMs and the routed experts' GEMMs are weight-streaming GEMVs, the
+// routed ones over the touched experts only, reading z through the slot ->
+// token map (no permute).
 #include <algorithm>
 #include <cmath>
 #include <atomic>
@@ -63,9 +72,14 @@ int64_t hs_cols(const lmoe_config &c) { return 2 * (int64_t)c.f_shared + (c.stan
 
 struct Layout {
     size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, partial,
-        partial_side, cutoff, status;
+        partial_side, cutoff, status, touched;
     size_t total;
 };
+
+// Words of the 256-byte control slot at the start of every workspace.
+constexpr int CTL_STATUS = 0;      // device status word (bounded waits that gave up)
+constexpr int CTL_TICKET = 1;      // route_small_kernel's block ticket (zero at launch)
+constexpr int CTL_NTOUCHED = 2;    // number of touched experts (few-token plan)
 
 }  // namespace
 
@@ -112,8 +126,11 @@ namespace {
 // half the SMs is split along K into as many parts as keep all parts in one
 // wave (fp32 partial tiles, then an ordered reduction that applies the
 // epilogue).
-constexpr int64_t ROUTER_SMALL_MAX_T = 8;
 constexpr int SPLIT_MAX = 16;
+
+// Few-token plans of the tensor-core path.
+bool small_route(const lmoe_handle *h, int64_t T) { return h->tc && T <= ROUTE_SMALL_MAX_T; }
+bool gemv_experts(const lmoe_handle *h, int64_t T) { return h->tc && T <= GEMV_MAX_T; }
 
 // K splits for a dense GEMM of M rows, N columns on (128 cg) x 256 tiles, nkb
 // k-blocks of 64.
@@ -136,6 +153,7 @@ int router_cg(int64_t T) { return T >= 256 ? 2 : 1; }
 
 struct SplitPlan {
     int router, down, shared, final_;
+    bool fused_router;            // router + top-k in one launch (tc_router_topk)
     size_t partial_floats;        // router and final GEMMs: largest ks * T * N
     size_t partial_side_floats;   // down and shared gate/up GEMMs (the side stream's)
 };
@@ -145,8 +163,11 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     const lmoe_config &c = h->cfg;
     const int64_t ld_hs = hs_cols(c);
     SplitPlan sp;
-    sp.router = (h->tc && T > ROUTER_SMALL_MAX_T)
-                    ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true, router_cg(T)) : 1;
+    const int fused_ks = (h->tc && T > ROUTE_SMALL_MAX_T) ? tc_router_topk_splits(T, c.E, c.d) : 0;
+    sp.fused_router = fused_ks > 0;
+    sp.router = sp.fused_router ? fused_ks
+                : (h->tc && T > ROUTE_SMALL_MAX_T) ? plan_ksplit(h, T, c.E, 3 * (int64_t)c.d / TC_BK, true, router_cg(T))
+                                                   : 1;
     const bool gemv = h->tc && T <= GEMV_MAX_T;   // few tokens: dense GEMMs as weight-streaming GEMVs
     sp.down = (c.standard || gemv) ? 1 : plan_ksplit(h, T, c.l, c.d / TC_BK);
     sp.shared = gemv ? 1 : plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
@@ -155,6 +176,14 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     sp.partial_floats = std::max(need(sp.router, c.E), need(sp.final_, c.d));
     sp.partial_side_floats = std::max(need(sp.down, c.l), need(sp.shared, 4 * (int64_t)c.f_shared));
     return sp;
+}
+
+// The down-projection writes z straight into the token's k slot rows (no z
+// buffer, no permute) when it is one tensor-core GEMM: it then runs after the
+// dispatch, on the caller's stream.
+bool scatter_down(const lmoe_handle *h, int64_t T)
+{
+    return h->tc && !h->cfg.standard && !gemv_experts(h, T) && plan_splits(h, T).down <= 1;
 }
 
 // The two-stream order: tensor-core path and no stage events (those time the
@@ -188,7 +217,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     Layout L;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes, 256); return at; };
-    L.status = take(256);   // first: the same offset for every T (chunked host forwards share it)
+    L.status = take(256);   // control slot first: the same offset for every T (chunked host forwards share it)
     L.r32 = take(sizeof(float) * T * c.E);
     L.p32 = take(sizeof(float) * S);
     L.blockhist = take(sizeof(int32_t) * nb * c.E);
@@ -199,7 +228,9 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.slot_of = take(sizeof(int32_t) * S);
     L.perm_tok = take(sizeof(int32_t) * S);
     L.perm_w = take(sizeof(float) * S);
-    L.z = take(c.standard ? 0 : h->tb * T * c.l);   // the standard form permutes x itself
+    // z rows: none in the standard form (which permutes x itself) or when the
+    // down-projection writes the slot rows directly
+    L.z = take((c.standard || scatter_down(h, T)) ? 0 : h->tb * T * c.l);
     L.Zp = take(h->tb * S * c.l);
     L.H = take(h->tb * S * c.f);
     L.Yp = take(h->tb * S * c.l);
@@ -208,6 +239,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.partial = take(sizeof(float) * sp.partial_floats);
     L.partial_side = take(sizeof(float) * sp.partial_side_floats);
     L.cutoff = take(sizeof(float) * T);
+    L.touched = take(sizeof(int32_t) * c.E);
     L.total = o;
     return L;
 }
@@ -393,12 +425,13 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 3: *offset = L.offsets; *bytes = sizeof(int32_t) * (c.E + 1); break;
     case 4: *offset = L.slot_of; *bytes = sizeof(int32_t) * S; break;
     case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
-    case 6: *offset = L.z; *bytes = c.standard ? 0 : h->tb * T * c.l; break;
+    case 6: *offset = L.z; *bytes = (c.standard || scatter_down(h, T)) ? 0 : h->tb * T * c.l; break;
     case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
     case 8: *offset = L.Yp; *bytes = h->tb * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
     case 10: *offset = L.status; *bytes = sizeof(int32_t); break;
     case 11: *offset = L.cutoff; *bytes = sizeof(float) * T; break;
+    case 12: *offset = L.Zp; *bytes = gemv_experts(h, T) ? 0 : h->tb * S * c.l; break;
     default: return fail(LMOE_ERR_INVALID_ARG, "unknown region %d", region);
     }
     return LMOE_OK;
@@ -434,14 +467,18 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
 {
     g_err.clear();
     if (!h || !launches) return fail(LMOE_ERR_INVALID_ARG, "NULL argument");
-    // kernels: router, top-k, scan, dispatch, down (none in the standard form), permute,
-    // gate/up, down+combine, norm, shared, final; plus one reduction per split-K GEMM
-    // other than the router's (which the top-k kernel reduces).  The two memsets
-    // (status word, per-block expert counts) are not kernels and are not counted.
+    // kernels: router, top-k, scan, dispatch (one kernel for few tokens), down
+    // (none in the standard form), permute (none when the routed GEMVs read z
+    // through the slot map), gate/up, down+combine, norm, shared, final; plus one
+    // reduction per split-K GEMM other than the router's (which the top-k kernel
+    // reduces).  Memsets (control words, per-block expert counts) are not kernels
+    // and are not counted.
     if (T == 0) { *launches = 0; return LMOE_OK; }
     const lmoe_config &c = h->cfg;
     const SplitPlan sp = plan_splits(h, T);
-    *launches = 11 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1);
+    *launches = 11 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1) -
+                (small_route(h, T) ? 3 : 0) - (gemv_experts(h, T) ? 1 : 0) - (sp.fused_router ? 1 : 0) -
+                (scatter_down(h, T) ? 1 : 0);
     return LMOE_OK;
 }
 
@@ -535,19 +572,39 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     const int bm = h->tc ? TC_BM * cg_grouped : SIMT_BM;
     const int max_mtiles = (int)((S + bm - 1) / bm + c.E);
 
-    if (reset_status) LMOE_CUDA(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    // control words: the status word (kept across the chunks of one host call),
+    // the routing ticket and the touched count
+    if (reset_status) LMOE_CUDA(cudaMemsetAsync(status, 0, 3 * sizeof(int32_t), s));
+    else LMOE_CUDA(cudaMemsetAsync(status + CTL_TICKET, 0, 2 * sizeof(int32_t), s));
+    int32_t *touched = (int32_t *)(ws + L.touched);
+    // the top-k kernel's per-block expert counts start at zero (cleared here,
+    // so that the router GEMM and the top-k kernel follow each other directly)
+    if (!small_route(h, T)) LMOE_CUDA(cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * (size_t)nb * c.E, s));
     const SplitPlan sp = plan_splits(h, T);
     float *partial = (float *)(ws + L.partial);             // router, final
     float *partial_side = (float *)(ws + L.partial_side);   // down, shared gate/up
-    const bool router_partial = h->tc && T > ROUTER_SMALL_MAX_T && sp.router > 1;
+    const bool small = small_route(h, T);
+    const bool gemv_routed = gemv_experts(h, T);
+    const bool fused_router = sp.fused_router;
+    const bool scatter = scatter_down(h, T);
+    const bool router_partial = h->tc && !small && !fused_router && sp.router > 1;
 
     // ---- the stages, each launched on stream `q`
     auto st_router = [&](cudaStream_t q) -> lmoe_status {   // r = sigmoid(x W_r^T)
         GemmArgs g = {};
         g.A = x; g.lda = c.d; g.M = (int)T; g.N = c.E; g.K = c.d;
         g.epi.out = r32; g.epi.ldo = c.E;
-        if (h->tc && T <= ROUTER_SMALL_MAX_T) {
-            LMOE_CUDA(launch_router_small((const bf16 *)x, h->Wr, T, c.E, c.d, r32, q));
+        if (small) {   // the whole routing (stages 1-4) in one launch
+            SmallRouteArgs a = {};
+            a.x = (const bf16 *)x; a.Wr = h->Wr; a.bias = h->b; a.T = (int)T; a.E = c.E; a.d = c.d; a.k = c.k;
+            a.bm = bm; a.r = r32; a.sel = selected_experts; a.p32 = p32; a.p_out = mixture_weights;
+            a.cutoff = (float *)(ws + L.cutoff); a.counts = counts; a.offsets = offsets; a.tile_off = tile_off;
+            a.slot_of = slot_of; a.perm_tok = perm_tok; a.perm_w = perm_w; a.touched = touched;
+            a.n_touched = status + CTL_NTOUCHED; a.ticket = status + CTL_TICKET;
+            LMOE_CUDA(launch_route_small(a, tk, q));
+        } else if (fused_router) {   // router, sigmoid, top-k and p in one launch
+            LMOE_CUDA(tc_router_topk((const bf16 *)x, h->Wr3, h->b, T, c.E, c.d, c.k, partial, r32, selected_experts,
+                                     p32, mixture_weights, tk, (float *)(ws + L.cutoff), blockhist, status, q));
         } else if (router_partial) {
             // raw logits in split-K slabs; the top-k kernel sums them and applies the sigmoid
             GemmArgs gp = g;
@@ -563,15 +620,18 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         return LMOE_OK;
     };
     auto st_topk = [&](cudaStream_t q) -> lmoe_status {
+        if (small || fused_router) return LMOE_OK;
         LMOE_CUDA(launch_topk(router_partial ? partial : r32, router_partial ? sp.router : 0, r32, h->b, T, c.E, c.k,
                               selected_experts, p32, mixture_weights, tk, blockhist, (float *)(ws + L.cutoff), q));
         return LMOE_OK;
     };
     auto st_scan = [&](cudaStream_t q) -> lmoe_status {
+        if (small) return LMOE_OK;
         LMOE_CUDA(launch_scan(blockhist, nb, c.E, counts, base, q));
         return LMOE_OK;
     };
     auto st_dispatch = [&](cudaStream_t q) -> lmoe_status {
+        if (small) return LMOE_OK;
         LMOE_CUDA(launch_dispatch(selected_experts, p32, base, counts, T, c.E, c.k, bm, offsets, tile_off, slot_of,
                                   perm_tok, perm_w, q));
         return LMOE_OK;
@@ -619,22 +679,41 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     };
     auto st_down = [&](cudaStream_t q) -> lmoe_status {
         if (c.standard) return LMOE_OK;   // experts read x itself
+        if (scatter) {                    // z rows straight to the slot rows: Zp[slot_of[t, j]] = z[t]
+            GemmArgs g = gd;
+            g.epi.out = Zp;
+            g.epi.ldo = c.l;
+            g.epi.slot_of = slot_of;
+            g.epi.kslots = c.k;
+            LMOE_CUDA(tc_gemm(EPI_SCATTER, g, 0, cg_dense, status, q));
+            return LMOE_OK;
+        }
         if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_STORE, gd, q));
         else if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down, partial_side, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, q));
         return LMOE_OK;
     };
     auto st_permute = [&](cudaStream_t q) -> lmoe_status {
+        if (gemv_routed || scatter) return LMOE_OK;   // z read through the slot map, or already scattered
         LMOE_CUDA(launch_permute_rows(c.standard ? x : z, perm_tok, Zp, S, c.l, (int)h->tb, q));
         return LMOE_OK;
     };
     auto st_gate_up = [&](cudaStream_t q) -> lmoe_status {
-        if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, cg_grouped, status, q));
+        if (gemv_routed) {
+            GemmArgs g = gu;
+            g.A = c.standard ? x : z;
+            g.lda = c.l;
+            LMOE_CUDA(launch_gemv_grouped(EPI_GLU, g, touched, status + CTL_NTOUCHED,
+                                          (int)std::min<int64_t>(c.E, S), perm_tok, (int)T, q));
+        } else if (h->tc) LMOE_CUDA(tc_gemm(EPI_GLU, gu, max_mtiles, cg_grouped, status, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gu, max_mtiles, q));
         return LMOE_OK;
     };
     auto st_down_combine = [&](cudaStream_t q) -> lmoe_status {
-        if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, cg_grouped, status, q));
+        if (gemv_routed)
+            LMOE_CUDA(launch_gemv_grouped(EPI_COMBINE, gc, touched, status + CTL_NTOUCHED,
+                                          (int)std::min<int64_t>(c.E, S), nullptr, (int)T, q));
+        else if (h->tc) LMOE_CUDA(tc_gemm(EPI_COMBINE, gc, max_mtiles, cg_grouped, status, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_COMBINE, tk, tk, tk, gc, max_mtiles, q));
         return LMOE_OK;
     };
@@ -682,23 +761,26 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         return LMOE_OK;
     }
 
-    // Two streams: the down-projection and the shared experts' gate/up GEMM
-    // need only x, so they run on the handle's side stream (the down GEMM
-    // first, beside the router GEMM, neither of which fills the GPU alone)
-    // while the caller's stream does the router and the latency-bound routing
-    // steps (top-k, scan, dispatch, permute), whose blocks fit beside the GEMM
-    // blocks on the same SMs.  The caller's stream waits for z before the
-    // permute, and for the shared GEMM before the routed gate/up GEMM: the
-    // routed GEMMs then start with every SM free, as their static tile
-    // schedule wants.
+    // Two streams: the shared experts' gate/up GEMM needs only x, so it runs on
+    // the handle's side stream while the caller's stream does the router and
+    // the latency-bound routing steps (top-k, scan, dispatch), whose blocks fit
+    // beside the GEMM blocks on the same SMs, and then the down-projection,
+    // whose epilogue writes z straight into the slot rows.  Where that
+    // down-projection is split along K (few tokens) or a GEMV, it runs on the
+    // side stream first instead, and the caller's stream waits for z before
+    // the permute.  The caller's stream waits for the shared GEMM before the
+    // routed gate/up GEMM: the routed GEMMs then start with every SM free, as
+    // their static tile schedule wants.
     {
         // record + wait as one step, so that a forward from another host thread
         // cannot slip its own record in between
         std::lock_guard<std::mutex> lock(h->fork_mutex);
         LMOE_CUDA(cudaEventRecord(h->ev_fork, s));
         LMOE_CUDA(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-        RUN(st_down(h->side));
-        LMOE_CUDA(cudaEventRecord(h->ev_z, h->side));
+        if (!scatter) {
+            RUN(st_down(h->side));
+            LMOE_CUDA(cudaEventRecord(h->ev_z, h->side));
+        }
         RUN(st_shared(h->side));
         LMOE_CUDA(cudaEventRecord(h->ev_join, h->side));
     }
@@ -706,9 +788,13 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     RUN(st_topk(s));
     RUN(st_scan(s));
     RUN(st_dispatch(s));
-    // a later record on the in-order side stream covers this forward's GEMMs too
-    LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_z, 0));
-    RUN(st_permute(s));
+    if (scatter) {
+        RUN(st_down(s));      // needs slot_of from the dispatch
+    } else {
+        // a later record on the in-order side stream covers this forward's GEMMs too
+        LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_z, 0));
+        RUN(st_permute(s));
+    }
     LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
     RUN(st_gate_up(s));
     RUN(st_down_combine(s));

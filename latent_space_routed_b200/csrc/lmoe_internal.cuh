@@ -31,6 +31,36 @@ template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __f
 
 __device__ __forceinline__ float sigmoidf_(float a) { return 1.0f / (1.0f + expf(-a)); }
 
+// Programmatic dependent launch.  Kernels of the forward are launched with
+// programmatic stream serialization (launch_pdl), so a kernel may start while
+// its predecessor on the stream is still finishing; griddep_wait() blocks
+// until that predecessor has completed and its writes are visible, and every
+// kernel calls it before it reads a predecessor's output or writes anything a
+// predecessor may still read.  Without a predecessor it returns at once.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream start launching (it still waits for this
+// one's completion in its own griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, args...);
+}
+
 // Gate of every expert: SwiGLU silu(g) * v, or the capped SiTU-GLU
 // cg tanh(g/cg) sigmoid(g) * cu tanh(v/cu) ("Stable LatentMoE" names SiTU-GLU;
 // this capped form reproduces its worked example).
@@ -44,11 +74,10 @@ __device__ __forceinline__ float glu_act(int act, float g, float v, float cg, fl
 // ---------------------------------------------------------------- epilogues
 // Every GEMM here computes C[m, n] = sum_k A[m, k] B[n, k] (both K-major) and
 // hands each row chunk of fp32 accumulators to one of these epilogues.
-// (Mode 2 is unused: the down-projection stores z once and a permute kernel
-// copies it to the slot rows.)
 enum EpiMode {
     EPI_STORE = 0,    // out[m, n] = C                      (final GEMM -> y)
     EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
+    EPI_SCATTER = 2,  // out[slot_of[m, j], n] = C, j < k   (down-projection -> z in the token's k slot rows)
     EPI_GLU = 3,      // out[m, n'] = act(C[gate], C[up])   (gate/up GEMMs -> h)
     EPI_COMBINE = 4,  // out[m, n] = w[m] * C               (routed down -> p-weighted rows)
     EPI_GLU_SITU = 5, // EPI_GLU with the SiTU gate, as its own instantiation
@@ -65,6 +94,8 @@ struct EpiArgs {
     int ib;                  // EPI_GLU: gate/up interleave block (columns)
     const void *residual;    // EPI_STORE: out = C + residual[m, n] (token dtype) when not NULL
     int64_t ldr;             // row stride of residual, elements
+    const int32_t *slot_of;  // EPI_SCATTER: [M, kslots] output rows of every input row
+    int kslots;
 };
 
 // Write n <= 32 consecutive values v[0..n) of row `row` starting at output column `col`.
@@ -146,14 +177,40 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
                                  float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s,
                                  const void *residual = nullptr, int64_t ldr = 0);
-// Dense bf16 GEMM of a few tokens (g.M = T <= GEMV_MAX_T, rows of A and B
+// Dense bf16 GEMM of a few tokens (g.M = T <= GEMV_MAX_T, rows of B
 // contiguous, K a multiple of 8) on CUDA cores, streaming B: EPI_STORE (with
 // the optional residual) or EPI_GLU (gate/up rows interleaved in blocks of ib).
-constexpr int GEMV_MAX_T = 2;
+constexpr int GEMV_MAX_T = 4;
 cudaError_t launch_gemv(int mode, const GemmArgs &g, cudaStream_t s);
-// Router scores for a few tokens on CUDA cores: r[t, e] = sigmoid(sum_k x[t, k] W[e, k]),
-// x bf16 [T, d], W fp32 [E, d] (fixed summation order, deterministic).
-cudaError_t launch_router_small(const bf16 *x, const float *W, int64_t T, int E, int d, float *r, cudaStream_t s);
+// The routed experts' GEMMs of a few slot rows per expert, streaming only the
+// touched experts' weights: g.offsets [E+1] gives each expert's slot rows
+// (at most max_rows_per_group <= GEMV_MAX_T of them), touched[0 .. *n_touched)
+// the experts with at least one (max_touched bounds the count); input row of
+// slot s is amap[s] (or s when amap is NULL), output row s.  EPI_GLU
+// (g.epi.ib-interleaved gate/up rows) or EPI_COMBINE (g.epi.row_w[s] * sum).
+cudaError_t launch_gemv_grouped(int mode, const GemmArgs &g, const int32_t *touched, const int32_t *n_touched,
+                                int max_touched, const int32_t *amap, int max_rows_per_group, cudaStream_t s);
+// The whole routing of T <= ROUTE_SMALL_MAX_T tokens in one launch: router
+// scores r [T, E] (fp32, CUDA cores), top-k, p (fp32 and token dtype), the
+// Quantile-Balancing cutoff, expert counts, offsets [E+1], the m-tile prefix
+// for tiles of bm rows, slot_of, the slot -> token map and slot weights, and
+// the touched experts in ascending order with their count.  *ticket must be
+// zero at launch; the kernel leaves it zero.
+constexpr int ROUTE_SMALL_MAX_T = 8;
+struct SmallRouteArgs {
+    const bf16 *x;
+    const float *Wr, *bias;
+    int T, E, d, k, bm;
+    float *r;
+    int32_t *sel;
+    float *p32;
+    void *p_out;
+    float *cutoff;
+    int32_t *counts, *offsets, *tile_off, *slot_of, *perm_tok;
+    float *perm_w;
+    int32_t *touched, *n_touched, *ticket;
+};
+cudaError_t launch_route_small(const SmallRouteArgs &a, int out_bf16, cudaStream_t s);
 
 // Weight repacking (create time).
 cudaError_t launch_pack_glu(const void *G, const void *U, void *P, int nE, int F, int K, int ib, int elem_bytes,

@@ -48,7 +48,7 @@ __device__ __forceinline__ void store8(float *p, const float *v)
 }
 
 // One block per token, one thread per 8 consecutive latent columns: the
-// thread loads its columns from the token's k slot rows (four rows in flight
+// thread loads its columns from the token's k slot rows (eight rows in flight
 // at a time), adds them in fp32 in slot order, and keeps u in registers for
 // the norm.
 template <typename TT>
@@ -59,6 +59,8 @@ combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_
     __shared__ int slots[64];
     __shared__ float red[32];
     const int64_t t = blockIdx.x;
+    griddep_wait();
+    griddep_launch_dependents();
     for (int j = threadIdx.x; j < k; j += blockDim.x) slots[j] = slot_of[t * k + j];
     __syncthreads();
     const int c0 = threadIdx.x * 8;
@@ -66,6 +68,15 @@ combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_
     float u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (active) {
         int j = 0;
+        for (; j + 8 <= k; j += 8) {      // eight rows in flight, added in slot order
+            float v[8][8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) load8(Yp + (int64_t)slots[j + q] * l + c0, v[q]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) u[i] += v[q][i];
+        }
         for (; j + 4 <= k; j += 4) {
             float v[4][8];
 #pragma unroll
@@ -166,6 +177,8 @@ splitk_reduce_kernel(const float *__restrict__ partial, int ksplit, int64_t M, i
     const int64_t m = blockIdx.y;
     const int nout = (MODE == EPI_GLU) ? N / 2 : N;
     const int j0 = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    griddep_wait();
+    griddep_launch_dependents();
     if (j0 >= nout) return;
     const int64_t slab = M * (int64_t)N;
     float r[4];
@@ -232,15 +245,13 @@ cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, in
     const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
     dim3 grid((unsigned)((nvec + threads - 1) / threads), (unsigned)M);
     if (mode == EPI_GLU)
-        splitk_reduce_kernel<EPI_GLU><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo,
-                                                               nullptr, 0);
-    else if (mode == EPI_SIGMOID)
-        splitk_reduce_kernel<EPI_SIGMOID><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out,
-                                                                   ldo, nullptr, 0);
-    else
-        splitk_reduce_kernel<EPI_STORE><<<grid, threads, 0, s>>>(partial, ksplit, M, N, act, gate_cap, up_cap, ib, out, ldo,
-                                                                 (const bf16 *)residual, ldr);
-    return cudaGetLastError();
+        return launch_pdl(splitk_reduce_kernel<EPI_GLU>, grid, dim3(threads), 0, s, partial, ksplit, M, N, act,
+                          gate_cap, up_cap, ib, out, ldo, (const bf16 *)nullptr, (int64_t)0);
+    if (mode == EPI_SIGMOID)
+        return launch_pdl(splitk_reduce_kernel<EPI_SIGMOID>, grid, dim3(threads), 0, s, partial, ksplit, M, N, act,
+                          gate_cap, up_cap, ib, out, ldo, (const bf16 *)nullptr, (int64_t)0);
+    return launch_pdl(splitk_reduce_kernel<EPI_STORE>, grid, dim3(threads), 0, s, partial, ksplit, M, N, act, gate_cap,
+                      up_cap, ib, out, ldo, (const bf16 *)residual, ldr);
 }
 
 cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,
@@ -250,12 +261,10 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
     if (k > 64 || l % 8 || l > 8192 || ld_hs % 8 || col0 % 8) return cudaErrorInvalidValue;
     const int threads = ((l / 8 + 31) / 32) * 32;
     if (tok_bf16)
-        combine_norm_kernel<bf16><<<(unsigned)T, threads, 0, s>>>((const bf16 *)Yp, slot_of, l, k, eps, (bf16 *)u_out,
-                                                                    (bf16 *)hs, ld_hs, col0);
-    else
-        combine_norm_kernel<float><<<(unsigned)T, threads, 0, s>>>((const float *)Yp, slot_of, l, k, eps,
-                                                                     (float *)u_out, (float *)hs, ld_hs, col0);
-    return cudaGetLastError();
+        return launch_pdl(combine_norm_kernel<bf16>, dim3((unsigned)T), dim3(threads), 0, s, (const bf16 *)Yp, slot_of,
+                          l, k, eps, (bf16 *)u_out, (bf16 *)hs, ld_hs, col0);
+    return launch_pdl(combine_norm_kernel<float>, dim3((unsigned)T), dim3(threads), 0, s, (const float *)Yp, slot_of, l,
+                      k, eps, (float *)u_out, (float *)hs, ld_hs, col0);
 }
 
 cudaError_t launch_pack_glu(const void *G, const void *U, void *P, int nE, int F, int K, int ib, int elem_bytes,

@@ -18,6 +18,7 @@
 #include <float.h>
 
 #include "lmoe_internal.cuh"
+#include "topk.cuh"
 
 namespace lmoe {
 namespace {
@@ -25,49 +26,9 @@ namespace {
 constexpr int TOPK_WARPS = 8;   // one token per warp, 8 tokens per block
 constexpr int KMAX = 64;
 
-// "a before b": larger biased score first, equal scores to the lower index.
-__device__ __forceinline__ bool ahead(float va, int ia, float vb, int ib)
-{
-    return va > vb || (va == vb && ia < ib);
-}
-
-// Bitonic sort of a lane's N (score, expert) pairs into "ahead" order, in registers.
-template <int N>
-__device__ __forceinline__ void sort_lane(float (&v)[N], int (&ix)[N])
-{
-#pragma unroll
-    for (int kk = 2; kk <= N; kk <<= 1)
-#pragma unroll
-        for (int j = kk >> 1; j > 0; j >>= 1)
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                const int m = i ^ j;
-                if (m > i) {
-                    const bool first_ahead = ahead(v[i], ix[i], v[m], ix[m]);
-                    if (((i & kk) == 0) != first_ahead) {
-                        const float tv = v[i]; v[i] = v[m]; v[m] = tv;
-                        const int ti = ix[i]; ix[i] = ix[m]; ix[m] = ti;
-                    }
-                }
-            }
-}
-
-// Order-preserving 32-bit key of a score: a > b as floats exactly when
-// key(a) > key(b) as unsigned integers (for -0 and +0 alike only if the caller
-// made -0 into +0, which it does).
-__device__ __forceinline__ uint32_t score_key(float v)
-{
-    const uint32_t u = __float_as_uint(v);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Top-k for one token per warp.  Lane L holds experts L, L + 32, ... (EPL of
-// them, padded with -inf), sorts them, and the k rounds are a tournament over
-// the 32 lane heads: the largest head score (one warp max-reduction over the
-// score keys), then the lowest expert index among the heads with that score
-// (one min-reduction), so equal scores go to the lower index; the winning lane
-// pops its head.  The raw scores of the chosen experts are normalised by their
-// sum (a fixed butterfly order, so the result does not depend on timing).
+// Top-k for one token per warp (warp_topk), then the raw scores of the chosen
+// experts normalised by their sum (a fixed butterfly order, so the result does
+// not depend on timing), and each block's per-expert selection counts.
 //
 // nsplit = 0: r_in holds the router scores r [T, E].  nsplit > 0: r_in holds
 // nsplit fp32 partial slabs [nsplit, T, E] of the router logits (split-K
@@ -81,6 +42,8 @@ topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const floa
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = (int64_t)blockIdx.x * TOPK_WARPS + warp;
+    griddep_wait();
+    griddep_launch_dependents();
     if (t >= T) return;
     float v[EPL];
     int ix[EPL];
@@ -99,35 +62,12 @@ topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const floa
                 r_out[t * E + e] = r;
             }
         }
-        // NaN / -inf map to -FLT_MAX so that a real candidate always beats the
-        // padding; adding +0 turns -0 into +0, so equal scores get equal keys
-        v[i] = e < E ? fmaxf(r + bias[e], -FLT_MAX) + 0.0f : -INFINITY;
+        v[i] = e < E ? biased_key(r, bias[e]) : -INFINITY;
     }
-    sort_lane<EPL>(v, ix);
-    int mine0 = 0, mine1 = 0;    // selection j kept by lane j % 32 (slot j / 32)
-    for (int j = 0; j < k; ++j) {
-        const uint32_t key = score_key(v[0]);
-        const uint32_t best = __reduce_max_sync(0xffffffffu, key);
-        const int bi = (int)__reduce_min_sync(0xffffffffu, key == best ? (uint32_t)ix[0] : 0xffffffffu);
-        if (lane == (bi & 31)) {            // the winner pops its head
-#pragma unroll
-            for (int i = 0; i + 1 < EPL; ++i) { v[i] = v[i + 1]; ix[i] = ix[i + 1]; }
-            v[EPL - 1] = -INFINITY;
-            ix[EPL - 1] = 0x7fffffff;
-        }
-        if (lane == (j & 31)) {
-            if (j < 32) mine0 = bi; else mine1 = bi;
-        }
-    }
-    // Quantile-Balancing cutoff: the (k+1)-th biased score, one more round
-    // (-inf when k = E leaves nothing unselected)
-    {
-        const uint32_t key = score_key(v[0]);
-        const uint32_t best = __reduce_max_sync(0xffffffffu, key);
-        const int bi = (int)__reduce_min_sync(0xffffffffu, key == best ? (uint32_t)ix[0] : 0xffffffffu);
-        const float cv = __shfl_sync(0xffffffffu, v[0], bi & 31);
-        if (lane == 0) cutoff[t] = k < E ? cv : -INFINITY;
-    }
+    int mine0, mine1;
+    float cv;
+    warp_topk<EPL>(v, ix, k, E, lane, &mine0, &mine1, &cv);
+    if (lane == 0) cutoff[t] = cv;
     const float *rr = nsplit ? r_out : r_in;
     if (nsplit) __syncwarp();               // r_out of this token, written by every lane, is visible
     const float r0 = lane < k ? rr[t * E + mine0] : 0.f;
@@ -192,6 +132,8 @@ scan_cols_kernel(const int32_t *__restrict__ blockhist, int nb, int32_t *__restr
 {
     __shared__ int s_warp[SCAN_NT / 32];
     const int e = blockIdx.x;
+    griddep_wait();
+    griddep_launch_dependents();
     const int32_t *h = blockhist + (int64_t)e * nb;
     int32_t *o = base + (int64_t)e * nb;
     int carry = 0;
@@ -230,6 +172,8 @@ dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, 
     int *s_off = s_dyn;                             // [E + 1]
     uint32_t *bits = (uint32_t *)(s_dyn + E + 1);   // [E]
     __shared__ int s_warp[DISP_NT / 32];
+    griddep_wait();
+    griddep_launch_dependents();
     {   // expert offsets: E <= 1024 counts, four per thread
         const int e0 = threadIdx.x * 4;
         int v[4], tv[4];
@@ -280,57 +224,193 @@ dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, 
     }
 }
 
-// Router for a few tokens: one block per (expert row e, ROUTER_TB tokens).
-// The block's 8 warps stream W[e] (fp32, 16-byte loads) in interleaved
-// 512-byte pieces against the same columns of each token; each warp adds its
-// lanes in a fixed butterfly order and the warps' partial sums are added in
-// warp order, so the result does not depend on timing.
-constexpr int ROUTER_TB = 8;
-constexpr int ROUTER_WARPS = 8;
+// The whole routing of a few tokens (T <= ROUTE_SMALL_MAX_T) in one launch.
+//
+// Every block first computes the router scores of one expert row e for all T
+// tokens: its 8 warps split W_r[e] (fp32) into interleaved 4 KB pieces, each
+// lane keeping four 16-byte loads in flight, against the same columns of every
+// token; lanes are added in a fixed butterfly order and warps in warp order
+// (deterministic), and r[t, e] = sigmoid of the sum.  The block then counts
+// itself done on a ticket; the last block to finish (all scores are written
+// and, by the writers' fences, visible) does the rest:
+//   top-k of each token (one warp per token, warp_topk), the Quantile-Balancing
+//   cutoff, p from the raw scores;
+//   the stable counting sort of the T k slots by expert in shared memory: one
+//   bit word per expert marks the tokens that chose it, counts are popcounts,
+//   offsets and the m-tile prefix (tiles of bm rows) are block scans, and slot
+//   (t, j) with e = sel[t, j] goes to offsets[e] + #{t' < t that chose e};
+//   the touched experts (count > 0) in ascending order, for the grouped GEMVs;
+// and puts the ticket back to zero for the next call.
+constexpr int RS_WARPS = 8;
 
-__global__ void __launch_bounds__(ROUTER_WARPS * 32)
-router_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ W, int64_t T, int E, int d,
-                    float *__restrict__ r)
+template <typename TO, int EPL>
+__global__ void __launch_bounds__(RS_WARPS * 32)
+route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, const float *__restrict__ bias, int T,
+                   int E, int d, int k, int bm, float *__restrict__ r, int32_t *__restrict__ sel,
+                   float *__restrict__ p32, TO *__restrict__ p_out, float *__restrict__ cutoff,
+                   int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ tile_off,
+                   int32_t *__restrict__ slot_of, int32_t *__restrict__ perm_tok, float *__restrict__ perm_w,
+                   int32_t *__restrict__ touched, int32_t *__restrict__ n_touched, int32_t *ticket)
 {
-    __shared__ float part[ROUTER_WARPS][ROUTER_TB];
+    __shared__ float part[RS_WARPS][ROUTE_SMALL_MAX_T];
+    __shared__ int s_last;
+    __shared__ uint32_t s_bits[1024];
+    __shared__ int s_off[1024 + 1];
+    __shared__ int s_sel[ROUTE_SMALL_MAX_T * KMAX];
+    __shared__ float s_p[ROUTE_SMALL_MAX_T * KMAX];
+    __shared__ int s_warp[RS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = blockIdx.x;
-    const int64_t t0 = (int64_t)blockIdx.y * ROUTER_TB;
-    float acc[ROUTER_TB];
+    griddep_wait();
+    griddep_launch_dependents();
+
+    // ---- router scores of expert e
+    float acc[ROUTE_SMALL_MAX_T];
 #pragma unroll
-    for (int j = 0; j < ROUTER_TB; ++j) acc[j] = 0.f;
-    const float4 *w = reinterpret_cast<const float4 *>(W + (int64_t)e * d);
-    for (int c = warp * 32 + lane; c < d / 4; c += ROUTER_WARPS * 32) {
-        const float4 wv = __ldg(w + c);
+    for (int t = 0; t < ROUTE_SMALL_MAX_T; ++t) acc[t] = 0.f;
+    const float4 *w = reinterpret_cast<const float4 *>(Wr + (int64_t)e * d);
+    const int nv = d / 4;
+    constexpr int STEP = RS_WARPS * 32;
+    for (int c0 = warp * 32 + lane; c0 < nv; c0 += 4 * STEP) {
+        float4 wv[4];
 #pragma unroll
-        for (int j = 0; j < ROUTER_TB; ++j) {
-            if (t0 + j < T) {
-                const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (t0 + j) * d) + c);
-                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
-                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
-                acc[j] = fmaf(wv.x, a.x, acc[j]);
-                acc[j] = fmaf(wv.y, a.y, acc[j]);
-                acc[j] = fmaf(wv.z, b.x, acc[j]);
-                acc[j] = fmaf(wv.w, b.y, acc[j]);
+        for (int u = 0; u < 4; ++u) wv[u] = c0 + u * STEP < nv ? __ldg(w + c0 + u * STEP) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int t = 0; t < ROUTE_SMALL_MAX_T; ++t) {
+            if (t < T) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (c0 + u * STEP < nv) {
+                        const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (int64_t)t * d) + c0 + u * STEP);
+                        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.x));
+                        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xv.y));
+                        acc[t] = fmaf(wv[u].x, a.x, acc[t]);
+                        acc[t] = fmaf(wv[u].y, a.y, acc[t]);
+                        acc[t] = fmaf(wv[u].z, b.x, acc[t]);
+                        acc[t] = fmaf(wv[u].w, b.y, acc[t]);
+                    }
+                }
             }
         }
     }
 #pragma unroll
-    for (int j = 0; j < ROUTER_TB; ++j) {
+    for (int t = 0; t < ROUTE_SMALL_MAX_T; ++t)
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-    }
+        for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
     if (lane == 0) {
 #pragma unroll
-        for (int j = 0; j < ROUTER_TB; ++j) part[warp][j] = acc[j];
+        for (int t = 0; t < ROUTE_SMALL_MAX_T; ++t) part[warp][t] = acc[t];
     }
     __syncthreads();
-    if (threadIdx.x < ROUTER_TB && t0 + threadIdx.x < T) {
+    if (threadIdx.x < T) {
         float a = 0.f;
 #pragma unroll
-        for (int q = 0; q < ROUTER_WARPS; ++q) a += part[q][threadIdx.x];
-        r[(t0 + threadIdx.x) * E + e] = sigmoidf_(a);
+        for (int q = 0; q < RS_WARPS; ++q) a += part[q][threadIdx.x];
+        r[(int64_t)threadIdx.x * E + e] = sigmoidf_(a);
+        __threadfence();                       // the score is visible before the ticket counts this block
     }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // ---- the last block: top-k, p, cutoff (one warp per token)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) s_bits[i] = 0u;
+    __syncthreads();
+    for (int t = warp; t < T; t += RS_WARPS) {
+        float v[EPL];
+        int ix[EPL];
+        float rv[EPL];
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const int ee = lane + 32 * i;
+            ix[i] = ee;
+            rv[i] = ee < E ? __ldcg(r + (int64_t)t * E + ee) : 0.f;
+            v[i] = ee < E ? biased_key(rv[i], bias[ee]) : -INFINITY;
+        }
+        int mine0, mine1;
+        float cv;
+        warp_topk<EPL>(v, ix, k, E, lane, &mine0, &mine1, &cv);
+        if (lane == 0) cutoff[t] = cv;
+        const float r0 = lane < k ? __ldcg(r + (int64_t)t * E + mine0) : 0.f;
+        const float r1 = lane + 32 < k ? __ldcg(r + (int64_t)t * E + mine1) : 0.f;
+        float sum = r0 + r1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int j = lane + 32 * h;
+            if (j < k) {
+                const int ee = h ? mine1 : mine0;
+                const float p = (h ? r1 : r0) / sum;
+                sel[(int64_t)t * k + j] = ee;
+                p32[(int64_t)t * k + j] = p;
+                p_out[(int64_t)t * k + j] = from_f32<TO>(p);
+                s_sel[t * k + j] = ee;
+                s_p[t * k + j] = p;
+                atomicOr(&s_bits[ee], 1u << t);
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- counting sort of the T k slots by expert
+    {
+        const int e0 = threadIdx.x * 4;
+        int c[4], tl[4], used[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            c[q] = e0 + q < E ? __popc(s_bits[e0 + q]) : 0;
+            tl[q] = (c[q] + bm - 1) / bm;
+            used[q] = c[q] > 0 ? 1 : 0;
+        }
+        int total = 0;
+        int run = block_exclusive_scan<RS_WARPS * 32>(c[0] + c[1] + c[2] + c[3], s_warp, &total);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (e0 + q < E) {
+                s_off[e0 + q] = run;
+                offsets[e0 + q] = run;
+                counts[e0 + q] = c[q];
+            }
+            run += c[q];
+        }
+        if (threadIdx.x == 0) {
+            s_off[E] = total;
+            offsets[E] = total;
+        }
+        int ttot = 0;
+        int trun = block_exclusive_scan<RS_WARPS * 32>(tl[0] + tl[1] + tl[2] + tl[3], s_warp, &ttot);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (e0 + q < E) tile_off[e0 + q] = trun;
+            trun += tl[q];
+        }
+        if (threadIdx.x == 0) tile_off[E] = ttot;
+        int ntot = 0;
+        int nrun = block_exclusive_scan<RS_WARPS * 32>(used[0] + used[1] + used[2] + used[3], s_warp, &ntot);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (used[q]) touched[nrun] = e0 + q;
+            nrun += used[q];
+        }
+        if (threadIdx.x == 0) *n_touched = ntot;
+    }
+    __syncthreads();
+    const int S = T * k;
+    for (int i = threadIdx.x; i < S; i += blockDim.x) {
+        const int t = i / k;
+        const int ee = s_sel[i];
+        const int pos = s_off[ee] + __popc(s_bits[ee] & ((1u << t) - 1u));
+        slot_of[i] = pos;
+        perm_tok[pos] = t;
+        perm_w[pos] = s_p[i];
+    }
+    if (threadIdx.x == 0) *ticket = 0;
 }
 
 // Zp[m, :] = z[perm_tok[m], :]: one warp per slot row, 16-byte vectors.
@@ -339,6 +419,8 @@ permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ per
                     int64_t S, int vec_per_row)
 {
     const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    griddep_wait();
+    griddep_launch_dependents();
     if (m >= S) return;
     const int lane = threadIdx.x & 31;
     const uint4 *src = z + (int64_t)perm_tok[m] * vec_per_row;
@@ -348,23 +430,14 @@ permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ per
 
 }  // namespace
 
-cudaError_t launch_router_small(const bf16 *x, const float *W, int64_t T, int E, int d, float *r, cudaStream_t s)
-{
-    if (T == 0) return cudaSuccess;
-    if (d % 4) return cudaErrorInvalidValue;
-    dim3 grid((unsigned)E, (unsigned)((T + ROUTER_TB - 1) / ROUTER_TB));
-    router_small_kernel<<<grid, ROUTER_WARPS * 32, 0, s>>>(x, W, T, E, d, r);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
                                 cudaStream_t s)
 {
     if (S == 0) return cudaSuccess;
     if (((int64_t)l * elem_bytes) % 16) return cudaErrorInvalidValue;
     const int vpr = (int)((int64_t)l * elem_bytes / 16);
-    permute_rows_kernel<<<(unsigned)((S + 7) / 8), 256, 0, s>>>((const uint4 *)z, perm_tok, (uint4 *)Zp, S, vpr);
-    return cudaGetLastError();
+    return launch_pdl(permute_rows_kernel, dim3((unsigned)((S + 7) / 8)), dim3(256), 0, s, (const uint4 *)z, perm_tok,
+                      (uint4 *)Zp, S, vpr);
 }
 
 namespace {
@@ -374,9 +447,8 @@ cudaError_t run_topk(const float *r_in, int nsplit, float *r_out, const float *b
                      int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, float *cutoff, cudaStream_t s)
 {
     const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
-    topk_kernel<TO, EPL><<<nblk, TOPK_WARPS * 32, 0, s>>>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, (TO *)p_out,
-                                                         blockhist, nb, cutoff);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel<TO, EPL>, dim3(nblk), dim3(TOPK_WARPS * 32), 0, s, r_in, nsplit, r_out, bias, T, E,
+                      k, sel, p32, (TO *)p_out, blockhist, nb, cutoff);
 }
 
 template <typename TO>
@@ -403,17 +475,46 @@ cudaError_t launch_topk(const float *r_in, int nsplit, float *r_out, const float
 {
     if (k > KMAX || E > 1024 || nsplit < 0) return cudaErrorInvalidValue;
     const int64_t nb = (T + ROUTE_TPB - 1) / ROUTE_TPB;
-    cudaError_t e = cudaMemsetAsync(blockhist, 0, sizeof(int32_t) * nb * E, s);
-    if (e != cudaSuccess) return e;
     if (out_bf16)
         return run_topk_epl<bf16>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, cutoff, s);
     return run_topk_epl<float>(r_in, nsplit, r_out, bias, T, E, k, sel, p32, p_out, blockhist, (int)nb, cutoff, s);
 }
 
+namespace {
+
+template <typename TO, int EPL>
+cudaError_t run_route_small(const SmallRouteArgs &a, cudaStream_t s)
+{
+    return launch_pdl(route_small_kernel<TO, EPL>, dim3((unsigned)a.E), dim3(RS_WARPS * 32), 0, s, a.x, a.Wr, a.bias,
+                      a.T, a.E, a.d, a.k, a.bm, a.r, a.sel, a.p32, (TO *)a.p_out, a.cutoff, a.counts, a.offsets,
+                      a.tile_off, a.slot_of, a.perm_tok, a.perm_w, a.touched, a.n_touched, a.ticket);
+}
+
+template <typename TO>
+cudaError_t run_route_small_epl(const SmallRouteArgs &a, cudaStream_t s)
+{
+    const int epl = (a.E + 31) / 32;
+    if (epl <= 1) return run_route_small<TO, 1>(a, s);
+    if (epl <= 2) return run_route_small<TO, 2>(a, s);
+    if (epl <= 4) return run_route_small<TO, 4>(a, s);
+    if (epl <= 8) return run_route_small<TO, 8>(a, s);
+    if (epl <= 16) return run_route_small<TO, 16>(a, s);
+    return run_route_small<TO, 32>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_route_small(const SmallRouteArgs &a, int out_bf16, cudaStream_t s)
+{
+    if (a.T < 1 || a.T > ROUTE_SMALL_MAX_T || a.k > KMAX || a.E > 1024 || a.d % 4 || a.bm < 1)
+        return cudaErrorInvalidValue;
+    if (out_bf16) return run_route_small_epl<bf16>(a, s);
+    return run_route_small_epl<float>(a, s);
+}
+
 cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts, int32_t *base, cudaStream_t s)
 {
-    scan_cols_kernel<<<E, SCAN_NT, 0, s>>>(blockhist, nb, base, counts);
-    return cudaGetLastError();
+    return launch_pdl(scan_cols_kernel, dim3(E), dim3(SCAN_NT), 0, s, blockhist, nb, base, counts);
 }
 
 cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, const int32_t *counts,
@@ -423,9 +524,8 @@ cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t 
     if (E > 1024) return cudaErrorInvalidValue;
     const int nb = (int)((T + ROUTE_TPB - 1) / ROUTE_TPB);
     const size_t smem = sizeof(int) * (2 * (size_t)E + 1);
-    dispatch_kernel<<<nb, DISP_NT, smem, s>>>(sel, p32, base, counts, T, E, k, nb, bm, offsets, tile_off, slot_of,
-                                               perm_tok, perm_w);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_kernel, dim3(nb), dim3(DISP_NT), smem, s, sel, p32, base, counts, T, E, k, nb, bm,
+                      offsets, tile_off, slot_of, perm_tok, perm_w);
 }
 
 }  // namespace lmoe

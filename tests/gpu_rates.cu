@@ -11,11 +11,16 @@
 //   bulk  bytes per second moved from global memory into shared memory by the
 //         bulk-copy engine (cp.async.bulk ... complete_tx), one CTA per SM,
 //         each keeping `stages` copies of `chunk` bytes in flight over a buffer
-//         of `span` bytes (L2-resident when small, HBM-bound when large).
+//         of `span` bytes (L2-resident when small, HBM-bound when large), issued
+//         by one thread or split over two;
+//   tile  the same with tiled tensor copies (cp.async.bulk.tensor.2d, 128-byte
+//         swizzle, boxes of 64 bf16 x R rows: the GEMM's operand loads).
 //
 // Every wait is bounded (about 2 s of SM cycles); a wait that gives up sets
 // *status, the CTA drains what it still has in flight (again bounded) and
 // returns.  Output: one JSON object per line on stdout.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -97,24 +102,34 @@ mma_kernel(int M, int N, int nacc, int blocked, int iters, unsigned long long *c
     const uint32_t sa = su32(ops), sb = sa + 128 * 128;
     if (threadIdx.x == 0 && rank == 0) {
         const long long t0 = clock64();
+        uint64_t ad[4], bd[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            ad[k] = desc_sw128(sa + 32u * k);
+            bd[k] = desc_sw128(sb + 32u * k);
+        }
+        auto mma = [&](uint32_t d, int k, uint32_t acc) {
+            if (CG == 2)
+                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                             "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                             ::"r"(d), "l"(ad[k]), "l"(bd[k]), "r"(idesc), "r"(acc));
+            else
+                asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                             "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                             ::"r"(d), "l"(ad[k]), "l"(bd[k]), "r"(idesc), "r"(acc));
+        };
+        // the issuing loop is kept to a few instructions per MMA (precomputed
+        // descriptors, no division): a heavier loop throttles the issue itself
         for (int it = 0; it < iters; ++it) {
-            // interleaved: k-step outer, accumulator inner; blocked: accumulator
-            // outer, so one accumulator takes all 4 k-steps of a 64-wide slice
-            for (int q = 0; q < 4 * nacc; ++q) {
-                const int k = blocked ? q % 4 : q / nacc, a = blocked ? q / 4 : q % nacc;
-                const uint64_t ad = desc_sw128(sa + 32u * k), bd = desc_sw128(sb + 32u * k);
-                {
-                    const uint32_t d = tmem + (uint32_t)(a * N);
-                    const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
-                    if (CG == 2)
-                        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                                     "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                                     ::"r"(d), "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
-                    else
-                        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                                     "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                                     ::"r"(d), "l"(ad), "l"(bd), "r"(idesc), "r"(acc));
+            if (blocked) {      // accumulator outer: one accumulator takes all 4 k-steps of a 64-wide slice
+                for (int a = 0; a < nacc; ++a) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) mma(tmem + (uint32_t)(a * N), k, (it > 0 || k > 0) ? 1u : 0u);
                 }
+            } else {            // k-step outer, accumulator inner
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    for (int a = 0; a < nacc; ++a) mma(tmem + (uint32_t)(a * N), k, (it > 0 || k > 0) ? 1u : 0u);
             }
         }
         if (CG == 2)
@@ -141,39 +156,55 @@ mma_kernel(int M, int N, int nacc, int blocked, int iters, unsigned long long *c
 
 static constexpr int MMA_SMEM = 128 * 128 + 256 * 128 + 1024;
 
-// ------------------------------------------------------------------ bulk copies
-constexpr int MAX_STAGES = 12;
+// ------------------------------------------------------------------ bulk and tile copies
+constexpr int MAX_STAGES = 24;
 
-__global__ void __launch_bounds__(32, 1)
-bulk_kernel(const uint8_t *src, size_t span, int chunk, int stages, int iters, int *status)
+// One ring of `stages` copies per issuing thread (threads 0 and 32 when
+// issuers = 2, each with its own half of the buffer and barriers).
+template <bool TILED>
+__global__ void __launch_bounds__(64, 1)
+copy_kernel(const uint8_t *src, size_t span, const __grid_constant__ CUtensorMap tm, int tile_rows, int rows_total,
+            int kblocks, int chunk, int stages, int issuers, int iters, int *status)
 {
-    extern __shared__ __align__(1024) uint8_t buf[];
+    extern __shared__ uint8_t dynbuf[];
     __shared__ __align__(8) uint64_t bars[MAX_STAGES];
-    if (threadIdx.x != 0) return;
-    for (int s = 0; s < stages; ++s) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&bars[s])) : "memory");
+    uint8_t *buf = dynbuf + ((1024 - (su32(dynbuf) & 1023)) & 1023);   // 1024-aligned (128-byte swizzle)
+    const int who = threadIdx.x == 0 ? 0 : (threadIdx.x == 32 && issuers == 2 ? 1 : -1);
+    if (who < 0) return;
+    const int st = stages / issuers, s_base = who * st;
+    for (int s = 0; s < st; ++s) asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&bars[s_base + s])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    const size_t nchunks = span / (size_t)chunk;
-    size_t pos = ((size_t)blockIdx.x * 977) % nchunks;
+    const size_t nchunks = TILED ? (size_t)(rows_total / tile_rows) * kblocks : span / (size_t)chunk;
+    size_t pos = ((size_t)blockIdx.x * 977 + who * 131) % nchunks;
+    const int my_iters = iters / issuers;
     int issued = 0, done = 0;
     bool ok = true;
-    for (int it = 0; it < iters && ok; ++it) {
-        const int s = it % stages;
-        if (it >= stages) {   // the copy that used this stage last has landed
-            ok = wait_bounded(su32(&bars[s]), (uint32_t)((it / stages - 1) & 1));
+    for (int it = 0; it < my_iters && ok; ++it) {
+        const int s = it % st;
+        if (it >= st) {   // the copy that used this stage last has landed
+            ok = wait_bounded(su32(&bars[s_base + s]), (uint32_t)((it / st - 1) & 1));
             if (!ok) break;
             ++done;
         }
-        const uint32_t bar = su32(&bars[s]);
+        const uint32_t bar = su32(&bars[s_base + s]);
+        const uint32_t dst = su32(buf + (size_t)(s_base + s) * chunk);
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(chunk) : "memory");
-        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                     ::"r"(su32(buf + (size_t)s * chunk)), "l"(src + pos * chunk), "r"(chunk), "r"(bar) : "memory");
+        if (TILED) {
+            const int c0 = (int)(pos % kblocks) * 64, c1 = (int)(pos / kblocks) * tile_rows;
+            asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                         " [%0], [%1, {%3, %4}], [%2];"
+                         ::"r"(dst), "l"((uint64_t)&tm), "r"(bar), "r"(c0), "r"(c1) : "memory");
+        } else {
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         ::"r"(dst), "l"(src + pos * chunk), "r"(chunk), "r"(bar) : "memory");
+        }
         ++issued;
         pos += 148 * 3 + 1;
         if (pos >= nchunks) pos %= nchunks;
     }
     // drain every copy still in flight (bounded)
     for (int i = done; i < issued; ++i)
-        if (!wait_bounded(su32(&bars[i % stages]), (uint32_t)((i / stages) & 1))) { ok = false; break; }
+        if (!wait_bounded(su32(&bars[s_base + i % st]), (uint32_t)((i / st) & 1))) { ok = false; break; }
     if (!ok) atomicOr(status, 4);
 }
 
@@ -232,38 +263,75 @@ int main(int argc, char **argv)
         }
     }
 
-    // bulk copies: an L2-resident span and an HBM-sized one
-    const size_t spans[] = {(size_t)16 << 20, (size_t)48 << 20, (size_t)4 << 30};
-    // (chunk bytes, stages): 128 KB and 192 KB in flight per SM in 16 KB copies, 192 KB in 32 KB copies
-    const int cases[][2] = {{16384, 8}, {16384, 12}, {32768, 6}};
+    // copies: L2-resident and HBM-sized spans; bulk (1D) and tiled (2D, the GEMM's form)
     uint8_t *src;
-    CK(cudaMalloc(&src, spans[2]));
-    CK(cudaMemset(src, 1, spans[2]));
-    for (size_t span : spans) {
-        for (const auto &cs : cases) {
-            const int chunk = cs[0], stages = cs[1];
-            const size_t smem = (size_t)chunk * stages;
-            CK(cudaFuncSetAttribute(bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-            const int iters = (int)(((size_t)8 << 30) / ((size_t)sms * chunk));   // 8 GiB in all
-            cudaEvent_t a, b;
-            CK(cudaEventCreate(&a));
-            CK(cudaEventCreate(&b));
-            float best = 1e30f;
-            for (int rep = 0; rep < 3; ++rep) {
-                CK(cudaEventRecord(a));
-                bulk_kernel<<<sms, 32, smem>>>(src, span, chunk, stages, iters, status);
-                CK(cudaEventRecord(b));
-                CK(cudaEventSynchronize(b));
-                float ms = 0;
-                CK(cudaEventElapsedTime(&ms, a, b));
-                if (ms < best) best = ms;
+    const size_t big = (size_t)4 << 30;
+    CK(cudaMalloc(&src, big));
+    CK(cudaMemset(src, 1, big));
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        CK(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+        encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    }
+    CK(cudaFuncSetAttribute(copy_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
+    CK(cudaFuncSetAttribute(copy_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
+    // (tiled, span bytes, chunk bytes, stages, issuers)
+    struct Case { int tiled; size_t span; int chunk, stages, issuers; };
+    const Case cases[] = {
+        {0, (size_t)48 << 20, 8192, 8, 1},  {0, (size_t)48 << 20, 8192, 24, 1}, {0, (size_t)48 << 20, 16384, 4, 1},
+        {0, (size_t)48 << 20, 16384, 8, 1}, {0, (size_t)48 << 20, 16384, 12, 1}, {0, (size_t)48 << 20, 16384, 12, 2},
+        {0, (size_t)48 << 20, 32768, 2, 1}, {0, (size_t)48 << 20, 32768, 4, 1}, {0, (size_t)48 << 20, 32768, 6, 1},
+        {0, (size_t)48 << 20, 32768, 6, 2}, {0, (size_t)48 << 20, 65536, 3, 1}, {0, (size_t)16 << 20, 32768, 6, 1},
+        {0, big, 16384, 8, 1},               {0, big, 32768, 6, 1},               {0, big, 65536, 3, 1},
+        {1, (size_t)48 << 20, 16384, 4, 1}, {1, (size_t)48 << 20, 16384, 8, 1}, {1, (size_t)48 << 20, 16384, 12, 1},
+        {1, (size_t)48 << 20, 16384, 12, 2}, {1, (size_t)48 << 20, 32768, 3, 1}, {1, (size_t)48 << 20, 32768, 6, 1},
+        {1, (size_t)48 << 20, 32768, 6, 2}, {1, big, 16384, 12, 1},              {1, big, 32768, 6, 1}};
+    for (const Case &cs : cases) {
+        const size_t smem = (size_t)cs.chunk * cs.stages + 1024;
+        CUtensorMap tm;
+        memset(&tm, 0, sizeof tm);
+        const int K = 1024, rows = cs.chunk / 128;            // tiles: 64 bf16 (128 bytes) x rows
+        const int rows_total = (int)(cs.span / (K * 2));
+        if (cs.tiled) {
+            cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows_total};
+            cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+            cuuint32_t box[2] = {64, (cuuint32_t)rows};
+            cuuint32_t estr[2] = {1, 1};
+            if (encode(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, src, dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+                fprintf(stderr, "tensor map encode failed\n");
+                return 2;
             }
-            const double bytes = (double)sms * iters * chunk;
-            printf("{\"probe\": \"bulk\", \"span_bytes\": %zu, \"chunk\": %d, \"stages\": %d, \"ctas\": %d, "
-                   "\"GBps\": %.1f}\n", span, chunk, stages, sms, bytes / (best * 1e-3) / 1e9);
-            cudaEventDestroy(a);
-            cudaEventDestroy(b);
         }
+        const int iters = (int)(((size_t)8 << 30) / ((size_t)sms * cs.chunk));   // 8 GiB in all
+        cudaEvent_t a, b;
+        CK(cudaEventCreate(&a));
+        CK(cudaEventCreate(&b));
+        float best = 1e30f;
+        for (int rep = 0; rep < 3; ++rep) {
+            CK(cudaEventRecord(a));
+            if (cs.tiled)
+                copy_kernel<true><<<sms, 64, smem>>>(src, cs.span, tm, rows, rows_total, K / 64, cs.chunk, cs.stages,
+                                                     cs.issuers, iters, status);
+            else
+                copy_kernel<false><<<sms, 64, smem>>>(src, cs.span, tm, rows, rows_total, K / 64, cs.chunk, cs.stages,
+                                                      cs.issuers, iters, status);
+            CK(cudaGetLastError());
+            CK(cudaEventRecord(b));
+            CK(cudaEventSynchronize(b));
+            float ms = 0;
+            CK(cudaEventElapsedTime(&ms, a, b));
+            if (ms < best) best = ms;
+        }
+        const double bytes = (double)sms * (iters / cs.issuers * cs.issuers) * cs.chunk;
+        printf("{\"probe\": \"%s\", \"span_bytes\": %zu, \"chunk\": %d, \"stages\": %d, \"issuers\": %d, "
+               "\"ctas\": %d, \"GBps\": %.1f}\n", cs.tiled ? "tile" : "bulk", cs.span, cs.chunk, cs.stages,
+               cs.issuers, sms, bytes / (best * 1e-3) / 1e9);
+        cudaEventDestroy(a);
+        cudaEventDestroy(b);
     }
     int st = 0;
     CK(cudaMemcpy(&st, status, sizeof st, cudaMemcpyDeviceToHost));

@@ -232,11 +232,13 @@ def test_router_scores_and_dispatch_are_exact():
     np.testing.assert_array_equal(layer.region(T, "offsets", torch.int32, (w.E + 1,)).cpu().numpy(), offsets)
     np.testing.assert_array_equal(layer.region(T, "slot_of", torch.int32, (T, w.k)).cpu().numpy(), slot_expected)
     np.testing.assert_array_equal(layer.region(T, "perm_tok", torch.int32, (T * w.k,)).cpu().numpy(), perm_expected)
-    # the latent z = W_down x of every token (bf16-rounded), which the routed
-    # GEMM reads through the slot -> token map
-    z = layer.region(T, "Z", torch.bfloat16, (T, w.l)).float().cpu()
-    ref = x.double() @ W["W_down"].double().T
-    assert ((z.double() - ref).abs().max() / ref.abs().max()).item() < 1e-2
+    # the latent z = W_down x of every token (bf16-rounded) in each of its k
+    # expert-sorted slot rows, which the routed gate/up GEMM reads
+    zp = layer.region(T, "Zp", torch.bfloat16, (T * w.k, w.l)).float().cpu()
+    slots = torch.from_numpy(slot_expected.astype(np.int64))
+    ref = (x.double() @ W["W_down"].double().T)
+    got = zp[slots.reshape(-1)].reshape(T, w.k, w.l).double()
+    assert ((got - ref[:, None, :]).abs().max() / ref.abs().max()).item() < 1e-2
     layer.close()
 
 
