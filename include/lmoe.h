@@ -267,8 +267,7 @@ LMOE_API lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t 
  * region: 0 router scores r [T, E] fp32; 1 mixture weights fp32 [T, k];
  * 2 per-expert counts [E] int32; 3 expert offsets [E+1] int32;
  * 4 slot index of (t, j) [T, k] int32; 5 token of each permuted slot [T*k]
- * int32; 6 latent rows z [T, l] (0 bytes in the standard form, and when the
- * down-projection writes its rows straight into the slot rows); 7 routed
+ * int32; 6 latent rows z [T, l] (0 bytes in the standard form); 7 routed
  * hidden H [T*k, f] (slot order); 8 p-weighted expert outputs [T*k, l] (token
  * dtype); 9 [shared hidden | RMSNorm(u)] [T, 2 f_shared + l] (no RMSNorm
  * columns in the standard form); 10 device status word (int32); 11 Quantile-Balancing

@@ -52,23 +52,29 @@ namespace lmoe {
 namespace {
 
 constexpr int BN = TC_BN, BK = TC_BK;
-constexpr int THREADS = 320;   // 2 role warps + 8 epilogue warps
+// Warps: 0 and 10..12 TMA producers, 1 MMA issuer / TMEM owner, 2..9 epilogue.
+// Each thread's tensor copies go out one after another (measured on B200: one
+// issuing thread moves 16 KB tiles at about 6.4 TB/s across the chip, two
+// threads at twice that), so up to four producers share the k-steps.
+//
+// Producer q of P takes k-steps it = q (mod P) into ring slot it % S and first
+// waits for that slot's previous use to be consumed, by the parity of the
+// slot's "empty" barrier.  A parity wait is only sound while the barrier is at
+// most one phase behind, i.e. while the use before the previous one has been
+// consumed: the producer's own previous wait (k-step it - P) guaranteed the
+// consumption of it - P - S, which covers it - 2 S exactly when P <= S.  So a
+// ring of S stages runs min(NPROD, S) producers.
+constexpr int NPROD = 4;
+constexpr int THREADS = 32 * (2 + 8 + NPROD - 1);
+__device__ __forceinline__ int producer_index(int warp) { return warp == 0 ? 0 : (warp >= 10 ? warp - 9 : -1); }
 constexpr int TMEM_COLS = 2 * BN;
 constexpr long long WAIT_LIMIT_CYCLES = 4000000000ll;   // about 2 s at 2 GHz
 constexpr int MAX_E = 1024;
-// NH: 256-column halves per output tile.  NH = 1: (128 CG) x 256 tiles in two
-// double-buffered 256-column accumulators.  NH = 2 (CTA pairs): 256 x 512
-// tiles in one 512-column accumulator of two halves, each filled by its own
-// M = 256, N = 256 MMAs from the same A stage, so every operand byte a CTA
-// moves feeds a third more MMA work (48 KB per k-step for 128 x 512 outputs
-// instead of 32 KB for 128 x 256).
-template <int CG, int NH = 1> struct Tiles {
+template <int CG> struct Tiles {
     static constexpr int A_BYTES = 128 * BK * 2;                // this CTA's 128 A rows
-    static constexpr int B_HALF_BYTES = (BN / CG) * BK * 2;     // this CTA's share of one half's B rows
-    static constexpr int B_BYTES = NH * B_HALF_BYTES;
+    static constexpr int B_BYTES = (BN / CG) * BK * 2;          // this CTA's share of B rows
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TILE_M = 128 * CG;
-    static constexpr int TILE_N = BN * NH;
     // kind::f16, D fp32, A and B bf16, both K-major, M = 128 CG, N = BN
     static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                       ((uint32_t)(TILE_M >> 4) << 24);
@@ -79,14 +85,14 @@ template <int CG, int NH = 1> struct Tiles {
 // stored by TMA), and as many operand stages as fit (at most 6): the weight
 // tiles of a grouped GEMM mostly come from HBM, and the ring is what keeps
 // their loads in flight.
-template <int CG, int OB, int NH = 1> struct Cfg : Tiles<CG, NH> {
+template <int CG, int OB> struct Cfg : Tiles<CG> {
     static constexpr int EPI_CHUNK = 32 * 32 * OB;
     static constexpr int EPI_STAGING = 8 * EPI_CHUNK;
     static constexpr int TABLES = 2 * (int)sizeof(int) * (MAX_E + 1);
     static constexpr int FIXED = 1024 + EPI_STAGING + 256 + TABLES;
-    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG, NH>::STAGE_BYTES;
+    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG>::STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG, NH>::STAGE_BYTES;
+    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG>::STAGE_BYTES;
     static_assert(STAGES >= 3, "operand ring too shallow");
 };
 
@@ -376,12 +382,12 @@ struct Tile {
 
 // Grouped mode reads the expert row offsets and m-tile prefix from shared
 // memory (staged once per CTA), so decoding a tile costs no global round trip.
-template <int CG, int NH>
+template <int CG>
 __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off, const int *s_offsets, int tile)
 {
     Tile t;
     const int mt = tile / p.ntn, nt = tile % p.ntn;
-    t.n0 = nt * BN * NH;
+    t.n0 = nt * BN;
     if (p.offsets) {
         int lo = 0, hi = p.E - 1;  // last e with tile_off[e] <= mt
         while (lo < hi) {
@@ -399,12 +405,12 @@ __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off,
     return t;
 }
 
-template <int MODE, typename TO, int CG, int NH>
+template <int MODE, typename TO, int CG>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmC, const TcParams p)
 {
-    using C = Cfg<CG, (int)sizeof(TO), NH>;
+    using C = Cfg<CG, (int)sizeof(TO)>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -415,7 +421,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // bars[0..S) full, [S..2S) empty, [2S..2S+2) acc full, [2S+2..2S+4) acc empty
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
     int *abort_flag = reinterpret_cast<int *>(tmem_holder + 1);
-    int *drain_counts = abort_flag + 1;                      // [0] loads issued, [1] stages consumed
+    int *drain_counts = abort_flag + 1;   // [0, NPROD) k-steps issued by each producer, [NPROD] consumed
     int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * C::STAGE_BYTES + C::EPI_STAGING + 256);
     int *s_offsets = s_tile_off + (MAX_E + 1);                                                 // [E+1]
 
@@ -439,7 +445,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             mbar_init(acce_bar(a), 8 * CG);  // every epilogue warp of the group
         }
         *abort_flag = 0;
-        drain_counts[0] = drain_counts[1] = 0;
+        for (int i = 0; i <= NPROD; ++i) drain_counts[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&tmA);
@@ -474,18 +480,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     const int total = (p.offsets ? s_tile_off[p.E] * p.ntn : p.max_tiles) * p.ksplit;   // work items
     const int nkb_total = p.nkb * p.nterms;
+    const int pw = producer_index(warp);
+    constexpr int NP = NPROD < STAGES ? NPROD : STAGES;   // producers in use (see NPROD)
 
-    if (warp == 0) {
-        if (lane == 0) {
-            // ---------------------------------------------------- TMA producer
+    if (pw >= 0) {
+        if (lane == 0 && pw < NP) {
+            // ---------------------------------------------------- TMA producers
+            // Producer pw issues the loads of k-steps it with it % NP == pw:
+            // a thread's tensor copies go out one after another, so several
+            // issuing threads are what keeps the operand ring full.
             int it = 0;
             bool ok = true;
             for (int item = group; item < total && ok; item += ngroups) {
-                const Tile t = decode<CG, NH>(p, s_tile_off, s_offsets, item / p.ksplit);
-                const int nh = (NH == 2 && p.N - t.n0 > BN) ? 2 : 1;   // halves with columns in this tile
+                const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
                 const int split = item % p.ksplit;
                 const int kb_end = (split + 1) * nkb_total / p.ksplit;
                 for (int kb = split * nkb_total / p.ksplit; kb < kb_end; ++kb, ++it) {
+                    if (it % NP != pw) continue;
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
@@ -497,12 +508,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
                     const uint32_t fb = CG == 2 ? map_to_rank(full_bar(s), 0) : full_bar(s);
-                    if (leader) mbar_expect_tx(full_bar(s), CG * (C::A_BYTES + nh * C::B_HALF_BYTES));
+                    if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
                     tma_load_2d<CG>(sa, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
-                    for (int h = 0; h < nh; ++h)
-                        tma_load_2d<CG>(sa + C::A_BYTES + h * C::B_HALF_BYTES, &tmB, fb, kk,
-                                        (int)(t.brow + h * BN + (BN / CG) * rank + term * p.term_rows));
-                    drain_counts[0] = it + 1;
+                    tma_load_2d<CG>(sa + C::A_BYTES, &tmB, fb, kk,
+                                    (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
+                    drain_counts[pw] = it + 1;
                 }
             }
         }
@@ -510,17 +520,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (lane == 0 && leader) {
             // ---------------------------------------------------- MMA issuer (leader CTA)
             int it = 0, local = 0;
-            int uses[2] = {0, 0};       // NH = 2: tiles that have used each half so far
             bool ok = true;
             for (int item = group; item < total && ok; item += ngroups, ++local) {
-                // NH = 1: this tile's accumulator alternates; NH = 2: halves 0 and 1
-                const int acc = NH == 1 ? (local & 1) : 0;
-                const uint32_t aph = NH == 1 ? ((uint32_t)(local >> 1) & 1u) : ((uint32_t)uses[0] & 1u);
-                int nh = 1;
-                if (NH == 2) {
-                    const Tile t = decode<CG, NH>(p, s_tile_off, s_offsets, item / p.ksplit);
-                    nh = p.N - t.n0 > BN ? 2 : 1;
-                }
+                const int acc = local & 1;
+                const uint32_t aph = (uint32_t)(local >> 1) & 1u;
                 const int split = item % p.ksplit;
                 const int kb_begin = split * nkb_total / p.ksplit, kb_end = (split + 1) * nkb_total / p.ksplit;
                 if (!mbar_wait(acce_bar(acc), aph ^ 1u)) {
@@ -547,40 +550,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                     tc_fence_after();
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
-                    for (int h = 0; h < nh; ++h) {
-                        // NH = 2: the first k-step's MMAs into half 1 wait until the
-                        // epilogue has read the previous tile's half 1 (half 0's
-                        // MMAs already run meanwhile)
-                        if (NH == 2 && h == 1 && kb == kb_begin) {
-                            if (!mbar_wait(acce_bar(1), ((uint32_t)uses[1] & 1u) ^ 1u)) {
-                                atomicOr(p.status, ST_MMA);
-                                *(volatile int *)abort_flag = 1;
-                                ok = false;
-                                break;        // half 0's MMAs of this stage are committed below
-                            }
-                            tc_fence_after();
-                        }
 #pragma unroll
-                        for (int k = 0; k < BK / 16; ++k) {
-                            const uint64_t ad = sdesc_sw128(sa + 32u * k);
-                            const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + h * C::B_HALF_BYTES + 32u * k);
-                            umma_bf16<CG>(dt + (uint32_t)(h * BN), ad, bd, (kb > kb_begin || k > 0) ? 1u : 0u);
-                        }
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = sdesc_sw128(sa + 32u * k);
+                        const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + 32u * k);
+                        umma_bf16<CG>(dt, ad, bd, (kb > kb_begin || k > 0) ? 1u : 0u);
                     }
                     umma_commit<CG>(empty_bar(s));
-                    drain_counts[1] = it + 1;
-                    if (!ok) break;
+                    drain_counts[NPROD] = it + 1;
                 }
-                if (ok) {
-                    if (NH == 2) {
-                        for (int h = 0; h < nh; ++h) {
-                            umma_commit<CG>(accf_bar(h));
-                            ++uses[h];
-                        }
-                    } else {
-                        umma_commit<CG>(accf_bar(acc));
-                    }
-                }
+                if (ok) umma_commit<CG>(accf_bar(acc));
             }
         }
     } else {
@@ -591,14 +570,24 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
         const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * C::EPI_CHUNK;
         int local = 0;
-        int uses[2] = {0, 0};           // NH = 2: tiles that have used each half so far
-        bool stop = false;
-        for (int item = group; item < total && !stop; item += ngroups, ++local) {
-            const Tile t = decode<CG, NH>(p, s_tile_off, s_offsets, item / p.ksplit);
-            const int nh = (NH == 2 && p.N - t.n0 > BN) ? 2 : 1;
+        for (int item = group; item < total; item += ngroups, ++local) {
+            const int acc = local & 1;
+            const uint32_t aph = (uint32_t)(local >> 1) & 1u;
+            const bool got = mbar_wait(accf_bar(acc), aph);
+            if (!got || *(volatile int *)abort_flag) {
+                if (lane == 0) {
+                    atomicOr(p.status, ST_EPILOGUE);
+                    *(volatile int *)abort_flag = 1;
+                }
+                break;
+            }
+            tc_fence_after();
+            const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
             const int64_t slab = (int64_t)(item % p.ksplit) * p.split_rows;   // 0 unless split K
             const int64_t row = t.row0 + 128 * rank + 32 * q + lane;
             const bool valid = row < t.row_end;
+            const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
+            float v[32], u[32];
             // Emit 32 output columns [col, col + n) of this warp's 32 rows: whole
             // chunks go through the staging buffer and one TMA store; chunks that
             // straddle an expert's last row (or a ragged column edge) store per lane.
@@ -618,127 +607,78 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     store_n((TO *)p.epi.out + (slab + row) * p.epi.ldo + col, x, n);
                 }
             };
-            // one 256-column accumulator at a time: NH = 1 the tile's (alternating
-            // between two), NH = 2 each half of the tile in turn
-            for (int hu = 0; hu < nh; ++hu) {
-                const int acc = NH == 1 ? (local & 1) : hu;
-                const uint32_t aph = NH == 1 ? ((uint32_t)(local >> 1) & 1u) : ((uint32_t)uses[hu] & 1u);
-                const bool got = mbar_wait(accf_bar(acc), aph);
-                if (!got || *(volatile int *)abort_flag) {
-                    if (lane == 0) {
-                        atomicOr(p.status, ST_EPILOGUE);
-                        *(volatile int *)abort_flag = 1;
-                    }
-                    stop = true;
-                    break;
+            if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
+                const int half = BN / 2;
+#pragma unroll 1
+                for (int c = 32 * hset; c < half; c += 64) {
+                    __syncwarp();
+                    tmem_ld32_pair(tq + c, tq + half + c, v, u);   // gate and up columns, one wait
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
+                                                                                       p.epi.up_cap);
+                    emit(v, t.n0 / 2 + c, 32);
                 }
-                tc_fence_after();
-                const int n0 = t.n0 + (NH == 2 ? hu * BN : 0);      // first GEMM column of this accumulator
-                const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
-                float v[32], u[32];
-                if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
-                    const int half = BN / 2;
+            } else {
 #pragma unroll 1
-                    for (int c = 32 * hset; c < half; c += 64) {
-                        __syncwarp();
-                        tmem_ld32_pair(tq + c, tq + half + c, v, u);   // gate and up columns, one wait
+                for (int c = 32 * hset; c < BN; c += 128) {
+                    __syncwarp();
+                    tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // warp-collective: every lane
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
-                                                                                           p.epi.up_cap);
-                        emit(v, n0 / 2 + c, 32);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int c = 32 * hset; c < BN; c += 128) {
-                        __syncwarp();
-                        tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // warp-collective: every lane
+                    for (int part = 0; part < 2; ++part) {
+                        float *x = part ? u : v;
+                        const int col = t.n0 + c + 64 * part;
+                        int n = p.N - col;
+                        if (n > 32) n = 32;
+                        if (n <= 0) continue;             // uniform across the warp
+                        if (MODE == EPI_SIGMOID) {
 #pragma unroll
-                        for (int part = 0; part < 2; ++part) {
-                            float *x = part ? u : v;
-                            const int col = n0 + c + 64 * part;
-                            int n = p.N - col;
-                            if (n > 32) n = 32;
-                            if (n <= 0) continue;             // uniform across the warp
-                            if (MODE == EPI_SIGMOID) {
+                            for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
+                        } else if (MODE == EPI_STORE && sizeof(TO) == 2) {
+                            if (p.epi.residual && valid) {   // standard MoE: y = shared + u
+                                const bf16 *res = (const bf16 *)p.epi.residual + (slab + row) * p.epi.ldr + col;
+                                if (n == 32 && ((uintptr_t)res & 15u) == 0) {
 #pragma unroll
-                                for (int i = 0; i < 32; ++i) x[i] = sigmoidf_(x[i]);
-                            } else if (MODE == EPI_STORE && sizeof(TO) == 2) {
-                                if (p.epi.residual && valid) {   // standard MoE: y = shared + u
-                                    const bf16 *res = (const bf16 *)p.epi.residual + (slab + row) * p.epi.ldr + col;
-                                    if (n == 32 && ((uintptr_t)res & 15u) == 0) {
+                                    for (int q8 = 0; q8 < 4; ++q8) {   // four 16-byte loads
+                                        const uint4 w = *reinterpret_cast<const uint4 *>(res + 8 * q8);
+                                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                                        for (int q8 = 0; q8 < 4; ++q8) {   // four 16-byte loads
-                                            const uint4 w = *reinterpret_cast<const uint4 *>(res + 8 * q8);
-                                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                                            for (int i = 0; i < 4; ++i) {
-                                                const __nv_bfloat162 h2 =
-                                                    *reinterpret_cast<const __nv_bfloat162 *>(&ws[i]);
-                                                x[8 * q8 + 2 * i] += __low2float(h2);
-                                                x[8 * q8 + 2 * i + 1] += __high2float(h2);
-                                            }
+                                        for (int i = 0; i < 4; ++i) {
+                                            const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162 *>(&ws[i]);
+                                            x[8 * q8 + 2 * i] += __low2float(h2);
+                                            x[8 * q8 + 2 * i + 1] += __high2float(h2);
                                         }
-                                    } else {
-#pragma unroll
-                                        for (int i = 0; i < 32; ++i)
-                                            if (i < n) x[i] += __bfloat162float(res[i]);
                                     }
+                                } else {
+#pragma unroll
+                                    for (int i = 0; i < 32; ++i)
+                                        if (i < n) x[i] += __bfloat162float(res[i]);
                                 }
-                            } else if (MODE == EPI_COMBINE) {
-                                const float w = valid ? p.epi.row_w[row] : 0.f;   // bf16 rows: p-weighted here
-#pragma unroll
-                                for (int i = 0; i < 32; ++i) x[i] *= w;
                             }
-                            if (MODE == EPI_SCATTER) {
-                                // the token's latent row goes straight to its k slot rows
-                                if (valid) {
-                                    const int32_t *so = p.epi.slot_of + row * p.epi.kslots;
-                                    if (n == 32) {
-                                        uint4 w4[4];
+                        } else if (MODE == EPI_COMBINE) {
+                            const float w = valid ? p.epi.row_w[row] : 0.f;   // bf16 rows: p-weighted here
 #pragma unroll
-                                        for (int q4 = 0; q4 < 4; ++q4) {
-                                            uint32_t w[4];
-#pragma unroll
-                                            for (int i = 0; i < 4; ++i) {
-                                                const __nv_bfloat162 pr =
-                                                    __floats2bfloat162_rn(x[q4 * 8 + 2 * i], x[q4 * 8 + 2 * i + 1]);
-                                                w[i] = *reinterpret_cast<const uint32_t *>(&pr);
-                                            }
-                                            w4[q4] = make_uint4(w[0], w[1], w[2], w[3]);
-                                        }
-                                        for (int j = 0; j < p.epi.kslots; ++j) {
-                                            uint4 *d4 = reinterpret_cast<uint4 *>((bf16 *)p.epi.out +
-                                                                                 (int64_t)so[j] * p.epi.ldo + col);
-#pragma unroll
-                                            for (int q4 = 0; q4 < 4; ++q4) d4[q4] = w4[q4];
-                                        }
-                                    } else {
-                                        for (int j = 0; j < p.epi.kslots; ++j)
-                                            store_n((bf16 *)p.epi.out + (int64_t)so[j] * p.epi.ldo + col, x, n);
-                                    }
-                                }
-                            } else {
-                                emit(x, col, n);
-                            }
+                            for (int i = 0; i < 32; ++i) x[i] *= w;
                         }
+                        emit(x, col, n);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(CG == 2 ? map_to_rank(acce_bar(acc), 0) : acce_bar(acc));
-                if (NH == 2) ++uses[hu];
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(CG == 2 ? map_to_rank(acce_bar(acc), 0) : acce_bar(acc));
         }
         if (lane == 0) bulk_wait_all();             // this warp's TMA stores are complete
     }
 
     __syncthreads();
     if (*(volatile int *)abort_flag && threadIdx.x == 0 && leader) {
-        // Drain: loads issued but never consumed, then the MMAs behind the last commit.
-        const int issued = drain_counts[0], consumed = drain_counts[1];
+        // Drain: loads issued but never consumed (each producer's own k-steps),
+        // then the MMAs behind the last commit.
+        const int consumed = drain_counts[NPROD];
         bool ok = true;
-        for (int i = consumed; i < issued; ++i)
-            ok &= mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
+        for (int q = 0; q < NP; ++q)
+            for (int i = consumed; i < drain_counts[q]; ++i)
+                if (i % NP == q) ok &= mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
         if (consumed > 0) {
             const int i = consumed - 1;
             ok &= mbar_wait(empty_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
@@ -795,7 +735,7 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, 
 // CTA pairs, how many pairs fit at once), done on first use and cached.
 constexpr int MAX_DEVICES = 64;
 
-template <int MODE, typename TO, int CG, int NH>
+template <int MODE, typename TO, int CG>
 cudaError_t group_capacity(int *max_groups)
 {
     static std::atomic<int> cached[MAX_DEVICES];   // 0 = not yet known
@@ -806,15 +746,15 @@ cudaError_t group_capacity(int *max_groups)
         *max_groups = cached[dev];
         return cudaSuccess;
     }
-    auto kern = tc_gemm_kernel<MODE, TO, CG, NH>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG, (int)sizeof(TO), NH>::SMEM);
+    auto kern = tc_gemm_kernel<MODE, TO, CG>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<CG, (int)sizeof(TO)>::SMEM);
     if (e != cudaSuccess) return e;
     int groups = g_num_sms / CG;
     if (CG > 1) {
         cudaLaunchConfig_t q = {};
         q.gridDim = dim3(g_num_sms / CG * CG);
         q.blockDim = dim3(THREADS);
-        q.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO), NH>::SMEM;
+        q.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO)>::SMEM;
         cudaLaunchAttribute qa[1];
         qa[0].id = cudaLaunchAttributeClusterDimension;
         qa[0].val.clusterDim.x = CG;
@@ -832,19 +772,19 @@ cudaError_t group_capacity(int *max_groups)
 }
 
 // Persistent grid: min(work items, CTA groups that can be resident at once).
-template <int MODE, typename TO, int CG, int NH>
+template <int MODE, typename TO, int CG>
 cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const TcParams &p, cudaStream_t s)
 {
-    auto kern = tc_gemm_kernel<MODE, TO, CG, NH>;
+    auto kern = tc_gemm_kernel<MODE, TO, CG>;
     int max_groups = 0;
-    const cudaError_t e = group_capacity<MODE, TO, CG, NH>(&max_groups);
+    const cudaError_t e = group_capacity<MODE, TO, CG>(&max_groups);
     if (e != cudaSuccess) return e;
     const int items = p.max_tiles * p.ksplit;
     const int groups = items < max_groups ? items : max_groups;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(groups * CG);
     lc.blockDim = dim3(THREADS);
-    lc.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO), NH>::SMEM;
+    lc.dynamicSmemBytes = Cfg<CG, (int)sizeof(TO)>::SMEM;
     lc.stream = s;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -858,11 +798,10 @@ cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap
     return cudaLaunchKernelEx(&lc, kern, a, b, c, p);
 }
 
-template <int CG, int NH>
+template <int CG>
 cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t term_rows, int64_t b_rows_total,
                 int ksplit, int32_t *status, cudaStream_t s)
 {
-    static_assert(NH == 1 || CG == 2, "512-column tiles are for CTA pairs");
     if (!g_encode) return cudaErrorInitializationError;
     if (g.K % BK) return cudaErrorInvalidValue;
     if (((uintptr_t)g.A | (uintptr_t)g.B) & 15u) return cudaErrorMisalignedAddress;
@@ -874,22 +813,19 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.nkb = g.K / BK;
     p.nterms = nterms;
     p.term_rows = term_rows;
-    // GLU: N = 2F, F % (BN/2) == 0, so every 256-column half holds whole gate/up pairs
-    p.ntn = (g.N + BN * NH - 1) / (BN * NH);
+    p.ntn = (mode == EPI_GLU) ? g.N / BN : (g.N + BN - 1) / BN;   // GLU: N = 2F, F % (BN/2) == 0
     p.group_rows = g.offsets ? g.b_group_stride / g.ldb : 0;
     p.offsets = g.offsets;
     p.tile_off = g.tile_off;
     p.E = g.E;
-    const int mtiles = g.offsets ? max_mtiles : (g.M + Tiles<CG, NH>::TILE_M - 1) / Tiles<CG, NH>::TILE_M;
+    const int mtiles = g.offsets ? max_mtiles : (g.M + Tiles<CG>::TILE_M - 1) / Tiles<CG>::TILE_M;
     p.max_tiles = mtiles * p.ntn;
     p.ksplit = ksplit < 1 ? 1 : ksplit;
     p.split_rows = g.M;
     if (p.ksplit > 1 && (g.offsets || (mode != EPI_STORE_F32 && mode != EPI_SIGMOID_PARTIAL) ||
                          p.ksplit > p.nkb * nterms))
         return cudaErrorInvalidValue;
-    if (NH == 2 && (p.ksplit > 1 || nterms > 1 || mode == EPI_SIGMOID || mode == EPI_STORE_F32 ||
-                    mode == EPI_SIGMOID_PARTIAL))
-        return cudaErrorInvalidValue;
+
     p.epi = g.epi;
     p.status = status;
     p.stall_test = g_stall_next.exchange(0);
@@ -905,25 +841,14 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     memset(&tc, 0, sizeof tc);
     p.tma_store = make_out_map(&tc, g.epi.out, out_f32, (uint64_t)p.out_cols, (uint64_t)g.M * p.ksplit,
                                (uint64_t)g.epi.ldo * (out_f32 ? 4 : 2)) ? 1 : 0;
-    if (NH == 2) {
-        switch (mode) {
-        case EPI_GLU:
-            if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG, NH>(ta, tb, tc, p, s);
-            return launch<EPI_GLU, bf16, CG, NH>(ta, tb, tc, p, s);
-        case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG, NH>(ta, tb, tc, p, s);
-        case EPI_STORE: return launch<EPI_STORE, bf16, CG, NH>(ta, tb, tc, p, s);
-        default: return cudaErrorInvalidValue;
-        }
-    }
     switch (mode) {
-    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG, 1>(ta, tb, tc, p, s);
+    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG>(ta, tb, tc, p, s);
     case EPI_GLU:
-        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG, 1>(ta, tb, tc, p, s);
-        return launch<EPI_GLU, bf16, CG, 1>(ta, tb, tc, p, s);
-    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG, 1>(ta, tb, tc, p, s);
-    case EPI_STORE: return launch<EPI_STORE, bf16, CG, 1>(ta, tb, tc, p, s);
-    case EPI_SCATTER: return launch<EPI_SCATTER, bf16, CG, 1>(ta, tb, tc, p, s);
-    case EPI_STORE_F32: return launch<EPI_STORE, float, CG, 1>(ta, tb, tc, p, s);
+        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG>(ta, tb, tc, p, s);
+        return launch<EPI_GLU, bf16, CG>(ta, tb, tc, p, s);
+    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG>(ta, tb, tc, p, s);
+    case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tb, tc, p, s);
+    case EPI_STORE_F32: return launch<EPI_STORE, float, CG>(ta, tb, tc, p, s);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -997,7 +922,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         }
         mbar_init(accf, 1);
         *abort_flag = 0;
-        drain_counts[0] = drain_counts[1] = 0;
+        for (int i = 0; i <= NPROD; ++i) drain_counts[i] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&tmA);
@@ -1015,10 +940,13 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
-    if (warp == 0) {
-        if (lane == 0) {   // ------------------------------------------------ TMA producer
+    const int pw = producer_index(warp);
+    const int NP = NPROD < STAGES ? NPROD : STAGES;   // producers in use (see NPROD)
+    if (pw >= 0) {
+        if (lane == 0 && pw < NP) {   // ------------------------------------ TMA producers (k-step it % NP)
             int it = 0;
             for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+                if (it % NP != pw) continue;
                 const int s = it % STAGES;
                 const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                 if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
@@ -1033,7 +961,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 for (int h = 0; h < p.halves; ++h)
                     tma_load_2d<1>(sa + a_bytes + h * bh_bytes, &tmB, full_bar(s), kk,
                                    term * p.E + h * p.n_half);
-                drain_counts[0] = it + 1;
+                drain_counts[pw] = it + 1;
             }
         }
     } else if (warp == 1) {
@@ -1071,11 +999,11 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     }
                 }
                 umma_commit<1>(empty_bar(s));
-                drain_counts[1] = it + 1;
+                drain_counts[NPROD] = it + 1;
             }
             if (ok) umma_commit<1>(accf);
         }
-    } else {
+    } else if (warp <= 9) {
         // ---------------------------------------------------------------- epilogue warps 2..9
         const int q = warp & 3, hset = (warp - 2) >> 2;
         const bool got = mbar_wait(accf, 0u);
@@ -1175,11 +1103,13 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 
     __syncthreads();
     if (*(volatile int *)abort_flag && threadIdx.x == 0) {
-        // Drain: loads issued but never consumed, then the MMAs behind the last commit.
-        const int issued = drain_counts[0], consumed = drain_counts[1];
+        // Drain: loads issued but never consumed (each producer's own k-steps),
+        // then the MMAs behind the last commit.
+        const int consumed = drain_counts[NPROD];
         bool ok = true;
-        for (int i = consumed; i < issued; ++i)
-            ok &= mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
+        for (int q = 0; q < NP; ++q)
+            for (int i = consumed; i < drain_counts[q]; ++i)
+                if (i % NP == q) ok &= mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
         if (consumed > 0) {
             const int i = consumed - 1;
             ok &= mbar_wait(empty_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u);
@@ -1269,17 +1199,8 @@ cudaError_t tc_gemm(int mode, const GemmArgs &g, int max_mtiles, int cg, int32_t
 {
     // B rows: dense N; grouped E * (rows per expert)
     const int64_t b_rows = g.offsets ? (int64_t)g.E * (g.b_group_stride / g.ldb) : g.N;
-    if (cg == 2 && ksplit <= 1 && mode != EPI_SIGMOID && mode != EPI_STORE_F32 && mode != EPI_SCATTER) {
-        // 256 x 512 tiles where they still make many waves of CTA pairs (a
-        // handful of waves would lose more to the last one's idle pairs than
-        // the wider tile saves)
-        const int64_t mt = g.offsets ? (int64_t)max_mtiles : ((int64_t)g.M + 255) / 256;
-        const int64_t wide_tiles = mt * (((int64_t)g.N + 2 * BN - 1) / (2 * BN));
-        const int pairs = (g_num_sms > 0 ? g_num_sms : 148) / 2;
-        if (wide_tiles >= 6 * (int64_t)pairs) return run<2, 2>(mode, g, max_mtiles, 1, 0, b_rows, 1, status, s);
-    }
-    if (cg == 2) return run<2, 1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
-    return run<1, 1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
+    if (cg == 2) return run<2>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
+    return run<1>(mode, g, max_mtiles, 1, 0, b_rows, ksplit, status, s);
 }
 
 int tc_num_sms() { return g_num_sms; }
@@ -1292,8 +1213,8 @@ cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int cg, int32_t *
     r.B = Wr3;
     r.ldb = g.K;
     const int mode = ksplit > 1 ? EPI_SIGMOID_PARTIAL : EPI_SIGMOID;
-    if (cg == 2) return run<2, 1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
-    return run<1, 1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+    if (cg == 2) return run<2>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
+    return run<1>(mode, r, 0, 3, g.N, 3 * (int64_t)g.N, ksplit, status, s);
 }
 
 }  // namespace lmoe

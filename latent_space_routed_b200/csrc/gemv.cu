@@ -8,20 +8,24 @@
 // ("at low latency and small batch size, MoE is bound by the memory bandwidth
 // of loading weights").
 //
-// One warp owns a block of RB = 8 weight rows at a time (for the gate: 4 gate
-// rows and the matching 4 up rows of the interleaved layout) and runs over
-// the whole of K: each lane issues 16-byte non-allocating loads of its 8 rows
-// two steps ahead (256 bytes in flight per lane) and multiplies them with the
-// same columns of each input row (x is small and stays in L1).  Lane partial
-// sums are added with a fixed butterfly, so the result does not depend on
-// timing.  A persistent grid of 4-warp blocks hands row blocks out warp by
-// warp, so every SM streams until the work runs out.
+// Dense (one matrix, input rows 0..T-1): a block of 8 warps owns 4 weight rows
+// (for the gate: 2 gate rows and the matching 2 up rows of the interleaved
+// layout); its warps split K into interleaved 512-byte pieces, each lane
+// keeping 16 loads of 16 bytes in flight, and the warps' sums are added in
+// warp order.  Many small blocks keep every SM streaming even for the 26 MB
+// down-projection (N = 1792 rows).
 //
-// Dense mode: one matrix, input rows 0..T-1, output row t.
-// Grouped mode (the routed experts): work items are (touched expert, row
-// block); the expert's slot rows [offsets[e], offsets[e+1]) are its input rows
-// (through the slot -> token map amap when given, e.g. z rows of the tokens)
+// Grouped (the routed experts): one warp owns a block of RB = 8 weight rows
+// at a time (4 gate + 4 up rows for the gate) of one touched expert and runs
+// over the whole of K, 16 loads of 16 bytes in flight per lane; a persistent
+// grid of 4-warp blocks gives each warp a contiguous run of (touched expert,
+// row block) items.  The expert's slot rows [offsets[e], offsets[e+1]) are its input rows
+// (through the slot -> token map amap when given: the z rows of the tokens)
 // and its output rows; W is the expert's slice.
+//
+// Either way each weight vector meets the same columns of every input row (x
+// is small and stays in L1), lane sums are added with a fixed butterfly and
+// nothing depends on timing.
 #include "lmoe_internal.cuh"
 
 namespace lmoe {
@@ -50,6 +54,90 @@ __device__ __forceinline__ float dot8(const uint4 &w, const uint4 &x, float acc)
         acc = fmaf(a.y, b.y, acc);
     }
     return acc;
+}
+
+constexpr int DV_ROWS = 4;       // dense: weight rows per block
+constexpr int DV_WARPS = 8;      // dense: warps per block (split K)
+
+template <int TT, int MODE>
+__global__ void __launch_bounds__(DV_WARPS * 32)
+dense_gemv_kernel(const bf16 *__restrict__ x, int64_t ldx, int T, int K, const bf16 *__restrict__ W, int N, EpiArgs e)
+{
+    __shared__ float part[DV_WARPS][TT][DV_ROWS];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    griddep_wait();
+    griddep_launch_dependents();
+    int64_t rows[DV_ROWS];
+    int64_t out0;
+    if (MODE == EPI_GLU) {
+        // outputs j0, j0 + 1: gate rows (j / ib) 2 ib + j % ib, up rows ib after them
+        const int64_t j0 = (int64_t)blockIdx.x * 2;
+        const int64_t g = (j0 / e.ib) * 2 * e.ib + (j0 % e.ib);
+        rows[0] = g;
+        rows[1] = g + 1;
+        rows[2] = g + e.ib;
+        rows[3] = g + e.ib + 1;
+        out0 = j0;
+    } else {
+        out0 = (int64_t)blockIdx.x * DV_ROWS;
+#pragma unroll
+        for (int r = 0; r < DV_ROWS; ++r) rows[r] = out0 + r < N ? out0 + r : N - 1;   // clamped rows are dropped
+    }
+    float acc[TT][DV_ROWS];
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+        for (int r = 0; r < DV_ROWS; ++r) acc[t][r] = 0.f;
+    const int nv = K / 8;   // 16-byte vectors per row
+#pragma unroll 4
+    for (int c = warp * 32 + lane; c < nv; c += DV_WARPS * 32) {
+        uint4 wv[DV_ROWS];
+#pragma unroll
+        for (int r = 0; r < DV_ROWS; ++r) wv[r] = ld_stream(W + rows[r] * K + (int64_t)c * 8);
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            if (t < T) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + (int64_t)t * ldx) + c);
+#pragma unroll
+                for (int r = 0; r < DV_ROWS; ++r) acc[t][r] = dot8(wv[r], xv, acc[t][r]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+#pragma unroll
+        for (int r = 0; r < DV_ROWS; ++r)
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc[t][r] += __shfl_xor_sync(0xffffffffu, acc[t][r], off);
+    if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < TT; ++t)
+#pragma unroll
+            for (int r = 0; r < DV_ROWS; ++r) part[warp][t][r] = acc[t][r];
+    }
+    __syncthreads();
+    // thread (t, r) adds the warps' sums in warp order and writes its output
+    const int t = threadIdx.x / DV_ROWS, r = threadIdx.x % DV_ROWS;
+    if (t >= TT || t >= T) return;
+    bf16 *out = (bf16 *)e.out;
+    if (MODE == EPI_GLU) {
+        if (r >= 2) return;
+        float gsum = 0.f, usum = 0.f;
+#pragma unroll
+        for (int w = 0; w < DV_WARPS; ++w) {
+            gsum += part[w][t][r];
+            usum += part[w][t][r + 2];
+        }
+        out[(int64_t)t * e.ldo + out0 + r] = __float2bfloat16_rn(glu_act(e.act, gsum, usum, e.gate_cap, e.up_cap));
+    } else {
+        const int64_t n = out0 + r;
+        if (n >= N) return;
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < DV_WARPS; ++w) v += part[w][t][r];
+        if (e.residual) v += __bfloat162float(((const bf16 *)e.residual)[(int64_t)t * e.ldr + n]);
+        out[(int64_t)t * e.ldo + n] = __float2bfloat16_rn(v);
+    }
 }
 
 struct GemvParams {
@@ -101,25 +189,33 @@ stream_gemv_kernel(const GemvParams p)
     const int groups = p.offsets ? *p.n_touched : 1;
     const int items = groups * nrb;
     const int nv = p.K / 8;   // 16-byte vectors per row
-    for (int item = gw; item < items; item += total_warps) {
+    // each warp takes a contiguous run of items: consecutive row blocks of the
+    // same expert, whose rows are contiguous in memory and whose expert, slot
+    // rows and input rows are looked up once per expert, not per item
+    const int per = (items + total_warps - 1) / total_warps;
+    const int i_end = min(items, (gw + 1) * per);
+    int cur = -1, s0 = 0, cnt = p.T;
+    const bf16 *W = p.W;
+    const bf16 *xr[TT];
+    for (int item = gw * per; item < i_end; ++item) {
         const int grp = item / nrb, rb = item % nrb;
         int64_t rows[RB];
         int col0;
         item_rows<MODE>(p, rb, rows, &col0);
-        const bf16 *W = p.W;
-        int s0 = 0, cnt = p.T;
-        if (p.offsets) {
-            const int e = p.touched[grp];
-            W += (int64_t)e * p.w_group_stride;
-            s0 = p.offsets[e];
-            cnt = p.offsets[e + 1] - s0;
-        }
-        const bf16 *xr[TT];
+        if (grp != cur) {
+            cur = grp;
+            if (p.offsets) {
+                const int e = p.touched[grp];
+                W = p.W + (int64_t)e * p.w_group_stride;
+                s0 = p.offsets[e];
+                cnt = p.offsets[e + 1] - s0;
+            }
 #pragma unroll
-        for (int t = 0; t < TT; ++t) {
-            const int s = s0 + (t < cnt ? t : 0);
-            const int64_t src = p.amap ? (int64_t)p.amap[s] : (int64_t)s;
-            xr[t] = p.x + src * p.ldx;
+            for (int t = 0; t < TT; ++t) {
+                const int s = s0 + (t < cnt ? t : 0);
+                const int64_t src = p.amap ? (int64_t)p.amap[s] : (int64_t)s;
+                xr[t] = p.x + src * p.ldx;
+            }
         }
         float acc[TT][RB];
 #pragma unroll
@@ -203,23 +299,31 @@ cudaError_t dispatch_tt(int tt, int mode, const GemvParams &p, int max_items, cu
 
 }  // namespace
 
+namespace {
+
+template <int TT>
+cudaError_t run_dense(int mode, const GemmArgs &g, cudaStream_t s)
+{
+    const bf16 *x = (const bf16 *)g.A, *W = (const bf16 *)g.B;
+    if (mode == EPI_GLU)
+        return launch_pdl(dense_gemv_kernel<TT, EPI_GLU>, dim3((unsigned)(g.N / 4)), dim3(DV_WARPS * 32), 0, s, x,
+                          g.lda, g.M, g.K, W, g.N, g.epi);
+    return launch_pdl(dense_gemv_kernel<TT, EPI_STORE>, dim3((unsigned)((g.N + DV_ROWS - 1) / DV_ROWS)),
+                      dim3(DV_WARPS * 32), 0, s, x, g.lda, g.M, g.K, W, g.N, g.epi);
+}
+
+}  // namespace
+
 cudaError_t launch_gemv(int mode, const GemmArgs &g, cudaStream_t s)
 {
     if (g.M < 1 || g.M > GEMV_MAX_T) return cudaErrorInvalidValue;
     if (mode != EPI_STORE && mode != EPI_GLU) return cudaErrorInvalidValue;
     if (g.K % 8 || g.lda % 8 || g.ldb != g.K) return cudaErrorInvalidValue;
-    if (mode == EPI_GLU && (g.N % RB || g.epi.ib % (RB / 2))) return cudaErrorInvalidValue;
+    if (mode == EPI_GLU && (g.N % 4 || g.epi.ib % 2)) return cudaErrorInvalidValue;
     if (((uintptr_t)g.A | (uintptr_t)g.B) & 15u) return cudaErrorMisalignedAddress;
-    GemvParams p = {};
-    p.x = (const bf16 *)g.A;
-    p.ldx = g.lda;
-    p.W = (const bf16 *)g.B;
-    p.K = g.K;
-    p.N = g.N;
-    p.T = g.M;
-    p.epi = g.epi;
-    const int nrb = mode == EPI_GLU ? g.N / RB : (g.N + RB - 1) / RB;
-    return dispatch_tt(g.M, mode, p, nrb, s);
+    if (g.M <= 1) return run_dense<1>(mode, g, s);
+    if (g.M <= 2) return run_dense<2>(mode, g, s);
+    return run_dense<4>(mode, g, s);
 }
 
 cudaError_t launch_gemv_grouped(int mode, const GemmArgs &g, const int32_t *touched, const int32_t *n_touched,

@@ -7,9 +7,8 @@
 //   2 top-k            sel, p (fp32 and token dtype), per-block expert counts
 //   3 scan             counts, offsets, per-block bases, m-tile prefix
 //   4 dispatch         slot_of[t, j], token and weight of every slot row
-//   5 down GEMM        z = x W_down^T, written to the token's k slot rows of
-//                      Zp (one tensor-core GEMM), or to z [T, l] (split-K, GEMV)
-//   6 permute          Zp[m] = z[token of slot m] [S, l] (only with z [T, l])
+//   5 down GEMM        z = x W_down^T                           [T, l]
+//   6 permute          Zp[m] = z[token of slot m]               [S, l]
 //   7 gate/up GEMM     per expert: h = act(G z, U z)            [S, f]
 //   8 down GEMM        per expert: Y = p * (h D^T)              [S, l] token dtype
 //   9 combine+norm     u = sum_j Y[slot_of[t, j]], n = RMSNorm(u)
@@ -178,14 +177,6 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     return sp;
 }
 
-// The down-projection writes z straight into the token's k slot rows (no z
-// buffer, no permute) when it is one tensor-core GEMM: it then runs after the
-// dispatch, on the caller's stream.
-bool scatter_down(const lmoe_handle *h, int64_t T)
-{
-    return h->tc && !h->cfg.standard && !gemv_experts(h, T) && plan_splits(h, T).down <= 1;
-}
-
 // The two-stream order: tensor-core path and no stage events (those time the
 // stages one after another on one stream).
 bool use_side_stream(const lmoe_handle *h) { return h->tc && h->side && !h->stage_events; }
@@ -228,9 +219,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.slot_of = take(sizeof(int32_t) * S);
     L.perm_tok = take(sizeof(int32_t) * S);
     L.perm_w = take(sizeof(float) * S);
-    // z rows: none in the standard form (which permutes x itself) or when the
-    // down-projection writes the slot rows directly
-    L.z = take((c.standard || scatter_down(h, T)) ? 0 : h->tb * T * c.l);
+    L.z = take(c.standard ? 0 : h->tb * T * c.l);   // the standard form permutes x itself
     L.Zp = take(h->tb * S * c.l);
     L.H = take(h->tb * S * c.f);
     L.Yp = take(h->tb * S * c.l);
@@ -425,7 +414,7 @@ lmoe_status lmoe_workspace_region(const lmoe_handle *h, int64_t T, int32_t regio
     case 3: *offset = L.offsets; *bytes = sizeof(int32_t) * (c.E + 1); break;
     case 4: *offset = L.slot_of; *bytes = sizeof(int32_t) * S; break;
     case 5: *offset = L.perm_tok; *bytes = sizeof(int32_t) * S; break;
-    case 6: *offset = L.z; *bytes = (c.standard || scatter_down(h, T)) ? 0 : h->tb * T * c.l; break;
+    case 6: *offset = L.z; *bytes = c.standard ? 0 : h->tb * T * c.l; break;
     case 7: *offset = L.H; *bytes = h->tb * S * c.f; break;
     case 8: *offset = L.Yp; *bytes = h->tb * S * c.l; break;
     case 9: *offset = L.HS; *bytes = h->tb * T * (2 * (int64_t)c.f_shared + c.l); break;
@@ -477,8 +466,7 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
     const lmoe_config &c = h->cfg;
     const SplitPlan sp = plan_splits(h, T);
     *launches = 11 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1) -
-                (small_route(h, T) ? 3 : 0) - (gemv_experts(h, T) ? 1 : 0) - (sp.fused_router ? 1 : 0) -
-                (scatter_down(h, T) ? 1 : 0);
+                (small_route(h, T) ? 3 : 0) - (gemv_experts(h, T) ? 1 : 0) - (sp.fused_router ? 1 : 0);
     return LMOE_OK;
 }
 
@@ -586,7 +574,6 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     const bool small = small_route(h, T);
     const bool gemv_routed = gemv_experts(h, T);
     const bool fused_router = sp.fused_router;
-    const bool scatter = scatter_down(h, T);
     const bool router_partial = h->tc && !small && !fused_router && sp.router > 1;
 
     // ---- the stages, each launched on stream `q`
@@ -679,22 +666,13 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     };
     auto st_down = [&](cudaStream_t q) -> lmoe_status {
         if (c.standard) return LMOE_OK;   // experts read x itself
-        if (scatter) {                    // z rows straight to the slot rows: Zp[slot_of[t, j]] = z[t]
-            GemmArgs g = gd;
-            g.epi.out = Zp;
-            g.epi.ldo = c.l;
-            g.epi.slot_of = slot_of;
-            g.epi.kslots = c.k;
-            LMOE_CUDA(tc_gemm(EPI_SCATTER, g, 0, cg_dense, status, q));
-            return LMOE_OK;
-        }
         if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_STORE, gd, q));
         else if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gd, sp.down, partial_side, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gd, 0, q));
         return LMOE_OK;
     };
     auto st_permute = [&](cudaStream_t q) -> lmoe_status {
-        if (gemv_routed || scatter) return LMOE_OK;   // z read through the slot map, or already scattered
+        if (gemv_routed) return LMOE_OK;   // the routed GEMVs read z through the slot -> token map
         LMOE_CUDA(launch_permute_rows(c.standard ? x : z, perm_tok, Zp, S, c.l, (int)h->tb, q));
         return LMOE_OK;
     };
@@ -761,26 +739,25 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         return LMOE_OK;
     }
 
-    // Two streams: the shared experts' gate/up GEMM needs only x, so it runs on
-    // the handle's side stream while the caller's stream does the router and
-    // the latency-bound routing steps (top-k, scan, dispatch), whose blocks fit
-    // beside the GEMM blocks on the same SMs, and then the down-projection,
-    // whose epilogue writes z straight into the slot rows.  Where that
-    // down-projection is split along K (few tokens) or a GEMV, it runs on the
-    // side stream first instead, and the caller's stream waits for z before
-    // the permute.  The caller's stream waits for the shared GEMM before the
-    // routed gate/up GEMM: the routed GEMMs then start with every SM free, as
-    // their static tile schedule wants.
+    // Two streams: the down-projection and the shared experts' gate/up GEMM
+    // need only x, so they run on the handle's side stream (the down GEMM
+    // first, beside the router GEMM, neither of which fills the GPU alone)
+    // while the caller's stream does the router and the latency-bound routing
+    // steps (top-k, scan, dispatch, permute), whose blocks fit beside the GEMM
+    // blocks on the same SMs.  The caller's stream waits for z before the
+    // permute, and for the shared GEMM before the routed gate/up GEMM: the
+    // routed GEMMs then start with every SM free, as their static tile
+    // schedule wants.  (A down-projection that writes z straight into the k
+    // slot rows from its epilogue, after the dispatch, was measured 5x slower
+    // than this GEMM plus the row-contiguous permute.)
     {
         // record + wait as one step, so that a forward from another host thread
         // cannot slip its own record in between
         std::lock_guard<std::mutex> lock(h->fork_mutex);
         LMOE_CUDA(cudaEventRecord(h->ev_fork, s));
         LMOE_CUDA(cudaStreamWaitEvent(h->side, h->ev_fork, 0));
-        if (!scatter) {
-            RUN(st_down(h->side));
-            LMOE_CUDA(cudaEventRecord(h->ev_z, h->side));
-        }
+        RUN(st_down(h->side));
+        LMOE_CUDA(cudaEventRecord(h->ev_z, h->side));
         RUN(st_shared(h->side));
         LMOE_CUDA(cudaEventRecord(h->ev_join, h->side));
     }
@@ -788,13 +765,9 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     RUN(st_topk(s));
     RUN(st_scan(s));
     RUN(st_dispatch(s));
-    if (scatter) {
-        RUN(st_down(s));      // needs slot_of from the dispatch
-    } else {
-        // a later record on the in-order side stream covers this forward's GEMMs too
-        LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_z, 0));
-        RUN(st_permute(s));
-    }
+    // a later record on the in-order side stream covers this forward's GEMMs too
+    LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_z, 0));
+    RUN(st_permute(s));
     LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
     RUN(st_gate_up(s));
     RUN(st_down_combine(s));

@@ -77,7 +77,6 @@ __device__ __forceinline__ float glu_act(int act, float g, float v, float cg, fl
 enum EpiMode {
     EPI_STORE = 0,    // out[m, n] = C                      (final GEMM -> y)
     EPI_SIGMOID = 1,  // out32[m, n] = sigmoid(C)           (router -> r)
-    EPI_SCATTER = 2,  // out[slot_of[m, j], n] = C, j < k   (down-projection -> z in the token's k slot rows)
     EPI_GLU = 3,      // out[m, n'] = act(C[gate], C[up])   (gate/up GEMMs -> h)
     EPI_COMBINE = 4,  // out[m, n] = w[m] * C               (routed down -> p-weighted rows)
     EPI_GLU_SITU = 5, // EPI_GLU with the SiTU gate, as its own instantiation
@@ -94,8 +93,6 @@ struct EpiArgs {
     int ib;                  // EPI_GLU: gate/up interleave block (columns)
     const void *residual;    // EPI_STORE: out = C + residual[m, n] (token dtype) when not NULL
     int64_t ldr;             // row stride of residual, elements
-    const int32_t *slot_of;  // EPI_SCATTER: [M, kslots] output rows of every input row
-    int kslots;
 };
 
 // Write n <= 32 consecutive values v[0..n) of row `row` starting at output column `col`.

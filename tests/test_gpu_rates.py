@@ -7,8 +7,10 @@ k-steps of a slice to one accumulator before the next), and the bulk-copy engine
 over an L2-resident and an HBM-sized buffer.  The test builds it with nvcc,
 runs it once, prints its JSON lines (``pytest -s`` shows them) and checks that
 every bounded wait completed and that the numbers are physically sensible:
-the largest shape issues at a rate near the tensor pipe's per-SM peak, and
-L2-resident copies are at least as fast as HBM-bound ones.
+the largest shape issues at a rate near the tensor pipe's per-SM peak,
+L2-resident copies are at least as fast as HBM-bound ones, and a second
+issuing thread speeds tiled copies up where more copies in flight from one
+thread do not.
 """
 import json
 import os
@@ -52,3 +54,10 @@ def test_mma_and_bulk_copy_rates():
     l2 = max(ln["GBps"] for ln in bulk if ln["span_bytes"] <= (48 << 20))
     hbm = max(ln["GBps"] for ln in bulk if ln["span_bytes"] > (1 << 30))
     assert l2 >= 0.9 * hbm, (l2, hbm)
+    # the finding the GEMM's producer warps rest on: tiled copies out of an
+    # L2-resident buffer go faster with a second issuing thread, not with more
+    # copies in flight from one
+    tile = {(ln["chunk"], ln["stages"], ln["issuers"]): ln["GBps"] for ln in lines
+            if ln["probe"] == "tile" and ln["span_bytes"] <= (48 << 20)}
+    assert tile[(16384, 12, 2)] > 1.5 * tile[(16384, 12, 1)], tile
+    assert tile[(16384, 12, 1)] < 1.2 * tile[(16384, 4, 1)], tile
