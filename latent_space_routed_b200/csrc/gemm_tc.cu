@@ -154,17 +154,23 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
 }
 
 // Arrive on a barrier given by its shared::cluster address (own CTA or peer).
+// Default semantics (release, CTA scope): what the arrive orders is this
+// warp's TMEM reads, already fenced by tcgen05.fence::before_thread_sync.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// Default semantics (acquire, CTA scope).  A phase completes only when its
+// transaction bytes (TMA, including a peer CTA's copies into this pair) and
+// its arrivals are in, which is what orders the consumers' reads; measured, a
+// cluster-scope acquire on every wait of the MMA issuer costs tensor-pipe time.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
