@@ -525,14 +525,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else if (warp == 1) {
         if (lane == 0 && leader) {
             // ---------------------------------------------------- MMA issuer (leader CTA)
+            // Between MMAs this thread does as little as it can (measured: a few
+            // extra instructions per MMA cost tensor-pipe time): the ring slot
+            // and phase advance incrementally, the shared-memory descriptors
+            // are a base plus constants, and the abort flag and the TMEM fence
+            // are looked at once per tile, not per k-step.
+            const uint64_t desc_base = sdesc_sw128(sbase);
+            constexpr uint32_t STAGE16 = C::STAGE_BYTES >> 4, A16 = C::A_BYTES >> 4;
             int it = 0, local = 0;
+            int s = 0;
+            uint32_t ph = 0u;
             bool ok = true;
             for (int item = group; item < total && ok; item += ngroups, ++local) {
                 const int acc = local & 1;
                 const uint32_t aph = (uint32_t)(local >> 1) & 1u;
                 const int split = item % p.ksplit;
                 const int kb_begin = split * nkb_total / p.ksplit, kb_end = (split + 1) * nkb_total / p.ksplit;
-                if (!mbar_wait(acce_bar(acc), aph ^ 1u)) {
+                if (!mbar_wait(acce_bar(acc), aph ^ 1u) || *(volatile int *)abort_flag) {
                     atomicOr(p.status, ST_MMA);
                     *(volatile int *)abort_flag = 1;
                     break;
@@ -545,25 +554,26 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     break;
                 }
                 const uint32_t dt = tmem_base + (uint32_t)(acc * BN);
+                uint32_t accumulate = 0u;      // the tile's first MMA overwrites the accumulator
                 for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!mbar_wait(full_bar(s), ph) || *(volatile int *)abort_flag) {
+                    if (!mbar_wait(full_bar(s), ph)) {
                         atomicOr(p.status, ST_MMA);
                         *(volatile int *)abort_flag = 1;
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
+                    const uint64_t da = desc_base + (uint64_t)(s * STAGE16);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = sdesc_sw128(sa + 32u * k);
-                        const uint64_t bd = sdesc_sw128(sa + C::A_BYTES + 32u * k);
-                        umma_bf16<CG>(dt, ad, bd, (kb > kb_begin || k > 0) ? 1u : 0u);
+                        umma_bf16<CG>(dt, da + (uint64_t)(2 * k), da + (uint64_t)(A16 + 2 * k), accumulate);
+                        accumulate = 1u;
                     }
                     umma_commit<CG>(empty_bar(s));
                     drain_counts[NPROD] = it + 1;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (ok) umma_commit<CG>(accf_bar(acc));
             }

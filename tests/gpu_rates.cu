@@ -41,20 +41,30 @@ static constexpr long long LIMIT = 4000000000ll;
 
 __device__ __forceinline__ uint32_t su32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// CLUSTER: wait with cluster-scope acquire semantics; otherwise the default
+// (acquire, CTA scope).
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool try_wait(uint32_t bar, uint32_t par)
 {
     uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(par) : "memory");
+    if (CLUSTER)
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(bar), "r"(par) : "memory");
+    else
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(bar), "r"(par) : "memory");
     return ok != 0;
 }
 
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t par)
 {
     const long long t0 = clock64();
-    while (!try_wait(bar, par))
+    while (!try_wait<CLUSTER>(bar, par))
         if (clock64() - t0 > LIMIT) return false;
     return true;
 }
@@ -66,14 +76,15 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t a)
 }
 
 // ------------------------------------------------------------------ mma
-template <int CG>
+template <int CG, int NACC, bool BLOCKED>
 __global__ void __launch_bounds__(128, 1)
-mma_kernel(int M, int N, int nacc, int blocked, int iters, unsigned long long *cycles, int *status)
+mma_kernel(int M, int N, int commit_every, int iters, unsigned long long *cycles, int *status)
 {
     extern __shared__ uint8_t dyn[];                  // A 128 rows, B up to 256 rows (K = 64), 1024-aligned
     constexpr int OPS = 128 * 128 + 256 * 128;
     uint8_t *ops = dyn + ((1024 - (su32(dyn) & 1023)) & 1023);
     __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(8) uint64_t step_bar;      // commit_every > 0: a commit per that many k-step rounds
     __shared__ uint32_t tmem_holder;
     uint32_t rank = 0;
     if (CG == 2) asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
@@ -81,6 +92,7 @@ mma_kernel(int M, int N, int nacc, int blocked, int iters, unsigned long long *c
         reinterpret_cast<__nv_bfloat16 *>(ops)[i] = __float2bfloat16((float)((i * 7) % 13 - 6) * 0.125f);
     if (threadIdx.x == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&bar)) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(su32(&step_bar)) : "memory");
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -119,17 +131,34 @@ mma_kernel(int M, int N, int nacc, int blocked, int iters, unsigned long long *c
                              ::"r"(d), "l"(ad[k]), "l"(bd[k]), "r"(idesc), "r"(acc));
         };
         // the issuing loop is kept to a few instructions per MMA (precomputed
-        // descriptors, no division): a heavier loop throttles the issue itself
-        for (int it = 0; it < iters; ++it) {
-            if (blocked) {      // accumulator outer: one accumulator takes all 4 k-steps of a 64-wide slice
-                for (int a = 0; a < nacc; ++a) {
+        // descriptors, compile-time accumulator count and order, no division):
+        // a heavier loop throttles the issue itself
+        const int group_len = commit_every > 0 ? commit_every : iters;
+        for (int it0 = 0; it0 < iters; it0 += group_len) {
+            for (int it = it0; it < it0 + group_len && it < iters; ++it) {
+                if (BLOCKED) {      // accumulator outer: one accumulator takes all 4 k-steps of a 64-wide slice
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) mma(tmem + (uint32_t)(a * N), k, (it > 0 || k > 0) ? 1u : 0u);
+                    for (int a = 0; a < NACC; ++a)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) mma(tmem + (uint32_t)(a * N), k, (it > 0 || k > 0) ? 1u : 0u);
+                } else {            // k-step outer, accumulator inner
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+#pragma unroll
+                        for (int a = 0; a < NACC; ++a) mma(tmem + (uint32_t)(a * N), k, (it > 0 || k > 0) ? 1u : 0u);
                 }
-            } else {            // k-step outer, accumulator inner
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    for (int a = 0; a < nacc; ++a) mma(tmem + (uint32_t)(a * N), k, (it > 0 || k > 0) ? 1u : 0u);
+            }
+            if (commit_every > 0) {
+                // the GEMM's per-stage pattern: a commit to a barrier (here never
+                // waited for) after a stage's MMAs, then the next stage's wait on
+                // an already complete barrier
+                if (CG == 2)
+                    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                                 ::"r"(su32(&step_bar)), "h"((uint16_t)0x3) : "memory");
+                else
+                    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                                 ::"r"(su32(&step_bar)) : "memory");
+                (void)try_wait(su32(&bar), 1);
             }
         }
         if (CG == 2)
@@ -161,7 +190,7 @@ constexpr int MAX_STAGES = 24;
 
 // One ring of `stages` copies per issuing thread (threads 0 and 32 when
 // issuers = 2, each with its own half of the buffer and barriers).
-template <bool TILED>
+template <bool TILED, bool CLUSTER>
 __global__ void __launch_bounds__(64, 1)
 copy_kernel(const uint8_t *src, size_t span, const __grid_constant__ CUtensorMap tm, int tile_rows, int rows_total,
             int kblocks, int chunk, int stages, int issuers, int iters, int *status)
@@ -182,7 +211,7 @@ copy_kernel(const uint8_t *src, size_t span, const __grid_constant__ CUtensorMap
     for (int it = 0; it < my_iters && ok; ++it) {
         const int s = it % st;
         if (it >= st) {   // the copy that used this stage last has landed
-            ok = wait_bounded(su32(&bars[s_base + s]), (uint32_t)((it / st - 1) & 1));
+            ok = wait_bounded<CLUSTER>(su32(&bars[s_base + s]), (uint32_t)((it / st - 1) & 1));
             if (!ok) break;
             ++done;
         }
@@ -204,7 +233,7 @@ copy_kernel(const uint8_t *src, size_t span, const __grid_constant__ CUtensorMap
     }
     // drain every copy still in flight (bounded)
     for (int i = done; i < issued; ++i)
-        if (!wait_bounded(su32(&bars[s_base + i % st]), (uint32_t)((i / st) & 1))) { ok = false; break; }
+        if (!wait_bounded<CLUSTER>(su32(&bars[s_base + i % st]), (uint32_t)((i / st) & 1))) { ok = false; break; }
     if (!ok) atomicOr(status, 4);
 }
 
@@ -221,17 +250,36 @@ int main(int argc, char **argv)
     CK(cudaMalloc(&cycles, sizeof(unsigned long long) * sms));
     CK(cudaMemset(status, 0, sizeof(int)));
 
-    CK(cudaFuncSetAttribute(mma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM));
-    CK(cudaFuncSetAttribute(mma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM));
+#define LMOE_SMEM(CGV)                                                                                          \
+    CK(cudaFuncSetAttribute(mma_kernel<CGV, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM)); \
+    CK(cudaFuncSetAttribute(mma_kernel<CGV, 2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM)); \
+    CK(cudaFuncSetAttribute(mma_kernel<CGV, 2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM));  \
+    CK(cudaFuncSetAttribute(mma_kernel<CGV, 4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM)); \
+    CK(cudaFuncSetAttribute(mma_kernel<CGV, 4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, MMA_SMEM));
+    LMOE_SMEM(1)
+    LMOE_SMEM(2)
+#undef LMOE_SMEM
     // (cta_group, M, N): the kind::f16 shapes of both groups
     const int shapes[][3] = {{1, 128, 256}, {1, 128, 192}, {1, 128, 128}, {1, 128, 64}, {1, 64, 256}, {1, 64, 128},
                              {2, 256, 256}, {2, 256, 192}, {2, 256, 128}, {2, 256, 64}, {2, 128, 256}};
     const int iters = 2000;
     for (const auto &sh : shapes) {
         const int cg = sh[0], M = sh[1], N = sh[2];
-        for (int mode = 0; mode < 5; ++mode) {
-            const int nacc = mode < 3 ? (1 << mode) : (mode == 3 ? 2 : 4), blocked = mode >= 3;
+        for (int mode = 0; mode < 8; ++mode) {
+            // modes 0-4: accumulator counts and orders; 5-7: one accumulator with a
+            // commit + wait after every 1, 2 or 4 rounds of 4 k-steps
+            const int nacc = mode < 3 ? (1 << mode) : (mode == 3 ? 2 : (mode == 4 ? 4 : 1));
+            const int blocked = mode == 3 || mode == 4;
+            const int commit_every = mode == 5 ? 1 : (mode == 6 ? 2 : (mode == 7 ? 4 : 0));
             if (nacc * N > 512) continue;
+            if (commit_every && !((cg == 2 && M == 256 && N == 256) || (cg == 1 && M == 128 && N == 256))) continue;
+            void (*kern)(int, int, int, int, unsigned long long *, int *) = nullptr;
+#define LMOE_PICK(CGV)                                                                                   \
+            kern = nacc == 1 ? mma_kernel<CGV, 1, false>                                                 \
+                 : nacc == 2 ? (blocked ? mma_kernel<CGV, 2, true> : mma_kernel<CGV, 2, false>)         \
+                             : (blocked ? mma_kernel<CGV, 4, true> : mma_kernel<CGV, 4, false>);
+            if (cg == 2) { LMOE_PICK(2) } else { LMOE_PICK(1) }
+#undef LMOE_PICK
             const int groups = sms / cg;
             cudaLaunchConfig_t lc = {};
             lc.gridDim = dim3(groups * cg);
@@ -245,8 +293,7 @@ int main(int argc, char **argv)
             lc.numAttrs = 1;
             lc.dynamicSmemBytes = MMA_SMEM;
             for (int rep = 0; rep < 2; ++rep) {   // the first launch warms up
-                if (cg == 2) CK(cudaLaunchKernelEx(&lc, mma_kernel<2>, M, N, nacc, blocked, iters, cycles, status));
-                else CK(cudaLaunchKernelEx(&lc, mma_kernel<1>, M, N, nacc, blocked, iters, cycles, status));
+                CK(cudaLaunchKernelEx(&lc, kern, M, N, commit_every, iters, cycles, status));
                 CK(cudaDeviceSynchronize());
             }
             unsigned long long h[256];
@@ -258,8 +305,9 @@ int main(int argc, char **argv)
             const double cyc = mean / n_mma;                         // cycles per instruction
             const double flop = 2.0 * M * N * 16;                    // per instruction (whole cta group)
             printf("{\"probe\": \"mma\", \"cta_group\": %d, \"M\": %d, \"N\": %d, \"nacc\": %d, "
-                   "\"order\": \"%s\", \"cycles_per_mma\": %.2f, \"flop_per_clk_per_sm\": %.1f}\n",
-                   cg, M, N, nacc, blocked ? "blocked" : "interleaved", cyc, flop / cyc / cg);
+                   "\"order\": \"%s\", \"commit_every\": %d, \"cycles_per_mma\": %.2f, "
+                   "\"flop_per_clk_per_sm\": %.1f}\n",
+                   cg, M, N, nacc, blocked ? "blocked" : "interleaved", commit_every, cyc, flop / cyc / cg);
         }
     }
 
@@ -275,9 +323,12 @@ int main(int argc, char **argv)
         CK(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
         encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
     }
-    CK(cudaFuncSetAttribute(copy_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
-    CK(cudaFuncSetAttribute(copy_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
-    // (tiled, span bytes, chunk bytes, stages, issuers)
+    CK(cudaFuncSetAttribute(copy_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
+    CK(cudaFuncSetAttribute(copy_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
+    CK(cudaFuncSetAttribute(copy_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
+    CK(cudaFuncSetAttribute(copy_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 196608 + 1024));
+    // (tiled, span bytes, chunk bytes, stages, issuers); every case runs with
+    // CTA-scope and with cluster-scope waits
     struct Case { int tiled; size_t span; int chunk, stages, issuers; };
     const Case cases[] = {
         {0, (size_t)48 << 20, 8192, 8, 1},  {0, (size_t)48 << 20, 8192, 24, 1}, {0, (size_t)48 << 20, 16384, 4, 1},
@@ -288,6 +339,7 @@ int main(int argc, char **argv)
         {1, (size_t)48 << 20, 16384, 4, 1}, {1, (size_t)48 << 20, 16384, 8, 1}, {1, (size_t)48 << 20, 16384, 12, 1},
         {1, (size_t)48 << 20, 16384, 12, 2}, {1, (size_t)48 << 20, 32768, 3, 1}, {1, (size_t)48 << 20, 32768, 6, 1},
         {1, (size_t)48 << 20, 32768, 6, 2}, {1, big, 16384, 12, 1},              {1, big, 32768, 6, 1}};
+    for (int scope = 0; scope < 2; ++scope)
     for (const Case &cs : cases) {
         const size_t smem = (size_t)cs.chunk * cs.stages + 1024;
         CUtensorMap tm;
@@ -313,12 +365,10 @@ int main(int argc, char **argv)
         float best = 1e30f;
         for (int rep = 0; rep < 3; ++rep) {
             CK(cudaEventRecord(a));
-            if (cs.tiled)
-                copy_kernel<true><<<sms, 64, smem>>>(src, cs.span, tm, rows, rows_total, K / 64, cs.chunk, cs.stages,
-                                                     cs.issuers, iters, status);
-            else
-                copy_kernel<false><<<sms, 64, smem>>>(src, cs.span, tm, rows, rows_total, K / 64, cs.chunk, cs.stages,
-                                                      cs.issuers, iters, status);
+            auto kern = cs.tiled ? (scope ? copy_kernel<true, true> : copy_kernel<true, false>)
+                                 : (scope ? copy_kernel<false, true> : copy_kernel<false, false>);
+            kern<<<sms, 64, smem>>>(src, cs.span, tm, rows, rows_total, K / 64, cs.chunk, cs.stages, cs.issuers, iters,
+                                    status);
             CK(cudaGetLastError());
             CK(cudaEventRecord(b));
             CK(cudaEventSynchronize(b));
@@ -327,9 +377,9 @@ int main(int argc, char **argv)
             if (ms < best) best = ms;
         }
         const double bytes = (double)sms * (iters / cs.issuers * cs.issuers) * cs.chunk;
-        printf("{\"probe\": \"%s\", \"span_bytes\": %zu, \"chunk\": %d, \"stages\": %d, \"issuers\": %d, "
-               "\"ctas\": %d, \"GBps\": %.1f}\n", cs.tiled ? "tile" : "bulk", cs.span, cs.chunk, cs.stages,
-               cs.issuers, sms, bytes / (best * 1e-3) / 1e9);
+        printf("{\"probe\": \"%s\", \"wait_scope\": \"%s\", \"span_bytes\": %zu, \"chunk\": %d, "
+               "\"stages\": %d, \"issuers\": %d, \"ctas\": %d, \"GBps\": %.1f}\n", cs.tiled ? "tile" : "bulk",
+               scope ? "cluster" : "cta", cs.span, cs.chunk, cs.stages, cs.issuers, sms, bytes / (best * 1e-3) / 1e9);
         cudaEventDestroy(a);
         cudaEventDestroy(b);
     }

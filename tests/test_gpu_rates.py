@@ -3,14 +3,16 @@
 ``tests/gpu_rates.cu`` (a standalone program) times tcgen05.mma for the
 kind::f16 shapes of both CTA groups with one, two or four independent
 accumulators in flight (each k-step to every accumulator in turn, or all
-k-steps of a slice to one accumulator before the next), and the bulk-copy engine's global -> shared bandwidth
-over an L2-resident and an HBM-sized buffer.  The test builds it with nvcc,
+k-steps of a slice to one accumulator before the next), and the copy engine's
+global -> shared bandwidth (1D bulk and tiled tensor copies) over an
+L2-resident and an HBM-sized buffer, with one or two issuing threads and
+barrier waits of CTA or cluster scope.  The test builds it with nvcc,
 runs it once, prints its JSON lines (``pytest -s`` shows them) and checks that
 every bounded wait completed and that the numbers are physically sensible:
 the largest shape issues at a rate near the tensor pipe's per-SM peak,
-L2-resident copies are at least as fast as HBM-bound ones, and a second
-issuing thread speeds tiled copies up where more copies in flight from one
-thread do not.
+L2-resident copies are at least as fast as HBM-bound ones, and copies waited
+for with CTA-scope barrier waits run at least as fast as with cluster-scope
+ones.
 """
 import json
 import os
@@ -44,7 +46,8 @@ def test_mma_and_bulk_copy_rates():
     assert rc == 0, err
     done = [ln for ln in lines if ln["probe"] == "done"]
     assert done and done[0]["status"] == 0
-    mma = {(ln["cta_group"], ln["M"], ln["N"], ln["nacc"], ln["order"]): ln for ln in lines if ln["probe"] == "mma"}
+    mma = {(ln["cta_group"], ln["M"], ln["N"], ln["nacc"], ln["order"]): ln for ln in lines
+           if ln["probe"] == "mma" and ln["commit_every"] == 0}
     # the pair shape the routed GEMMs use: within a factor two of 8192 FLOP
     # per clock per SM (the tensor pipe's nominal dense bf16 rate: 2.25
     # PFLOP/s over 148 SMs near 1.9 GHz)
@@ -54,10 +57,9 @@ def test_mma_and_bulk_copy_rates():
     l2 = max(ln["GBps"] for ln in bulk if ln["span_bytes"] <= (48 << 20))
     hbm = max(ln["GBps"] for ln in bulk if ln["span_bytes"] > (1 << 30))
     assert l2 >= 0.9 * hbm, (l2, hbm)
-    # the finding the GEMM's producer warps rest on: tiled copies out of an
-    # L2-resident buffer go faster with a second issuing thread, not with more
-    # copies in flight from one
-    tile = {(ln["chunk"], ln["stages"], ln["issuers"]): ln["GBps"] for ln in lines
+    # the GEMM waits on its barriers with CTA-scope acquire semantics: on the
+    # same copies that is at least as fast as cluster-scope waits
+    tile = {(ln["wait_scope"], ln["chunk"], ln["stages"], ln["issuers"]): ln["GBps"] for ln in lines
             if ln["probe"] == "tile" and ln["span_bytes"] <= (48 << 20)}
-    assert tile[(16384, 12, 2)] > 1.5 * tile[(16384, 12, 1)], tile
-    assert tile[(16384, 12, 1)] < 1.2 * tile[(16384, 4, 1)], tile
+    for key in [k for k in tile if k[0] == "cta"]:
+        assert tile[key] >= 0.95 * tile[("cluster",) + key[1:]], (key, tile)
