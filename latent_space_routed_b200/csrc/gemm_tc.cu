@@ -70,9 +70,17 @@ __device__ __forceinline__ int producer_index(int warp) { return warp == 0 ? 0 :
 constexpr int TMEM_COLS = 2 * BN;
 constexpr long long WAIT_LIMIT_CYCLES = 4000000000ll;   // about 2 s at 2 GHz
 constexpr int MAX_E = 1024;
-template <int CG> struct Tiles {
-    static constexpr int A_BYTES = 128 * BK * 2;                // this CTA's 128 A rows
-    static constexpr int B_BYTES = (BN / CG) * BK * 2;          // this CTA's share of B rows
+// KPS: 64-wide k-blocks per ring stage.  The MMA issuer commits each stage's
+// "empty" barrier once, and a commit costs tensor-pipe time: measured on B200,
+// a commit after every 4 MMAs holds them at 75 % of the pipe's rate, after
+// every 8 (CTA pairs) at 93 %, after every 16 at 100 %.  So the CTA-pair
+// GEMMs with bf16 outputs (the large ones) take two k-blocks per stage, laid
+// out as [A kb0][A kb1][B kb0][B kb1], each a standard 128-byte-swizzled tile.
+template <int CG, int KPS = 1> struct Tiles {
+    static constexpr int A_SUB = 128 * BK * 2;                  // this CTA's 128 A rows, one k-block
+    static constexpr int B_SUB = (BN / CG) * BK * 2;            // this CTA's share of B rows, one k-block
+    static constexpr int A_BYTES = KPS * A_SUB;
+    static constexpr int B_BYTES = KPS * B_SUB;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int TILE_M = 128 * CG;
     // kind::f16, D fp32, A and B bf16, both K-major, M = 128 CG, N = BN
@@ -85,14 +93,15 @@ template <int CG> struct Tiles {
 // stored by TMA), and as many operand stages as fit (at most 6): the weight
 // tiles of a grouped GEMM mostly come from HBM, and the ring is what keeps
 // their loads in flight.
-template <int CG, int OB> struct Cfg : Tiles<CG> {
+template <int CG, int OB, int KPS_ = (CG == 2 && OB == 2) ? 2 : 1> struct Cfg : Tiles<CG, KPS_> {
+    static constexpr int KPS = KPS_;
     static constexpr int EPI_CHUNK = 32 * 32 * OB;
     static constexpr int EPI_STAGING = 8 * EPI_CHUNK;
     static constexpr int TABLES = 2 * (int)sizeof(int) * (MAX_E + 1);
     static constexpr int FIXED = 1024 + EPI_STAGING + 256 + TABLES;
-    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG>::STAGE_BYTES;
+    static constexpr int STAGES_FIT = (232448 - FIXED) / Tiles<CG, KPS_>::STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG>::STAGE_BYTES;
+    static constexpr size_t SMEM = (size_t)FIXED + (size_t)STAGES * Tiles<CG, KPS_>::STAGE_BYTES;
     static_assert(STAGES >= 3, "operand ring too shallow");
 };
 
@@ -310,10 +319,20 @@ __device__ __forceinline__ float rcp_approx(float x)
     return y;
 }
 
+// sigmoid(x) = (1 + tanh(x / 2)) / 2: one tanh.approx (a single MUFU
+// operation) instead of an exponential and a reciprocal; its error, a few
+// units in 2^-11, is below the bf16 rounding that follows.
+__device__ __forceinline__ float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <bool SITU>
 __device__ __forceinline__ float glu_fast(float g, float v, float cg, float cu)
 {
-    const float sg = rcp_approx(1.0f + __expf(-g));
+    const float sg = fmaf(0.5f, tanh_approx(0.5f * g), 0.5f);
     if (SITU) return cg * tanhf(g * rcp_approx(cg)) * sg * (cu * tanhf(v * rcp_approx(cu)));
     return g * sg * v;
 }
@@ -501,7 +520,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
                 const int split = item % p.ksplit;
                 const int kb_end = (split + 1) * nkb_total / p.ksplit;
-                for (int kb = split * nkb_total / p.ksplit; kb < kb_end; ++kb, ++it) {
+                for (int kb = split * nkb_total / p.ksplit; kb < kb_end; kb += C::KPS, ++it) {
                     if (it % NP != pw) continue;
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -511,13 +530,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         ok = false;
                         break;
                     }
-                    const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
+                    const int nk = kb_end - kb < C::KPS ? kb_end - kb : C::KPS;   // k-blocks in this stage
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
                     const uint32_t fb = CG == 2 ? map_to_rank(full_bar(s), 0) : full_bar(s);
-                    if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
-                    tma_load_2d<CG>(sa, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
-                    tma_load_2d<CG>(sa + C::A_BYTES, &tmB, fb, kk,
-                                    (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
+                    if (leader) mbar_expect_tx(full_bar(s), CG * nk * (C::A_SUB + C::B_SUB));
+                    for (int j = 0; j < nk; ++j) {
+                        const int term = (kb + j) / p.nkb, kk = ((kb + j) % p.nkb) * BK;
+                        tma_load_2d<CG>(sa + j * C::A_SUB, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
+                        tma_load_2d<CG>(sa + C::A_BYTES + j * C::B_SUB, &tmB, fb, kk,
+                                        (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
+                    }
                     drain_counts[pw] = it + 1;
                 }
             }
@@ -532,6 +554,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // are looked at once per tile, not per k-step.
             const uint64_t desc_base = sdesc_sw128(sbase);
             constexpr uint32_t STAGE16 = C::STAGE_BYTES >> 4, A16 = C::A_BYTES >> 4;
+            constexpr uint32_t ASUB16 = C::A_SUB >> 4, BSUB16 = C::B_SUB >> 4;
             int it = 0, local = 0;
             int s = 0;
             uint32_t ph = 0u;
@@ -555,7 +578,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
                 const uint32_t dt = tmem_base + (uint32_t)(acc * BN);
                 uint32_t accumulate = 0u;      // the tile's first MMA overwrites the accumulator
-                for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+                for (int kb = kb_begin; kb < kb_end; kb += C::KPS, ++it) {
                     if (!mbar_wait(full_bar(s), ph)) {
                         atomicOr(p.status, ST_MMA);
                         *(volatile int *)abort_flag = 1;
@@ -564,9 +587,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                     const uint64_t da = desc_base + (uint64_t)(s * STAGE16);
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        umma_bf16<CG>(dt, da + (uint64_t)(2 * k), da + (uint64_t)(A16 + 2 * k), accumulate);
-                        accumulate = 1u;
+                    for (int j = 0; j < C::KPS; ++j) {
+                        if (j > 0 && kb + j >= kb_end) break;      // a tile's odd last k-block
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            umma_bf16<CG>(dt, da + (uint64_t)(j * ASUB16 + 2 * k),
+                                          da + (uint64_t)(A16 + j * BSUB16 + 2 * k), accumulate);
+                            accumulate = 1u;
+                        }
                     }
                     umma_commit<CG>(empty_bar(s));
                     drain_counts[NPROD] = it + 1;

@@ -3,7 +3,9 @@
 ``tests/gpu_rates.cu`` (a standalone program) times tcgen05.mma for the
 kind::f16 shapes of both CTA groups with one, two or four independent
 accumulators in flight (each k-step to every accumulator in turn, or all
-k-steps of a slice to one accumulator before the next), and the copy engine's
+k-steps of a slice to one accumulator before the next), and with a commit and
+a barrier wait after every 4, 8 or 16 MMAs (the GEMM's per-stage pattern),
+and the copy engine's
 global -> shared bandwidth (1D bulk and tiled tensor copies) over an
 L2-resident and an HBM-sized buffer, with one or two issuing threads and
 barrier waits of CTA or cluster scope.  The test builds it with nvcc,
@@ -11,8 +13,8 @@ runs it once, prints its JSON lines (``pytest -s`` shows them) and checks that
 every bounded wait completed and that the numbers are physically sensible:
 the largest shape issues at a rate near the tensor pipe's per-SM peak,
 L2-resident copies are at least as fast as HBM-bound ones, and copies waited
-for with CTA-scope barrier waits run at least as fast as with cluster-scope
-ones.
+for with CTA-scope barrier waits run as fast as with cluster-scope ones
+(within 10 %).
 """
 import json
 import os
@@ -58,8 +60,8 @@ def test_mma_and_bulk_copy_rates():
     hbm = max(ln["GBps"] for ln in bulk if ln["span_bytes"] > (1 << 30))
     assert l2 >= 0.9 * hbm, (l2, hbm)
     # the GEMM waits on its barriers with CTA-scope acquire semantics: on the
-    # same copies that is at least as fast as cluster-scope waits
+    # same copies that is as fast as cluster-scope waits, within 10 %
     tile = {(ln["wait_scope"], ln["chunk"], ln["stages"], ln["issuers"]): ln["GBps"] for ln in lines
             if ln["probe"] == "tile" and ln["span_bytes"] <= (48 << 20)}
     for key in [k for k in tile if k[0] == "cta"]:
-        assert tile[key] >= 0.95 * tile[("cluster",) + key[1:]], (key, tile)
+        assert tile[key] >= 0.9 * tile[("cluster",) + key[1:]], (key, tile)
