@@ -126,6 +126,7 @@ struct TcParams {
     int out_cols;               // columns of the output tensor map
     int stall_test;             // failure-detection test: the MMA warp waits on a barrier nobody signals
     int tma_store;              // 1: full chunks leave through TMA stores
+    int load3d;                 // 1: the tensor maps are 3D (KPS k-blocks per copy)
     int32_t *status;
 };
 
@@ -215,6 +216,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
             "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
             " [%0], [%1, {%3, %4}], [%2];"
             ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
+            : "memory");
+}
+
+// 3D tile load: coordinates {k inside the k-block, row, k-block}; with a box
+// of {64, rows, KPS} it brings KPS consecutive k-blocks of the same rows as KPS
+// standard 128-byte-swizzled tiles, one after another, in one copy.
+template <int CG>
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c1, int c2)
+{
+    if (CG == 2)
+        asm volatile(
+            "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4, %5}], [%2];"
+            ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(0), "r"(c1), "r"(c2)
+            : "memory");
+    else
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%3, %4, %5}], [%2];"
+            ::"r"(dst), "l"((uint64_t)map), "r"(bar), "r"(0), "r"(c1), "r"(c2)
             : "memory");
 }
 
@@ -533,12 +554,20 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     const int nk = kb_end - kb < C::KPS ? kb_end - kb : C::KPS;   // k-blocks in this stage
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
                     const uint32_t fb = CG == 2 ? map_to_rank(full_bar(s), 0) : full_bar(s);
-                    if (leader) mbar_expect_tx(full_bar(s), CG * nk * (C::A_SUB + C::B_SUB));
-                    for (int j = 0; j < nk; ++j) {
-                        const int term = (kb + j) / p.nkb, kk = ((kb + j) % p.nkb) * BK;
-                        tma_load_2d<CG>(sa + j * C::A_SUB, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
-                        tma_load_2d<CG>(sa + C::A_BYTES + j * C::B_SUB, &tmB, fb, kk,
-                                        (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
+                    if (C::KPS > 1 && p.load3d) {
+                        // one copy per operand; a k-block past the end reads as zeros
+                        // (and its MMAs are skipped) but still counts its bytes
+                        if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
+                        tma_load_3d<CG>(sa, &tmA, fb, (int)(t.row0 + 128 * rank), kb);
+                        tma_load_3d<CG>(sa + C::A_BYTES, &tmB, fb, (int)(t.brow + (BN / CG) * rank), kb);
+                    } else {
+                        if (leader) mbar_expect_tx(full_bar(s), CG * nk * (C::A_SUB + C::B_SUB));
+                        for (int j = 0; j < nk; ++j) {
+                            const int term = (kb + j) / p.nkb, kk = ((kb + j) % p.nkb) * BK;
+                            tma_load_2d<CG>(sa + j * C::A_SUB, &tmA, fb, kk, (int)(t.row0 + 128 * rank));
+                            tma_load_2d<CG>(sa + C::A_BYTES + j * C::B_SUB, &tmB, fb, kk,
+                                            (int)(t.brow + (BN / CG) * rank + term * p.term_rows));
+                        }
                     }
                     drain_counts[pw] = it + 1;
                 }
@@ -763,6 +792,22 @@ bool make_out_map(CUtensorMap *m, void *base, bool f32, uint64_t cols, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+// 3D view {64 k (contiguous), rows (row_bytes apart), k-blocks (128 bytes
+// apart)} of a K-major bf16 matrix, box {64, box_rows, kps}: one copy lands
+// kps k-blocks of box_rows rows as kps 128-byte-swizzled tiles back to back.
+bool make_map3(CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint64_t row_bytes, uint32_t box_rows,
+               uint32_t kps)
+{
+    cuuint64_t dims[3] = {(cuuint64_t)BK, rows, K / BK};
+    cuuint64_t strides[2] = {row_bytes, (cuuint64_t)BK * 2};
+    cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, kps};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_outer)
 {
     cuuint64_t dims[2] = {inner, outer};
@@ -875,11 +920,19 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.stall_test = g_stall_next.exchange(0);
     if (p.max_tiles == 0) return cudaSuccess;
     CUtensorMap ta, tb;
-    if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128)) return cudaErrorInvalidValue;
-    if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG))
-        return cudaErrorInvalidValue;
     if (mode == EPI_SIGMOID_PARTIAL) mode = EPI_STORE_F32;   // raw fp32 partial tiles; sigmoid after the sum
     const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_STORE_F32);
+    const int kps = Cfg<CG, 2>::KPS;
+    p.load3d = 0;
+    if (!out_f32 && kps > 1 && nterms == 1 && p.ksplit == 1 &&
+        make_map3(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128, kps) &&
+        make_map3(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG, kps)) {
+        p.load3d = 1;
+    } else {
+        if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128)) return cudaErrorInvalidValue;
+        if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG))
+            return cudaErrorInvalidValue;
+    }
     p.out_cols = (mode == EPI_GLU) ? g.N / 2 : g.N;
     CUtensorMap tc;
     memset(&tc, 0, sizeof tc);
