@@ -121,7 +121,7 @@ LMOE_API lmoe_status lmoe_config_from_base(int32_t d, int32_t m, int32_t N, int3
                                   int32_t n_shared, const char *variant, lmoe_config *out);
 
 /* Validate cfg, allocate handle-owned device memory on the current device and
- * repack the weights into it (gate/up rows interleaved per tile, the shared
+ * repack the weights into it (gate/up rows interleaved in blocks, the shared
  * down projections and W_up concatenated, the router split for the tensor
  * cores).  Work is enqueued on `stream`, which is synchronised before return,
  * so the caller may free its weight copies afterwards.

@@ -127,6 +127,7 @@ struct TcParams {
     int stall_test;             // failure-detection test: the MMA warp waits on a barrier nobody signals
     int tma_store;              // 1: full chunks leave through TMA stores
     int load3d;                 // 1: the tensor maps are 3D (KPS k-blocks per copy)
+    int half_tiles;             // 1: an expert's last m-tile of at most 64 CG rows runs as an M = 64 CG MMA
     int32_t *status;
 };
 
@@ -253,20 +254,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
 }
 
 template <int CG>
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate)
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
 {
     if (CG == 2)
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Tiles<CG>::IDESC), "r"(accumulate));
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
     else
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
             "setp.ne.b32 p, %4, 0;\n\t"
             "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(Tiles<CG>::IDESC), "r"(accumulate));
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 // Arrive on `bar` (the same offset in every CTA of the group) once all MMAs
@@ -424,6 +426,7 @@ struct Tile {
     int64_t row0, row_end;  // A rows [row0, row_end) of the whole (128 CG)-row tile are real
     int64_t brow;           // first B row of this tile (term 0)
     int n0;                 // first output column (GEMM n)
+    bool half;              // half tile: 64 rows per CTA, M = 64 CG
 };
 
 // Grouped mode reads the expert row offsets and m-tile prefix from shared
@@ -443,18 +446,20 @@ __device__ __forceinline__ Tile decode(const TcParams &p, const int *s_tile_off,
         t.row0 = (int64_t)s_offsets[lo] + (int64_t)(mt - s_tile_off[lo]) * Tiles<CG>::TILE_M;
         t.row_end = s_offsets[lo + 1];
         t.brow = (int64_t)lo * p.group_rows + t.n0;
+        t.half = CG == 2 && p.half_tiles && t.row_end - t.row0 <= 64 * CG;
     } else {
         t.row0 = (int64_t)mt * Tiles<CG>::TILE_M;
         t.row_end = p.M;
         t.brow = t.n0;
+        t.half = false;
     }
     return t;
 }
 
 template <int MODE, typename TO, int CG>
 __global__ void __launch_bounds__(THREADS, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmC, const TcParams p)
+tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAh,
+               const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC, const TcParams p)
 {
     using C = Cfg<CG, (int)sizeof(TO)>;
     constexpr int STAGES = C::STAGES;
@@ -468,6 +473,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
     int *abort_flag = reinterpret_cast<int *>(tmem_holder + 1);
     int *drain_counts = abort_flag + 1;   // [0, NPROD) k-steps issued by each producer, [NPROD] consumed
+    int *s_half = drain_counts + NPROD + 1;   // [STAGES] half-tile flag of the k-step in ring slot s
     int *s_tile_off = reinterpret_cast<int *>(gbase + (size_t)STAGES * C::STAGE_BYTES + C::EPI_STAGING + 256);
     int *s_offsets = s_tile_off + (MAX_E + 1);                                                 // [E+1]
 
@@ -496,6 +502,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        if (p.half_tiles) tma_prefetch_desc(&tmAh);
     }
     if (warp == 1) {
         if (CG == 2) {
@@ -553,12 +560,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                     const int nk = kb_end - kb < C::KPS ? kb_end - kb : C::KPS;   // k-blocks in this stage
                     const uint32_t sa = sbase + (uint32_t)s * C::STAGE_BYTES;
+                    if (leader) s_half[s] = t.half;   // published to the MMA thread by the arrive below
                     const uint32_t fb = CG == 2 ? map_to_rank(full_bar(s), 0) : full_bar(s);
                     if (C::KPS > 1 && p.load3d) {
                         // one copy per operand; a k-block past the end reads as zeros
                         // (and its MMAs are skipped) but still counts its bytes
-                        if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
-                        tma_load_3d<CG>(sa, &tmA, fb, (int)(t.row0 + 128 * rank), kb);
+                        if (t.half) {   // 64 A rows per CTA: [kb0 64 rows][kb1 64 rows]
+                            if (leader) mbar_expect_tx(full_bar(s), CG * (C::A_BYTES / 2 + C::B_BYTES));
+                            tma_load_3d<CG>(sa, &tmAh, fb, (int)(t.row0 + 64 * rank), kb);
+                        } else {
+                            if (leader) mbar_expect_tx(full_bar(s), CG * C::STAGE_BYTES);
+                            tma_load_3d<CG>(sa, &tmA, fb, (int)(t.row0 + 128 * rank), kb);
+                        }
                         tma_load_3d<CG>(sa + C::A_BYTES, &tmB, fb, (int)(t.brow + (BN / CG) * rank), kb);
                     } else {
                         if (leader) mbar_expect_tx(full_bar(s), CG * nk * (C::A_SUB + C::B_SUB));
@@ -584,6 +597,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const uint64_t desc_base = sdesc_sw128(sbase);
             constexpr uint32_t STAGE16 = C::STAGE_BYTES >> 4, A16 = C::A_BYTES >> 4;
             constexpr uint32_t ASUB16 = C::A_SUB >> 4, BSUB16 = C::B_SUB >> 4;
+            constexpr uint32_t IDESC_HALF = (C::IDESC & ~(0x1fu << 24)) | ((uint32_t)((64 * CG) >> 4) << 24);
             int it = 0, local = 0;
             int s = 0;
             uint32_t ph = 0u;
@@ -593,6 +607,9 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 const uint32_t aph = (uint32_t)(local >> 1) & 1u;
                 const int split = item % p.ksplit;
                 const int kb_begin = split * nkb_total / p.ksplit, kb_end = (split + 1) * nkb_total / p.ksplit;
+                // half tile: M = 64 CG, this CTA's k-blocks of A 64 rows (8 KB) apart; the
+                // flag comes with the tile's first stage (no table search in this thread)
+                uint32_t idesc = C::IDESC, astep = ASUB16;
                 if (!mbar_wait(acce_bar(acc), aph ^ 1u) || *(volatile int *)abort_flag) {
                     atomicOr(p.status, ST_MMA);
                     *(volatile int *)abort_flag = 1;
@@ -614,14 +631,18 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         ok = false;
                         break;
                     }
+                    if (kb == kb_begin && p.half_tiles && s_half[s]) {
+                        idesc = IDESC_HALF;
+                        astep = ASUB16 / 2;
+                    }
                     const uint64_t da = desc_base + (uint64_t)(s * STAGE16);
 #pragma unroll
                     for (int j = 0; j < C::KPS; ++j) {
                         if (j > 0 && kb + j >= kb_end) break;      // a tile's odd last k-block
 #pragma unroll
                         for (int k = 0; k < BK / 16; ++k) {
-                            umma_bf16<CG>(dt, da + (uint64_t)(j * ASUB16 + 2 * k),
-                                          da + (uint64_t)(A16 + j * BSUB16 + 2 * k), accumulate);
+                            umma_bf16<CG>(dt, da + (uint64_t)(j * astep + 2 * k),
+                                          da + (uint64_t)(A16 + j * BSUB16 + 2 * k), idesc, accumulate);
                             accumulate = 1u;
                         }
                     }
@@ -638,7 +659,11 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else {
         // -------------------------------------------------------- epilogue warps 2..9
         // Two warps per TMEM lane quarter; warp set h = 0/1 takes the 32-column
-        // chunks c = 32 h + 64 i, so each warp drains half of its 32 rows' tile.
+        // chunk pairs (c, c + 64) with c = 32 h + 128 i, so each warp drains half
+        // of its 32 rows' tile.  A half tile (M = 64 CG) holds this CTA's 64 rows
+        // with GEMM columns [0, 128) in lanes 0-63 and [128, 256) in lanes 64-127,
+        // both at TMEM columns [0, 128): quarter q has rows 32 (q & 1) + lane and
+        // GEMM columns 128 (q >> 1) + [0, 128), one chunk pair per warp.
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int hset = (warp - 2) >> 2;       // 0 for warps 2..5, 1 for warps 6..9
         const uint32_t ebuf = epi_base + (uint32_t)(warp - 2) * C::EPI_CHUNK;
@@ -657,14 +682,16 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tc_fence_after();
             const Tile t = decode<CG>(p, s_tile_off, s_offsets, item / p.ksplit);
             const int64_t slab = (int64_t)(item % p.ksplit) * p.split_rows;   // 0 unless split K
-            const int64_t row = t.row0 + 128 * rank + 32 * q + lane;
+            const int64_t chunk_row = t.half ? t.row0 + 64 * rank + 32 * (q & 1) : t.row0 + 128 * rank + 32 * q;
+            const int cbase = t.half ? 128 * (q >> 1) : 0;   // GEMM column of this quarter's TMEM column 0
+            const int npair = t.half ? 1 : 2;                // chunk pairs per warp
+            const int64_t row = chunk_row + lane;
             const bool valid = row < t.row_end;
             const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * BN);
             float v[32], u[32];
             // Emit 32 output columns [col, col + n) of this warp's 32 rows: whole
             // chunks go through the staging buffer and one TMA store; chunks that
             // straddle an expert's last row (or a ragged column edge) store per lane.
-            const int64_t chunk_row = t.row0 + 128 * rank + 32 * q;
             const bool rows_ok = (p.offsets || p.ksplit > 1) ? (chunk_row + 32 <= t.row_end) : true;
             auto emit = [&](const float *x, int col, int n) {
                 if (p.tma_store && rows_ok && n == 32) {
@@ -681,25 +708,28 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 }
             };
             if (MODE == EPI_GLU || MODE == EPI_GLU_SITU) {
-                const int half = BN / 2;
+                // gate/up rows interleaved in blocks of 64: GEMM columns [128 i, 128 i + 64)
+                // are gates of outputs 64 i + [0, 64), the next 64 their ups
 #pragma unroll 1
-                for (int c = 32 * hset; c < half; c += 64) {
+                for (int i = 0; i < npair; ++i) {
+                    const int c = 32 * hset + 128 * i;
                     __syncwarp();
-                    tmem_ld32_pair(tq + c, tq + half + c, v, u);   // gate and up columns, one wait
+                    tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // gate and up columns, one wait
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = glu_fast<MODE == EPI_GLU_SITU>(v[i], u[i], p.epi.gate_cap,
+                    for (int e = 0; e < 32; ++e) v[e] = glu_fast<MODE == EPI_GLU_SITU>(v[e], u[e], p.epi.gate_cap,
                                                                                        p.epi.up_cap);
-                    emit(v, t.n0 / 2 + c, 32);
+                    emit(v, (t.n0 + cbase) / 2 + 32 * hset + 64 * i, 32);
                 }
             } else {
 #pragma unroll 1
-                for (int c = 32 * hset; c < BN; c += 128) {
+                for (int i = 0; i < npair; ++i) {
+                    const int c = 32 * hset + 128 * i;
                     __syncwarp();
                     tmem_ld32_pair(tq + c, tq + c + 64, v, u);     // warp-collective: every lane
 #pragma unroll
                     for (int part = 0; part < 2; ++part) {
                         float *x = part ? u : v;
-                        const int col = t.n0 + c + 64 * part;
+                        const int col = t.n0 + cbase + c + 64 * part;
                         int n = p.N - col;
                         if (n > 32) n = 32;
                         if (n <= 0) continue;             // uniform across the warp
@@ -862,7 +892,8 @@ cudaError_t group_capacity(int *max_groups)
 
 // Persistent grid: min(work items, CTA groups that can be resident at once).
 template <int MODE, typename TO, int CG>
-cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &c, const TcParams &p, cudaStream_t s)
+cudaError_t launch(const CUtensorMap &a, const CUtensorMap &ah, const CUtensorMap &b, const CUtensorMap &c,
+                   const TcParams &p, cudaStream_t s)
 {
     auto kern = tc_gemm_kernel<MODE, TO, CG>;
     int max_groups = 0;
@@ -884,7 +915,7 @@ cudaError_t launch(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
     lc.numAttrs = 2;
-    return cudaLaunchKernelEx(&lc, kern, a, b, c, p);
+    return cudaLaunchKernelEx(&lc, kern, a, ah, b, c, p);
 }
 
 template <int CG>
@@ -919,7 +950,8 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.status = status;
     p.stall_test = g_stall_next.exchange(0);
     if (p.max_tiles == 0) return cudaSuccess;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tah, tb;
+    memset(&tah, 0, sizeof tah);
     if (mode == EPI_SIGMOID_PARTIAL) mode = EPI_STORE_F32;   // raw fp32 partial tiles; sigmoid after the sum
     const bool out_f32 = (mode == EPI_SIGMOID || mode == EPI_STORE_F32);
     const int kps = Cfg<CG, 2>::KPS;
@@ -928,6 +960,9 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
         make_map3(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128, kps) &&
         make_map3(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG, kps)) {
         p.load3d = 1;
+        // grouped: an expert's last m-tile of at most 128 rows loads 64 rows per CTA
+        p.half_tiles = (CG == 2 && g.offsets &&
+                        make_map3(&tah, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 64, kps)) ? 1 : 0;
     } else {
         if (!make_map(&ta, g.A, (uint64_t)g.K, (uint64_t)g.M, (uint64_t)g.lda * 2, 128)) return cudaErrorInvalidValue;
         if (!make_map(&tb, g.B, (uint64_t)g.K, (uint64_t)b_rows_total, (uint64_t)g.ldb * 2, BN / CG))
@@ -939,13 +974,13 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
     p.tma_store = make_out_map(&tc, g.epi.out, out_f32, (uint64_t)p.out_cols, (uint64_t)g.M * p.ksplit,
                                (uint64_t)g.epi.ldo * (out_f32 ? 4 : 2)) ? 1 : 0;
     switch (mode) {
-    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG>(ta, tb, tc, p, s);
+    case EPI_SIGMOID: return launch<EPI_SIGMOID, float, CG>(ta, tah, tb, tc, p, s);
     case EPI_GLU:
-        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG>(ta, tb, tc, p, s);
-        return launch<EPI_GLU, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tb, tc, p, s);
-    case EPI_STORE_F32: return launch<EPI_STORE, float, CG>(ta, tb, tc, p, s);
+        if (g.epi.act == LMOE_ACT_SITU) return launch<EPI_GLU_SITU, bf16, CG>(ta, tah, tb, tc, p, s);
+        return launch<EPI_GLU, bf16, CG>(ta, tah, tb, tc, p, s);
+    case EPI_COMBINE: return launch<EPI_COMBINE, bf16, CG>(ta, tah, tb, tc, p, s);
+    case EPI_STORE: return launch<EPI_STORE, bf16, CG>(ta, tah, tb, tc, p, s);
+    case EPI_STORE_F32: return launch<EPI_STORE, float, CG>(ta, tah, tb, tc, p, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -328,7 +328,7 @@ lmoe_status lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *str
     h->cfg = *cfg;
     cudaGetDevice(&h->device);
     h->tc = tc;
-    h->ib = tc ? TC_BN / 2 : SIMT_BN / 2;
+    h->ib = tc ? TC_BN / 4 : SIMT_BN / 2;   // tensor cores: 64-row blocks (see the GLU epilogue)
     h->tb = cfg->dtype == LMOE_BF16 ? 2 : 4;
     const lmoe_config &c = *cfg;
     const size_t tb = h->tb;
@@ -661,7 +661,7 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         gp.epi.ldo = g.N;
         cudaError_t e = tc_gemm(EPI_STORE_F32, gp, 0, 1, status, q, ks);
         if (e != cudaSuccess) return e;
-        return launch_splitk_reduce(part, ks, g.M, g.N, mode, g.epi.act, g.epi.gate_cap, g.epi.up_cap, TC_BN / 2,
+        return launch_splitk_reduce(part, ks, g.M, g.N, mode, g.epi.act, g.epi.gate_cap, g.epi.up_cap, g.epi.ib,
                                     g.epi.out, g.epi.ldo, q, g.epi.residual, g.epi.ldr);
     };
     auto st_down = [&](cudaStream_t q) -> lmoe_status {
