@@ -988,20 +988,33 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
 
 // ------------------------------------------------------------------ router + top-k
 // Router scores, biased top-k and renormalisation in one launch ("Stable
-// LatentMoE", equations for r, T_k(x) and p_i), for E <= 512 experts.
+// LatentMoE", equations for r, T_k(x) and p_i), for E <= 256 experts.
 //
 // A cluster of KS CTAs takes one 128-token tile: CTA `rank` runs the k-blocks
 // [rank, rank + 1) * NKB / KS of the three bf16 terms of the fp32 router
 // weight (hi + mid + lo; with bf16 tokens every product is exact in fp32)
-// through tcgen05.mma into one fp32 TMEM accumulator of E columns (two
-// 256-column halves for E = 512).  Its eight epilogue warps write the partial
-// logits to L2 (KS > 1; in rank slabs) or, for KS = 1, r = sigmoid(logit)
-// directly.  After a cluster barrier each CTA owns 128 / KS tokens of the
-// tile: one warp per token sums the KS partial logits in rank order (fixed
-// order, deterministic), applies the sigmoid and writes r, runs the warp
-// tournament on r + b (warp_topk: equal scores to the lower index), and writes
-// the selection, p from the raw scores, the Quantile-Balancing cutoff and the
-// per-32-token expert counts that the counting sort scans.
+// through tcgen05.mma into one fp32 TMEM accumulator of E columns.  Its eight
+// epilogue warps move the partial logits into its own shared memory (the
+// drained operand ring: 128 rows of E + 1 floats) or, for KS = 1,
+// r = sigmoid(logit) there and to global r.  After a cluster barrier each CTA
+// owns 128 / KS tokens of the tile: one warp per token reads the KS partial
+// logits of its row from the cluster's shared memory and sums them in rank
+// order (fixed order, deterministic), applies the sigmoid and writes r, runs
+// the warp tournament on r + b (warp_topk: equal scores to the lower index),
+// and writes the selection, p from the raw scores, the Quantile-Balancing
+// cutoff and the per-32-token expert counts that the counting sort scans.  A
+// last cluster barrier keeps every CTA's shared memory alive until its peers
+// have read it.
+constexpr int RT_SMEM_FIXED = 1024 + 256;   // alignment slack, barriers and flags
+constexpr int RT_MAX_KS = 8;                 // CTAs per cluster (portable cluster size)
+
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
 struct RtParams {
     int T, E, k;
     int nkb;                 // k-blocks of 64 per term (d / 64)
@@ -1010,7 +1023,6 @@ struct RtParams {
     uint32_t idesc;          // kind::f16, M = 128, N = n_half
     int stages, stage_bytes, tmem_cols;
     const float *bias;
-    float *partial;          // [ks][T][E] partial logits (ks > 1)
     float *r;                // [T][E]
     int32_t *sel;
     float *p32;
@@ -1046,6 +1058,8 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     const uint32_t accf = bar0 + 8u * (2 * STAGES);
     const int a_bytes = 128 * BK * 2, bh_bytes = p.n_half * BK * 2;
+    float *tile = reinterpret_cast<float *>(gbase);   // logit tile over the drained ring: [128][ld]
+    const int ld = p.E + 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -1076,16 +1090,16 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int NP = NPROD < STAGES ? NPROD : STAGES;   // producers in use (see NPROD)
     if (pw >= 0) {
         if (lane == 0 && pw < NP) {   // ------------------------------------ TMA producers (k-step it % NP)
-            int it = 0;
-            for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
-                if (it % NP != pw) continue;
-                const int s = it % STAGES;
-                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                if (!mbar_wait(empty_bar(s), ph ^ 1u) || *(volatile int *)abort_flag) {
+            // k-steps it = pw, pw + NP, ...; slot and phase advance incrementally (NP <= STAGES)
+            int s = pw;
+            uint32_t ph = 0u;
+            for (int it = pw; kb_begin + it < kb_end; it += NP) {
+                if (!mbar_wait(empty_bar(s), ph ^ 1u)) {
                     atomicOr(p.status, ST_PRODUCER);
                     *(volatile int *)abort_flag = 1;
                     break;
                 }
+                const int kb = kb_begin + it;
                 const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
                 const uint32_t sa = sbase + (uint32_t)s * p.stage_bytes;
                 mbar_expect_tx(full_bar(s), a_bytes + p.halves * bh_bytes);
@@ -1094,11 +1108,17 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     tma_load_2d<1>(sa + a_bytes + h * bh_bytes, &tmB, full_bar(s), kk,
                                    term * p.E + h * p.n_half);
                 drain_counts[pw] = it + 1;
+                s += NP;
+                if (s >= STAGES) {
+                    s -= STAGES;
+                    ph ^= 1u;
+                }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {   // ------------------------------------------------ MMA issuer
-            int it = 0;
+            // as in the GEMM: incremental slot and phase, descriptors as a base plus
+            // constants, and nothing else between the MMAs of a stage
             bool ok = true;
             if (p.stall_test && !mbar_wait(accf, 0u)) {
                 // only this thread commits that barrier: the wait runs out by design
@@ -1106,32 +1126,39 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 *(volatile int *)abort_flag = 1;
                 ok = false;
             }
+            const uint64_t desc0 = sdesc_sw128(sbase);
+            const uint32_t st16 = (uint32_t)p.stage_bytes >> 4, a16 = (uint32_t)a_bytes >> 4,
+                           bh16 = (uint32_t)bh_bytes >> 4;
+            int s = 0, it = 0;
+            uint32_t ph = 0u;
             for (int kb = kb_begin; kb < kb_end && ok; ++kb, ++it) {
-                const int s = it % STAGES;
-                const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                if (!mbar_wait(full_bar(s), ph) || *(volatile int *)abort_flag) {
+                if (!mbar_wait(full_bar(s), ph)) {
                     atomicOr(p.status, ST_MMA);
                     *(volatile int *)abort_flag = 1;
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t sa = sbase + (uint32_t)s * p.stage_bytes;
+                const uint64_t da = desc0 + (uint64_t)(s * st16);
+                const uint32_t acc0 = kb > kb_begin ? 1u : 0u;   // each half's first MMA overwrites
                 for (int h = 0; h < p.halves; ++h) {
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = sdesc_sw128(sa + 32u * k);
-                        const uint64_t bd = sdesc_sw128(sa + a_bytes + h * bh_bytes + 32u * k);
-                        const uint32_t acc = (kb > kb_begin || k > 0) ? 1u : 0u;
+                        const uint64_t ad = da + (uint64_t)(2 * k);
+                        const uint64_t bd = da + (uint64_t)(a16 + h * bh16 + 2 * k);
                         asm volatile(
                             "{\n\t.reg .pred q;\n\t"
                             "setp.ne.b32 q, %4, 0;\n\t"
                             "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, q;\n\t}"
-                            ::"r"(tmem_base + (uint32_t)(h * 256)), "l"(ad), "l"(bd), "r"(p.idesc), "r"(acc));
+                            ::"r"(tmem_base + (uint32_t)(h * 256)), "l"(ad), "l"(bd), "r"(p.idesc),
+                              "r"(k > 0 ? 1u : acc0));
                     }
                 }
                 umma_commit<1>(empty_bar(s));
                 drain_counts[NPROD] = it + 1;
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
             if (ok) umma_commit<1>(accf);
         }
@@ -1145,10 +1172,12 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 *(volatile int *)abort_flag = 1;
             }
         } else {
+            // every MMA has completed, so the operand ring is free for the logit tile
             tc_fence_after();
-            const int64_t row = row0 + 32 * q + lane;
+            const int lrow = 32 * q + lane;
+            const int64_t row = row0 + lrow;
             const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
-            float *dst = p.ks > 1 ? p.partial + ((int64_t)rank * p.T + row) * p.E : p.r + row * p.E;
+            float *srow = tile + lrow * ld;
             for (int c = 32 * hset; c < p.E; c += 64) {
                 uint32_t v[32];
                 asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -1162,15 +1191,14 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                                "=r"(v[31])
                              : "r"(tq + (uint32_t)c));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (row < p.T) {
-                    float f[32];
+                float f[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        f[i] = __uint_as_float(v[i]);
-                        if (p.ks == 1) f[i] = sigmoidf_(f[i]);
-                    }
-                    store32(dst + c, f);
+                for (int i = 0; i < 32; ++i) {
+                    f[i] = __uint_as_float(v[i]);
+                    if (p.ks == 1) f[i] = sigmoidf_(f[i]);
+                    srow[c + i] = f[i];        // rows E + 1 floats apart: lanes hit distinct banks
                 }
+                if (p.ks == 1 && row < p.T) store32(p.r + row * p.E + c, f);
             }
         }
     }
@@ -1179,15 +1207,22 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     __threadfence();
     tc_fence_before();
     __syncthreads();
-    if (p.ks > 1) cluster_sync();     // every rank's partial logits are written and visible
+    if (p.ks > 1) cluster_sync();     // every rank's partial logit tile is written and visible
 
     // ---------------------------------------------------------------- top-k, one warp per token
     if (!*(volatile int *)abort_flag) {
         const int own = 128 / p.ks;
-        const int64_t t0 = row0 + (int64_t)rank * own;
+        uint32_t peer[RT_MAX_KS];     // the logit tile in each CTA of the cluster
+#pragma unroll
+        for (int qq = 0; qq < RT_MAX_KS; ++qq) peer[qq] = qq < p.ks ? map_to_rank(sbase, (uint32_t)qq) : 0u;
+        float bias[EPL];              // this lane's experts' selection biases, for every token
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) bias[j] = lane + 32 * j < p.E ? p.bias[lane + 32 * j] : 0.f;
         for (int i = warp; i < own; i += THREADS / 32) {
-            const int64_t t = t0 + i;
+            const int lrow = rank * own + i;
+            const int64_t t = row0 + lrow;
             if (t >= p.T) break;
+            float *srow = tile + lrow * ld;
             float v[EPL];
             int ix[EPL];
 #pragma unroll
@@ -1197,23 +1232,30 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 float r = 0.f;
                 if (e < p.E) {
                     if (p.ks == 1) {
-                        r = p.r[t * p.E + e];
+                        r = srow[e];
                     } else {
+                        float part[RT_MAX_KS];
+                        const uint32_t off = 4u * (uint32_t)(lrow * ld + e);
+#pragma unroll
+                        for (int qq = 0; qq < RT_MAX_KS; ++qq) part[qq] = qq < p.ks ? ld_cluster_f32(peer[qq] + off) : 0.f;
                         float a = 0.f;
-                        for (int qq = 0; qq < p.ks; ++qq) a += __ldcg(p.partial + ((int64_t)qq * p.T + t) * p.E + e);
+#pragma unroll
+                        for (int qq = 0; qq < RT_MAX_KS; ++qq)
+                            if (qq < p.ks) a += part[qq];   // rank order
                         r = sigmoidf_(a);
                         p.r[t * p.E + e] = r;
+                        srow[e] = r;      // this CTA's own rows: no peer reads them
                     }
                 }
-                v[j] = e < p.E ? biased_key(r, p.bias[e]) : -INFINITY;
+                v[j] = e < p.E ? biased_key(r, bias[j]) : -INFINITY;
             }
             int mine0, mine1;
             float cv;
             warp_topk<EPL>(v, ix, p.k, p.E, lane, &mine0, &mine1, &cv);
             if (lane == 0) p.cutoff[t] = cv;
             __syncwarp();                 // this token's r, written by every lane, is visible
-            const float r0 = lane < p.k ? p.r[t * p.E + mine0] : 0.f;
-            const float r1 = lane + 32 < p.k ? p.r[t * p.E + mine1] : 0.f;
+            const float r0 = lane < p.k ? srow[mine0] : 0.f;
+            const float r1 = lane + 32 < p.k ? srow[mine1] : 0.f;
             float sum = r0 + r1;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -1232,6 +1274,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             }
         }
     }
+    if (p.ks > 1) cluster_sync();     // no CTA leaves while a peer may still read its logit tile
 
     __syncthreads();
     if (*(volatile int *)abort_flag && threadIdx.x == 0) {
@@ -1256,7 +1299,6 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                      : "memory");
 }
 
-constexpr int RT_SMEM_FIXED = 1024 + 256;   // alignment slack, barriers and flags
 
 // Stages and bytes of the router + top-k kernel for E experts.
 void rt_shape(int E, int *halves, int *n_half, int *stages, int *stage_bytes, int *tmem_cols)
@@ -1355,17 +1397,26 @@ namespace lmoe {
 
 int tc_router_topk_splits(int64_t T, int E, int d)
 {
-    if (T <= 0 || E > 512 || E % 32 || (E > 256 && E != 512) || d % BK) return 0;
+    // the logit tile (128 rows of E + 1 floats) must fit in the drained operand ring
+    if (T <= 0 || E > 256 || E % 32 || d % BK) return 0;
+    int halves, n_half, stages, stage_bytes, tmem_cols;
+    rt_shape(E, &halves, &n_half, &stages, &stage_bytes, &tmem_cols);
+    if ((size_t)128 * (E + 1) * sizeof(float) > (size_t)stages * stage_bytes) return 0;
     const int sms = g_num_sms > 0 ? g_num_sms : 148;
     const int64_t tiles = (T + 127) / 128;
     const int nkb_total = 3 * (d / BK);
     int ks = 1;
-    while (ks < 8 && tiles * ks * 2 <= sms && 2 * ks * 2 <= nkb_total) ks *= 2;
-    return ks;
+    while (ks < RT_MAX_KS && tiles * ks * 2 <= sms && 2 * ks * 2 <= nkb_total) ks *= 2;
+    // One CTA per tile leaves 128 tokens' top-k to its 13 warps, one token after
+    // another; measured on B200 (T = 16384, E = 256, k = 6) that phase is latency
+    // bound (about 1100 instructions per token at 13 cycles each) and the router
+    // GEMM plus the one-warp-per-token top-k kernel is faster.  From two CTAs per
+    // tile on, the fused launch is as fast or faster (T = 4096, E = 256).
+    return ks >= 2 ? ks : 0;
 }
 
 cudaError_t tc_router_topk(const bf16 *x, const bf16 *Wr3, const float *bias, int64_t T, int E, int d, int k,
-                           float *partial, float *r, int32_t *sel, float *p32, void *p_out, int out_bf16,
+                           float *r, int32_t *sel, float *p32, void *p_out, int out_bf16,
                            float *cutoff, int32_t *blockhist, int32_t *status, cudaStream_t s)
 {
     const int ks = tc_router_topk_splits(T, E, d);
@@ -1381,7 +1432,6 @@ cudaError_t tc_router_topk(const bf16 *x, const bf16 *Wr3, const float *bias, in
     rt_shape(E, &p.halves, &p.n_half, &p.stages, &p.stage_bytes, &p.tmem_cols);
     p.idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.n_half >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
     p.bias = bias;
-    p.partial = partial;
     p.r = r;
     p.sel = sel;
     p.p32 = p32;

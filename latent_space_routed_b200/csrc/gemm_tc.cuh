@@ -41,13 +41,14 @@ cudaError_t tc_gemm_router(const bf16 *Wr3, const GemmArgs &g, int cg, int32_t *
 // cores, fp32 router through its three-term bf16 split Wr3 = [3, E, d]) for
 // T tokens of x [T, d]: r [T, E] fp32, sel / p32 / p_out (token dtype) [T, k],
 // the Quantile-Balancing cutoff [T] and the per-32-token expert counts added
-// into blockhist [E][ceil(T / 32)] (zeroed by the caller).  partial holds
-// splits * T * E floats when tc_router_topk_splits() > 1.
+// into blockhist [E][ceil(T / 32)] (zeroed by the caller).  The split
+// logits are summed through the cluster's shared memory: no workspace.
 // tc_router_topk_splits: CTAs per 128-token tile (a cluster), or 0 when this
-// path does not apply (E > 512, E not a multiple of 32, 256 < E < 512).
+// path does not apply (E > 256 or E not a multiple of 32) or does not pay
+// (tiles enough to give every CTA a whole 128-token tile of its own).
 int tc_router_topk_splits(int64_t T, int E, int d);
 cudaError_t tc_router_topk(const bf16 *x, const bf16 *Wr3, const float *bias, int64_t T, int E, int d, int k,
-                           float *partial, float *r, int32_t *sel, float *p32, void *p_out, int out_bf16,
+                           float *r, int32_t *sel, float *p32, void *p_out, int out_bf16,
                            float *cutoff, int32_t *blockhist, int32_t *status, cudaStream_t s);
 
 }  // namespace lmoe

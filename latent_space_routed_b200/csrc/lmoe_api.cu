@@ -172,7 +172,7 @@ SplitPlan plan_splits(const lmoe_handle *h, int64_t T)
     sp.shared = gemv ? 1 : plan_ksplit(h, T, 4 * (int64_t)c.f_shared, c.d / TC_BK);
     sp.final_ = gemv ? 1 : plan_ksplit(h, T, c.d, ld_hs / TC_BK);
     auto need = [&](int ks, int64_t n) -> size_t { return ks > 1 ? (size_t)ks * (size_t)n * (size_t)T : 0; };
-    sp.partial_floats = std::max(need(sp.router, c.E), need(sp.final_, c.d));
+    sp.partial_floats = std::max(need(sp.fused_router ? 1 : sp.router, c.E), need(sp.final_, c.d));
     sp.partial_side_floats = std::max(need(sp.down, c.l), need(sp.shared, 4 * (int64_t)c.f_shared));
     return sp;
 }
@@ -590,7 +590,7 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
             a.n_touched = status + CTL_NTOUCHED; a.ticket = status + CTL_TICKET;
             LMOE_CUDA(launch_route_small(a, tk, q));
         } else if (fused_router) {   // router, sigmoid, top-k and p in one launch
-            LMOE_CUDA(tc_router_topk((const bf16 *)x, h->Wr3, h->b, T, c.E, c.d, c.k, partial, r32, selected_experts,
+            LMOE_CUDA(tc_router_topk((const bf16 *)x, h->Wr3, h->b, T, c.E, c.d, c.k, r32, selected_experts,
                                      p32, mixture_weights, tk, (float *)(ws + L.cutoff), blockhist, status, q));
         } else if (router_partial) {
             // raw logits in split-K slabs; the top-k kernel sums them and applies the sigmoid
