@@ -747,7 +747,7 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     // blocks on the same SMs.  The caller's stream waits for z before the
     // permute, and for the shared GEMM before the routed gate/up GEMM: the
     // routed GEMMs then start with every SM free, as their static tile
-    // schedule wants.  (A down-projection that writes z straight into the k
+    // schedule wants (with a few tokens, before the final GEMV instead).  (A down-projection that writes z straight into the k
     // slot rows from its epilogue, after the dispatch, was measured 5x slower
     // than this GEMM plus the row-contiguous permute.)
     {
@@ -768,10 +768,15 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     // a later record on the in-order side stream covers this forward's GEMMs too
     LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_z, 0));
     RUN(st_permute(s));
-    LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
+    // Weight-streaming GEMVs (a few tokens) share HBM, not SMs: the routed
+    // ones start as soon as z and the routing are ready, and only the final
+    // GEMV, which reads the shared experts' output, waits for the side stream.
+    const bool join_late = gemv_experts(h, T);
+    if (!join_late) LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
     RUN(st_gate_up(s));
     RUN(st_down_combine(s));
     RUN(st_combine_norm(s));
+    if (join_late) LMOE_CUDA(cudaStreamWaitEvent(s, h->ev_join, 0));
     RUN(st_final(s));
 #undef RUN
     return LMOE_OK;

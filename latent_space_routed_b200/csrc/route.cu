@@ -413,7 +413,10 @@ route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, con
     if (threadIdx.x == 0) *ticket = 0;
 }
 
-// Zp[m, :] = z[perm_tok[m], :]: one warp per slot row, 16-byte vectors.
+// Zp[m, :] = z[perm_tok[m], :]: one warp per slot row, 16-byte vectors, up
+// to PERMUTE_U loads in flight per lane before their stores (with one, the
+// copy is latency bound well below the HBM rate).
+constexpr int PERMUTE_U = 4;
 __global__ void __launch_bounds__(256)
 permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ perm_tok, uint4 *__restrict__ Zp,
                     int64_t S, int vec_per_row)
@@ -425,7 +428,15 @@ permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ per
     const int lane = threadIdx.x & 31;
     const uint4 *src = z + (int64_t)perm_tok[m] * vec_per_row;
     uint4 *dst = Zp + m * vec_per_row;
-    for (int i = lane; i < vec_per_row; i += 32) dst[i] = src[i];
+    for (int i0 = lane; i0 < vec_per_row; i0 += 32 * PERMUTE_U) {
+        uint4 v[PERMUTE_U];
+#pragma unroll
+        for (int u = 0; u < PERMUTE_U; ++u)
+            if (i0 + 32 * u < vec_per_row) v[u] = src[i0 + 32 * u];
+#pragma unroll
+        for (int u = 0; u < PERMUTE_U; ++u)
+            if (i0 + 32 * u < vec_per_row) dst[i0 + 32 * u] = v[u];
+    }
 }
 
 }  // namespace
