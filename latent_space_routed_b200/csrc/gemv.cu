@@ -61,7 +61,8 @@ constexpr int DV_WARPS = 8;      // dense: warps per block (split K)
 
 template <int TT, int MODE>
 __global__ void __launch_bounds__(DV_WARPS * 32)
-dense_gemv_kernel(const bf16 *__restrict__ x, int64_t ldx, int T, int K, const bf16 *__restrict__ W, int N, EpiArgs e)
+dense_gemv_kernel(const bf16 *__restrict__ x, int64_t ldx, int T, int K, const bf16 *__restrict__ W, int64_t ldw, int N,
+                  EpiArgs e)
 {
     __shared__ float part[DV_WARPS][TT][DV_ROWS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -93,7 +94,7 @@ dense_gemv_kernel(const bf16 *__restrict__ x, int64_t ldx, int T, int K, const b
     for (int c = warp * 32 + lane; c < nv; c += DV_WARPS * 32) {
         uint4 wv[DV_ROWS];
 #pragma unroll
-        for (int r = 0; r < DV_ROWS; ++r) wv[r] = ld_stream(W + rows[r] * K + (int64_t)c * 8);
+        for (int r = 0; r < DV_ROWS; ++r) wv[r] = ld_stream(W + rows[r] * ldw + (int64_t)c * 8);
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
             if (t < T) {
@@ -135,6 +136,11 @@ dense_gemv_kernel(const bf16 *__restrict__ x, int64_t ldx, int T, int K, const b
         float v = 0.f;
 #pragma unroll
         for (int w = 0; w < DV_WARPS; ++w) v += part[w][t][r];
+        if (MODE == EPI_STORE_F32) {   // fp32 partial of a GEMV split along K
+            ((float *)e.out)[(int64_t)t * e.ldo + n] = v;
+            return;
+        }
+        if (e.residual32) v += e.residual32[(int64_t)t * e.ldo + n];
         if (e.residual) v += __bfloat162float(((const bf16 *)e.residual)[(int64_t)t * e.ldr + n]);
         out[(int64_t)t * e.ldo + n] = __float2bfloat16_rn(v);
     }
@@ -307,9 +313,12 @@ cudaError_t run_dense(int mode, const GemmArgs &g, cudaStream_t s)
     const bf16 *x = (const bf16 *)g.A, *W = (const bf16 *)g.B;
     if (mode == EPI_GLU)
         return launch_pdl(dense_gemv_kernel<TT, EPI_GLU>, dim3((unsigned)(g.N / 4)), dim3(DV_WARPS * 32), 0, s, x,
-                          g.lda, g.M, g.K, W, g.N, g.epi);
+                          g.lda, g.M, g.K, W, g.ldb, g.N, g.epi);
+    if (mode == EPI_STORE_F32)
+        return launch_pdl(dense_gemv_kernel<TT, EPI_STORE_F32>, dim3((unsigned)((g.N + DV_ROWS - 1) / DV_ROWS)),
+                          dim3(DV_WARPS * 32), 0, s, x, g.lda, g.M, g.K, W, g.ldb, g.N, g.epi);
     return launch_pdl(dense_gemv_kernel<TT, EPI_STORE>, dim3((unsigned)((g.N + DV_ROWS - 1) / DV_ROWS)),
-                      dim3(DV_WARPS * 32), 0, s, x, g.lda, g.M, g.K, W, g.N, g.epi);
+                      dim3(DV_WARPS * 32), 0, s, x, g.lda, g.M, g.K, W, g.ldb, g.N, g.epi);
 }
 
 }  // namespace
@@ -317,8 +326,8 @@ cudaError_t run_dense(int mode, const GemmArgs &g, cudaStream_t s)
 cudaError_t launch_gemv(int mode, const GemmArgs &g, cudaStream_t s)
 {
     if (g.M < 1 || g.M > GEMV_MAX_T) return cudaErrorInvalidValue;
-    if (mode != EPI_STORE && mode != EPI_GLU) return cudaErrorInvalidValue;
-    if (g.K % 8 || g.lda % 8 || g.ldb != g.K) return cudaErrorInvalidValue;
+    if (mode != EPI_STORE && mode != EPI_GLU && mode != EPI_STORE_F32) return cudaErrorInvalidValue;
+    if (g.K % 8 || g.lda % 8 || g.ldb % 8 || g.ldb < g.K) return cudaErrorInvalidValue;
     if (mode == EPI_GLU && (g.N % 4 || g.epi.ib % 2)) return cudaErrorInvalidValue;
     if (((uintptr_t)g.A | (uintptr_t)g.B) & 15u) return cudaErrorMisalignedAddress;
     if (g.M <= 1) return run_dense<1>(mode, g, s);

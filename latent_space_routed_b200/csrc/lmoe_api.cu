@@ -71,7 +71,7 @@ int64_t hs_cols(const lmoe_config &c) { return 2 * (int64_t)c.f_shared + (c.stan
 
 struct Layout {
     size_t r32, p32, blockhist, base, counts, offsets, tile_off, slot_of, perm_tok, perm_w, z, Zp, H, Yp, HS, partial,
-        partial_side, cutoff, status, touched;
+        partial_side, cutoff, status, touched, final32;
     size_t total;
 };
 
@@ -130,6 +130,11 @@ constexpr int SPLIT_MAX = 16;
 // Few-token plans of the tensor-core path.
 bool small_route(const lmoe_handle *h, int64_t T) { return h->tc && T <= ROUTE_SMALL_MAX_T; }
 bool gemv_experts(const lmoe_handle *h, int64_t T) { return h->tc && T <= GEMV_MAX_T; }
+// Few tokens, latent form: the final GEMV's shared-expert columns (K = 2 f_s of
+// 2 f_s + l) run as their own GEMV into an fp32 partial on the side stream,
+// beside the routed GEMVs; the final GEMV after the combine + RMSNorm then
+// streams only W_up and adds the partial.
+bool split_final(const lmoe_handle *h, int64_t T) { return gemv_experts(h, T) && !h->cfg.standard; }
 
 // K splits for a dense GEMM of M rows, N columns on (128 cg) x 256 tiles, nkb
 // k-blocks of 64.
@@ -229,6 +234,7 @@ Layout plan(const lmoe_handle *h, int64_t T)
     L.partial_side = take(sizeof(float) * sp.partial_side_floats);
     L.cutoff = take(sizeof(float) * T);
     L.touched = take(sizeof(int32_t) * c.E);
+    L.final32 = take(split_final(h, T) ? sizeof(float) * T * c.d : 0);
     L.total = o;
     return L;
 }
@@ -466,7 +472,8 @@ lmoe_status lmoe_launch_count(const lmoe_handle *h, int64_t T, int32_t *launches
     const lmoe_config &c = h->cfg;
     const SplitPlan sp = plan_splits(h, T);
     *launches = 11 - (c.standard ? 1 : 0) + (sp.down > 1) + (sp.shared > 1) + (sp.final_ > 1) -
-                (small_route(h, T) ? 3 : 0) - (gemv_experts(h, T) ? 1 : 0) - (sp.fused_router ? 1 : 0);
+                (small_route(h, T) ? 3 : 0) - (gemv_experts(h, T) ? 1 : 0) - (sp.fused_router ? 1 : 0) +
+                (split_final(h, T) ? 1 : 0);
     return LMOE_OK;
 }
 
@@ -706,8 +713,26 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         else LMOE_CUDA(launch_simt_gemm(EPI_GLU, tk, tk, tk, gs, 0, q));
         return LMOE_OK;
     };
+    // split final GEMV: [h_s] [D_s1 | D_s2]^T into fp32, then n W_up^T + that
+    float *final32 = (float *)(ws + L.final32);
+    const bool split_fin = split_final(h, T);
+    auto st_final_shared = [&](cudaStream_t q) -> lmoe_status {
+        GemmArgs g = gf;
+        g.K = 2 * c.f_shared;
+        g.epi.out = final32;
+        g.epi.ldo = c.d;
+        LMOE_CUDA(launch_gemv(EPI_STORE_F32, g, q));
+        return LMOE_OK;
+    };
     auto st_final = [&](cudaStream_t q) -> lmoe_status {
-        if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_STORE, gf, q));
+        if (split_fin) {
+            GemmArgs g = gf;
+            g.A = (const char *)HS + h->tb * 2 * (int64_t)c.f_shared;
+            g.B = (const char *)h->Wcat + h->tb * 2 * (int64_t)c.f_shared;
+            g.K = c.l;
+            g.epi.residual32 = final32;
+            LMOE_CUDA(launch_gemv(EPI_STORE, g, q));
+        } else if (h->tc && T <= GEMV_MAX_T) LMOE_CUDA(launch_gemv(EPI_STORE, gf, q));
         else if (h->tc) LMOE_CUDA(dense_tc(EPI_STORE, gf, sp.final_, partial, q));
         else LMOE_CUDA(launch_simt_gemm(EPI_STORE, tk, tk, tk, gf, 0, q));
         return LMOE_OK;
@@ -733,7 +758,9 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         STAGE(7); RUN(st_down_combine(s));
         STAGE(8); RUN(st_combine_norm(s));
         STAGE(9); RUN(st_shared(s));
-        STAGE(10); RUN(st_final(s));
+        STAGE(10);
+        if (split_fin) RUN(st_final_shared(s));
+        RUN(st_final(s));
         STAGE(LMOE_NUM_STAGES);
 #undef STAGE
         return LMOE_OK;
@@ -759,6 +786,7 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
         RUN(st_down(h->side));
         LMOE_CUDA(cudaEventRecord(h->ev_z, h->side));
         RUN(st_shared(h->side));
+        if (split_fin) RUN(st_final_shared(h->side));
         LMOE_CUDA(cudaEventRecord(h->ev_join, h->side));
     }
     RUN(st_router(s));

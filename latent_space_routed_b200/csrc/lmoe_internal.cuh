@@ -93,6 +93,7 @@ struct EpiArgs {
     int ib;                  // EPI_GLU: gate/up interleave block (columns)
     const void *residual;    // EPI_STORE: out = C + residual[m, n] (token dtype) when not NULL
     int64_t ldr;             // row stride of residual, elements
+    const float *residual32; // dense GEMV, EPI_STORE: out = C + residual32[m, n] (fp32, row stride ldo) when not NULL
 };
 
 // Write n <= 32 consecutive values v[0..n) of row `row` starting at output column `col`.
@@ -174,9 +175,10 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
 cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, int N, int mode, int act, float gate_cap,
                                  float up_cap, int ib, void *out, int64_t ldo, cudaStream_t s,
                                  const void *residual = nullptr, int64_t ldr = 0);
-// Dense bf16 GEMM of a few tokens (g.M = T <= GEMV_MAX_T, rows of B
-// contiguous, K a multiple of 8) on CUDA cores, streaming B: EPI_STORE (with
-// the optional residual) or EPI_GLU (gate/up rows interleaved in blocks of ib).
+// Dense bf16 GEMM of a few tokens (g.M = T <= GEMV_MAX_T, B rows g.ldb >= K
+// elements apart, K a multiple of 8) on CUDA cores, streaming B: EPI_STORE
+// (with the optional residual and fp32 residual32), EPI_STORE_F32 (fp32
+// output) or EPI_GLU (gate/up rows interleaved in blocks of ib).
 constexpr int GEMV_MAX_T = 4;
 cudaError_t launch_gemv(int mode, const GemmArgs &g, cudaStream_t s);
 // The routed experts' GEMMs of a few slot rows per expert, streaming only the
