@@ -17,9 +17,9 @@
 // The standard-MoE form (config.standard) skips 5, permutes x, skips the norm
 // in 9 and computes y = h_s [D_s1 | D_s2]^T + u in 11.
 //
-// Tensor-core path: for E <= 512 (a multiple of 32, not between 256 and 512)
-// stages 1 and 2 are one launch (tc_router_topk: router GEMM, sigmoid, top-k,
-// p, cutoff, per-block counts).  Few tokens: up to ROUTE_SMALL_MAX_T tokens,
+// Tensor-core path: for E <= 256 (a multiple of 32) and tiles split over a
+// cluster, stages 1 and 2 are one launch (tc_router_topk: router GEMM,
+// sigmoid, top-k, p, cutoff, per-block counts).  Few tokens: up to ROUTE_SMALL_MAX_T tokens,
 // stages 1-4 are one launch (route_small_kernel); up to GEMV_MAX_T tokens the
 // dense GEMMs and the routed experts' GEMMs are weight-streaming GEMVs, the
 // routed ones over the touched experts only, reading z through the slot ->

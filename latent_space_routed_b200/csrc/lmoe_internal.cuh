@@ -179,7 +179,10 @@ cudaError_t launch_splitk_reduce(const float *partial, int ksplit, int64_t M, in
 // elements apart, K a multiple of 8) on CUDA cores, streaming B: EPI_STORE
 // (with the optional residual and fp32 residual32), EPI_STORE_F32 (fp32
 // output) or EPI_GLU (gate/up rows interleaved in blocks of ib).
-constexpr int GEMV_MAX_T = 4;
+// (measured on B200, decode_d7168: at T = 3 and 4 the GEMVs, whose loads serve
+// only the one or two slot rows most touched experts have, took 0.60 and 0.73
+// ms against 0.42 and 0.50 ms for the tensor-core tiles; equal at T = 1, 2)
+constexpr int GEMV_MAX_T = 2;
 cudaError_t launch_gemv(int mode, const GemmArgs &g, cudaStream_t s);
 // The routed experts' GEMMs of a few slot rows per expert, streaming only the
 // touched experts' weights: g.offsets [E+1] gives each expert's slot rows

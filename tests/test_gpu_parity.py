@@ -97,8 +97,9 @@ def test_bf16_situ_tensor_cores():
 
 @pytest.mark.parametrize("T", [1, 2, 3, 6, 8, 9, 127, 129, 333])
 def test_bf16_token_counts(T):
-    """Token counts across the few-token plans (CUDA-core router and dense
-    GEMVs up to 8 tokens, split-K tensor-core GEMMs above) and ragged tiles."""
+    """Token counts across the few-token plans (one CUDA-core routing launch up
+    to 8 tokens, weight-streaming GEMVs up to 2, split-K tensor-core GEMMs
+    above) and ragged tiles."""
     run_parity(MULTI, T=T)
 
 
