@@ -103,6 +103,14 @@ def test_bf16_token_counts(T):
     run_parity(MULTI, T=T)
 
 
+@pytest.mark.parametrize("T", [6000, 2500, 200])
+def test_fused_router_cluster_sizes(T):
+    """The fused router + top-k launch with clusters of 2, 4 and 8 CTAs per
+    128-token tile (47, 20 and 2 tiles of the multi-tile case): the split
+    logits are summed over the cluster's shared memory in rank order."""
+    run_parity(MULTI, T=T)
+
+
 @pytest.mark.parametrize("E,k", [(8, 8), (64, 1), (40, 17)])
 def test_bf16_selection_extremes(E, k):
     w = li.custom(f"sel_{E}_{k}", 300, 256, 128, 256, E, k, 256, dtype="bf16", seed=22)
