@@ -30,21 +30,24 @@ def _weights(w):
     return li.weights(w)
 
 
-def _layer(w, gemm=0, act=0):
+def _layer(w, gemm=0, act=0, W=None):
     lm = _lm()
-    W = _weights(w)
+    W = _weights(w) if W is None else W
     return lm.LatentMoE(lm.config_for(w, gemm=gemm, act=act), {k: v.cuda() for k, v in W.items()})
 
 
-def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0, expert_tails=False):
+def run_parity(w, T=None, gemm=0, act="swiglu", n_rows=None, seed=0, expert_tails=False, bias=None):
     """Whole batch on the GPU; oracle on every row, or on n_rows seeded rows
     (always with the last row, and with expert_tails also every token that
-    holds an expert's last slot row, where a tile's ragged edge falls)."""
+    holds an expert's last slot row, where a tile's ragged edge falls).
+    bias replaces the workload's selection bias on both sides."""
     lm = _lm()
     T = w.T if T is None else T
     W = _weights(w)
+    if bias is not None:
+        W["b"] = bias
     x = li.tokens(w, T)
-    layer = _layer(w, gemm, lm.LMOE_ACT_SITU if act == "situ" else lm.LMOE_ACT_SWIGLU)
+    layer = _layer(w, gemm, lm.LMOE_ACT_SITU if act == "situ" else lm.LMOE_ACT_SWIGLU, W=W)
     out = layer(x.cuda())
     torch.cuda.synchronize()
     layer.check_device(T)
@@ -109,6 +112,19 @@ def test_fused_router_cluster_sizes(T):
     128-token tile (47, 20 and 2 tiles of the multi-tile case): the split
     logits are summed over the cluster's shared memory in rank order."""
     run_parity(MULTI, T=T)
+
+
+@pytest.mark.parametrize("T", [1088, 1152, 1153, 1280, 1281])
+def test_expert_row_counts_at_tile_edges(T):
+    """A selection bias far above every score sends all T tokens to the same
+    six experts, so each routed GEMM sees six experts of exactly T slot rows
+    on CTA-pair tiles: last m-tiles of 64, 128, 129, 0 and 1 rows (the first
+    two and the last run as half tiles, M = 128; 129 rows take a full tile)."""
+    b = torch.zeros(MULTI.E, dtype=torch.float32)
+    b[[3, 7, 11, 15, 19, 23]] = 10.0
+    errs, out = run_parity(MULTI, T=T, bias=b)
+    sel = out["selected_experts"].cpu()
+    assert set(sel.unique().tolist()) == {3, 7, 11, 15, 19, 23}
 
 
 @pytest.mark.parametrize("E,k", [(8, 8), (64, 1), (40, 17)])
