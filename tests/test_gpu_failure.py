@@ -42,6 +42,43 @@ def test_bounded_wait_runs_out_and_is_reported():
     layer.close()
 
 
+def test_bounded_wait_in_the_fused_router_is_reported():
+    """The fused router + top-k launch (a cluster of 8 CTAs per 128 tokens at
+    E = 32, T = 256) runs first when stage events put every stage on one
+    stream in order; the stall hook makes its MMA thread's wait run out.  Every
+    CTA of each cluster still passes both cluster barriers, the status word
+    reports it, and the next forward is bit-identical to a clean one."""
+    import ctypes
+    import latent_space_routed_b200 as lm
+    w = li.custom("failure_router", 256, 512, 128, 256, 32, 4, 256, dtype="bf16", seed=43)
+    layer = lm.LatentMoE(lm.config_for(w), {k: v.cuda() for k, v in li.weights(w).items()})
+    x = li.tokens(w).cuda()
+    ns = lm.LMOE_NUM_STAGES + 1
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(ns)]
+    for e in events:   # materialise the events before taking their handles
+        e.record()
+    torch.cuda.synchronize()
+    arr = (ctypes.c_void_p * ns)(*[e.cuda_event for e in events])
+    lm.lmoe_set_stage_events(layer.handle, arr, ns)
+    ref = {k: v.clone() for k, v in layer(x).items()}
+    torch.cuda.synchronize()
+    layer.check_device(w.T)
+
+    lm.lmoe_debug_inject(lm.LMOE_INJECT_STALL_NEXT_GEMM)
+    layer(x)
+    with pytest.raises(lm.LmoeError) as ei:
+        layer.check_device(w.T)
+    assert ei.value.status == lm.LMOE_ERR_DEVICE_TIMEOUT
+
+    out = layer(x)                       # the context is still usable
+    torch.cuda.synchronize()
+    layer.check_device(w.T)
+    lm.lmoe_set_stage_events(layer.handle, None, 0)
+    for key in ref:
+        assert torch.equal(out[key], ref[key]), key
+    layer.close()
+
+
 @pytest.mark.parametrize("T", [256, 4200])
 def test_bounded_wait_is_reported_through_the_host_entry(T):
     """lmoe_forward_host (at 4200 tokens cut into two pipelined chunks): a wait
