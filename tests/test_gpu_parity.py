@@ -117,12 +117,13 @@ def test_fused_router_cluster_sizes(T):
 ODD = li.custom("odd_k_blocks", 1100, 448, 192, 256, 32, 6, 256, dtype="bf16", seed=23)
 
 
-def test_odd_k_block_counts():
+@pytest.mark.parametrize("act", ["swiglu", "situ"])
+def test_odd_k_block_counts(act):
     """K of 7 (down-projection, shared gate/up), 3 (routed gate/up) and 11
     (final GEMM) 64-wide k-blocks on CTA-pair tiles: the last ring stage holds
     one k-block, whose partner is read past the end of K (zero fill) and not
-    multiplied."""
-    run_parity(ODD)
+    multiplied.  Both gates, on CTA-pair tiles with half tiles."""
+    run_parity(ODD, act=act)
 
 
 @pytest.mark.parametrize("T", [1088, 1152, 1153, 1280, 1281])
