@@ -52,10 +52,15 @@ namespace lmoe {
 namespace {
 
 constexpr int BN = TC_BN, BK = TC_BK;
-// Warps: 0 and 10..12 TMA producers, 1 MMA issuer / TMEM owner, 2..9 epilogue.
+// Warps: 0, 10 and 11 TMA producers, 1 MMA issuer / TMEM owner, 2..9 epilogue.
 // Each thread's tensor copies go out one after another (measured on B200: one
 // issuing thread moves 16 KB tiles at about 6.4 TB/s across the chip, two
-// threads at twice that), so up to four producers share the k-steps.
+// threads at twice that), so up to three producers share the k-steps (with
+// two k-blocks per copy that keeps the CTA-pair GEMMs fed: a fourth producer
+// warp measured no faster).  Twelve warps of 128 registers leave room on each
+// of the SM's four schedulers for a small kernel's warps beside a GEMM CTA
+// (with thirteen, one scheduler's register file is full), so the latency-bound
+// routing kernels can run beside the shared-expert GEMM.
 //
 // Producer q of P takes k-steps it = q (mod P) into ring slot it % S and first
 // waits for that slot's previous use to be consumed, by the parity of the
@@ -64,7 +69,7 @@ constexpr int BN = TC_BN, BK = TC_BK;
 // consumed: the producer's own previous wait (k-step it - P) guaranteed the
 // consumption of it - P - S, which covers it - 2 S exactly when P <= S.  So a
 // ring of S stages runs min(NPROD, S) producers.
-constexpr int NPROD = 4;
+constexpr int NPROD = 3;
 constexpr int THREADS = 32 * (2 + 8 + NPROD - 1);
 __device__ __forceinline__ int producer_index(int warp) { return warp == 0 ? 0 : (warp >= 10 ? warp - 9 : -1); }
 constexpr int TMEM_COLS = 2 * BN;
@@ -128,6 +133,7 @@ struct TcParams {
     int tma_store;              // 1: full chunks leave through TMA stores
     int load3d;                 // 1: the tensor maps are 3D (KPS k-blocks per copy)
     int half_tiles;             // 1: an expert's last m-tile of at most 64 CG rows runs as an M = 64 CG MMA
+    int no_early_launch;        // 1: launched without programmatic dependent launch
     int32_t *status;
 };
 
@@ -914,7 +920,7 @@ cudaError_t launch(const CUtensorMap &a, const CUtensorMap &ah, const CUtensorMa
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = attr;
-    lc.numAttrs = 2;
+    lc.numAttrs = p.no_early_launch ? 1 : 2;
     return cudaLaunchKernelEx(&lc, kern, a, ah, b, c, p);
 }
 
@@ -948,6 +954,7 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
 
     p.epi = g.epi;
     p.status = status;
+    p.no_early_launch = g.no_early_launch;
     p.stall_test = g_stall_next.exchange(0);
     if (p.max_tiles == 0) return cudaSuccess;
     CUtensorMap ta, tah, tb;

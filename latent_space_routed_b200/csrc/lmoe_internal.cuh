@@ -130,6 +130,10 @@ struct GemmArgs {
     const int32_t *tile_off;  // grouped: [E+1] m-tile prefix for this kernel's BM
     int E;
     EpiArgs epi;
+    // 1: launch without programmatic dependent launch, so that the kernel's
+    // CTAs take SMs only once its stream predecessor has finished (instead of
+    // waiting on them early, where another stream's kernel would run)
+    int no_early_launch;
 };
 
 // ---------------------------------------------------------------- launchers
