@@ -997,28 +997,34 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
 // Router scores, biased top-k and renormalisation in one launch ("Stable
 // LatentMoE", equations for r, T_k(x) and p_i), for E <= 256 experts.
 //
-// A cluster of KS CTAs takes one 128-token tile: CTA `rank` runs the k-blocks
-// [rank, rank + 1) * NKB / KS of the three bf16 terms of the fp32 router
-// weight (hi + mid + lo; with bf16 tokens every product is exact in fp32)
-// through tcgen05.mma into one fp32 TMEM accumulator of E columns.  Its eight
-// epilogue warps move the partial logits into its own shared memory (the
-// drained operand ring: 128 rows of E + 1 floats) or, for KS = 1,
-// r = sigmoid(logit) there and to global r.  After a cluster barrier each CTA
-// owns 128 / KS tokens of the tile: one warp per token reads the KS partial
-// logits of its row from the cluster's shared memory and sums them in rank
-// order (fixed order, deterministic), applies the sigmoid and writes r, runs
-// the warp tournament on r + b (warp_topk: equal scores to the lower index),
-// and writes the selection, p from the raw scores, the Quantile-Balancing
-// cutoff and the per-32-token expert counts that the counting sort scans.  A
-// last cluster barrier keeps every CTA's shared memory alive until its peers
-// have read it.
+// A cluster of KS >= 2 CTAs takes one 128-token tile: CTA `rank` runs the
+// k-blocks [rank, rank + 1) * NKB / KS of the three bf16 terms of the fp32
+// router weight (hi + mid + lo; with bf16 tokens every product is exact in
+// fp32) through tcgen05.mma into one fp32 TMEM accumulator of E columns.  Its
+// eight epilogue warps move the partial logits into its own shared memory (the
+// drained operand ring: 128 rows of E floats, each row's 16-byte chunks
+// swizzled by the row's low three bits so that the warps' row-per-lane stores
+// and the column-per-lane reads below hit distinct banks).  After a cluster
+// barrier each CTA owns 128 / KS tokens of the tile.  All its threads read the
+// KS partials of those rows, chunk by chunk, from the cluster's shared memory,
+// sum them in rank order (fixed order, deterministic), apply the sigmoid and
+// write r to global memory and over their own partial.  Then one warp per
+// token runs the top-k on r + b (warp_topk_radix for 9 <= k <= 32, else the
+// tournament warp_topk; equal scores to the lower index) and writes the
+// selection, p from the raw scores, the Quantile-Balancing cutoff and the
+// per-32-token expert counts that the counting sort scans.  A last cluster
+// barrier keeps every CTA's shared memory alive until its peers have read it.
 constexpr int RT_SMEM_FIXED = 1024 + 256;   // alignment slack, barriers and flags
 constexpr int RT_MAX_KS = 8;                 // CTAs per cluster (portable cluster size)
+// The GEMM's warp roles plus four warps that wait out the MMA phase and join
+// the r and top-k phases, which are latency bound.
+constexpr int RT_THREADS = THREADS + 4 * 32;
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr)
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr)
 {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
     return v;
 }
 
@@ -1042,7 +1048,7 @@ struct RtParams {
 };
 
 template <typename TO, int EPL>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(RT_THREADS, 1)
 router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const RtParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -1065,8 +1071,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
     const uint32_t accf = bar0 + 8u * (2 * STAGES);
     const int a_bytes = 128 * BK * 2, bh_bytes = p.n_half * BK * 2;
-    float *tile = reinterpret_cast<float *>(gbase);   // logit tile over the drained ring: [128][ld]
-    const int ld = p.E + 1;
+    float *tile = reinterpret_cast<float *>(gbase);   // logit tile over the drained ring: [128][E], chunk-swizzled
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -1182,9 +1187,9 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             // every MMA has completed, so the operand ring is free for the logit tile
             tc_fence_after();
             const int lrow = 32 * q + lane;
-            const int64_t row = row0 + lrow;
             const uint32_t tq = tmem_base + ((uint32_t)(32 * q) << 16);
-            float *srow = tile + lrow * ld;
+            float *srow = tile + lrow * p.E;
+            const int sw = lrow & 7;
             for (int c = 32 * hset; c < p.E; c += 64) {
                 uint32_t v[32];
                 asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -1198,14 +1203,13 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                                "=r"(v[31])
                              : "r"(tq + (uint32_t)c));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                float f[32];
+                // 16-byte chunk i of these 32 columns goes to chunk position i ^ (row & 7):
+                // the 32 rows of a warp store spread over all banks
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    f[i] = __uint_as_float(v[i]);
-                    if (p.ks == 1) f[i] = sigmoidf_(f[i]);
-                    srow[c + i] = f[i];        // rows E + 1 floats apart: lanes hit distinct banks
-                }
-                if (p.ks == 1 && row < p.T) store32(p.r + row * p.E + c, f);
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4 *>(srow + c + 4 * (i ^ sw)) =
+                        make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
             }
         }
     }
@@ -1214,55 +1218,94 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     __threadfence();
     tc_fence_before();
     __syncthreads();
-    if (p.ks > 1) cluster_sync();     // every rank's partial logit tile is written and visible
+    cluster_sync();                   // every rank's partial logit tile is written and visible
 
-    // ---------------------------------------------------------------- top-k, one warp per token
+    const int own = 128 / p.ks;       // this CTA's tokens: tile rows [rank * own, (rank + 1) * own)
+    const int nch = p.E / 4;          // 16-byte chunks per row
     if (!*(volatile int *)abort_flag) {
-        const int own = 128 / p.ks;
-        uint32_t peer[RT_MAX_KS];     // the logit tile in each CTA of the cluster
+        // ------------------------------------------------ r = sigmoid(sum of the KS partial logits)
+        // Every thread takes chunks of this CTA's rows: the KS partials of the chunk
+        // from the cluster's shared memory, summed in rank order (fixed order,
+        // deterministic), the sigmoid, r to global memory and back over this CTA's
+        // own partial (no peer reads this CTA's rows).
+        uint32_t peer[RT_MAX_KS];
 #pragma unroll
         for (int qq = 0; qq < RT_MAX_KS; ++qq) peer[qq] = qq < p.ks ? map_to_rank(sbase, (uint32_t)qq) : 0u;
+        for (int u0 = threadIdx.x; u0 < own * nch; u0 += 2 * RT_THREADS) {
+            // two chunks per thread at a time: all their loads are issued before any sum
+            float4 part[2][RT_MAX_KS];
+            uint32_t off[2];
+            int64_t tok[2];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const int u = u0 + b * RT_THREADS;
+                const int lrow = rank * own + u / nch, c4 = u % nch;
+                tok[b] = u < own * nch ? row0 + lrow : (int64_t)p.T;
+                off[b] = 4u * (uint32_t)(lrow * p.E + 4 * (c4 ^ (lrow & 7)));
+                if (tok[b] < p.T) {
+#pragma unroll
+                    for (int qq = 0; qq < RT_MAX_KS; ++qq)
+                        if (qq < p.ks) part[b][qq] = ld_cluster_f32x4(peer[qq] + off[b]);
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                if (tok[b] >= p.T) continue;
+                const int c4 = (u0 + b * RT_THREADS) % nch;
+                float4 a = part[b][0];
+#pragma unroll
+                for (int qq = 1; qq < RT_MAX_KS; ++qq)
+                    if (qq < p.ks) {
+                        a.x += part[b][qq].x;
+                        a.y += part[b][qq].y;
+                        a.z += part[b][qq].z;
+                        a.w += part[b][qq].w;
+                    }
+                a = make_float4(sigmoidf_(a.x), sigmoidf_(a.y), sigmoidf_(a.z), sigmoidf_(a.w));
+                *reinterpret_cast<float4 *>(p.r + tok[b] * p.E + 4 * c4) = a;
+                *reinterpret_cast<float4 *>(reinterpret_cast<uint8_t *>(tile) + off[b]) = a;
+            }
+        }
+    }
+    __syncthreads();                  // this CTA's rows of r are in its shared memory
+
+    if (!*(volatile int *)abort_flag) {
+        // ---------------------------------------------------------------- top-k, one warp per token
         float bias[EPL];              // this lane's experts' selection biases, for every token
 #pragma unroll
         for (int j = 0; j < EPL; ++j) bias[j] = lane + 32 * j < p.E ? p.bias[lane + 32 * j] : 0.f;
-        for (int i = warp; i < own; i += THREADS / 32) {
+        const bool radix = topk_radix(p.k);
+        // per-warp scratch of the radix selection, past the tile in the drained ring
+        uint32_t *hist = reinterpret_cast<uint32_t *>(gbase + (size_t)128 * p.E * 4 + (size_t)warp * TOPK_SCRATCH_BYTES);
+        if (radix) {
+            reinterpret_cast<uint4 *>(hist)[lane] = make_uint4(0u, 0u, 0u, 0u);
+            reinterpret_cast<uint4 *>(hist)[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
+            __syncwarp();
+        }
+        for (int i = warp; i < own; i += RT_THREADS / 32) {
             const int lrow = rank * own + i;
             const int64_t t = row0 + lrow;
             if (t >= p.T) break;
-            float *srow = tile + lrow * ld;
+            const float *srow = tile + lrow * p.E;
+            const int sw = lrow & 7;
+            auto r_of = [&](int e) { return srow[4 * ((e >> 2) ^ sw) + (e & 3)]; };
             float v[EPL];
             int ix[EPL];
 #pragma unroll
             for (int j = 0; j < EPL; ++j) {
                 const int e = lane + 32 * j;
                 ix[j] = e;
-                float r = 0.f;
-                if (e < p.E) {
-                    if (p.ks == 1) {
-                        r = srow[e];
-                    } else {
-                        float part[RT_MAX_KS];
-                        const uint32_t off = 4u * (uint32_t)(lrow * ld + e);
-#pragma unroll
-                        for (int qq = 0; qq < RT_MAX_KS; ++qq) part[qq] = qq < p.ks ? ld_cluster_f32(peer[qq] + off) : 0.f;
-                        float a = 0.f;
-#pragma unroll
-                        for (int qq = 0; qq < RT_MAX_KS; ++qq)
-                            if (qq < p.ks) a += part[qq];   // rank order
-                        r = sigmoidf_(a);
-                        p.r[t * p.E + e] = r;
-                        srow[e] = r;      // this CTA's own rows: no peer reads them
-                    }
-                }
-                v[j] = e < p.E ? biased_key(r, bias[j]) : -INFINITY;
+                v[j] = e < p.E ? biased_key(r_of(e), bias[j]) : -INFINITY;
             }
-            int mine0, mine1;
+            int mine0, mine1 = 0;
             float cv;
-            warp_topk<EPL>(v, ix, p.k, p.E, lane, &mine0, &mine1, &cv);
+            if (radix)
+                warp_topk_radix<EPL>(v, p.k, p.E, lane, hist, &mine0, &cv);
+            else
+                warp_topk<EPL>(v, ix, p.k, p.E, lane, &mine0, &mine1, &cv);
             if (lane == 0) p.cutoff[t] = cv;
-            __syncwarp();                 // this token's r, written by every lane, is visible
-            const float r0 = lane < p.k ? srow[mine0] : 0.f;
-            const float r1 = lane + 32 < p.k ? srow[mine1] : 0.f;
+            const float r0 = lane < p.k ? r_of(mine0) : 0.f;
+            const float r1 = lane + 32 < p.k ? r_of(mine1) : 0.f;
             float sum = r0 + r1;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -1281,7 +1324,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             }
         }
     }
-    if (p.ks > 1) cluster_sync();     // no CTA leaves while a peer may still read its logit tile
+    cluster_sync();                   // no CTA leaves while a peer may still read its logit tile
 
     __syncthreads();
     if (*(volatile int *)abort_flag && threadIdx.x == 0) {
@@ -1329,7 +1372,7 @@ cudaError_t launch_rt(const CUtensorMap &a, const CUtensorMap &b, const RtParams
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3((unsigned)(tiles * p.ks));
-    lc.blockDim = dim3(THREADS);
+    lc.blockDim = dim3(RT_THREADS);
     lc.dynamicSmemBytes = smem;
     lc.stream = s;
     cudaLaunchAttribute attr[2];
@@ -1404,17 +1447,18 @@ namespace lmoe {
 
 int tc_router_topk_splits(int64_t T, int E, int d)
 {
-    // the logit tile (128 rows of E + 1 floats) must fit in the drained operand ring
+    // the logit tile (128 rows of E floats) and the top-k scratch must fit in the drained operand ring
     if (T <= 0 || E > 256 || E % 32 || d % BK) return 0;
     int halves, n_half, stages, stage_bytes, tmem_cols;
     rt_shape(E, &halves, &n_half, &stages, &stage_bytes, &tmem_cols);
-    if ((size_t)128 * (E + 1) * sizeof(float) > (size_t)stages * stage_bytes) return 0;
+    if ((size_t)128 * E * sizeof(float) + (size_t)(RT_THREADS / 32) * TOPK_SCRATCH_BYTES > (size_t)stages * stage_bytes)
+        return 0;
     const int sms = g_num_sms > 0 ? g_num_sms : 148;
     const int64_t tiles = (T + 127) / 128;
     const int nkb_total = 3 * (d / BK);
     int ks = 1;
     while (ks < RT_MAX_KS && tiles * ks * 2 <= sms && 2 * ks * 2 <= nkb_total) ks *= 2;
-    // One CTA per tile leaves 128 tokens' top-k to its 13 warps, one token after
+    // One CTA per tile leaves 128 tokens' top-k to its warps, one token after
     // another; measured on B200 (T = 16384, E = 256, k = 6) that phase is latency
     // bound (about 1100 instructions per token at 13 cycles each) and the router
     // GEMM plus the one-warp-per-token top-k kernel is faster.  From two CTAs per

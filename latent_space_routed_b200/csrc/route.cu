@@ -26,9 +26,10 @@ namespace {
 constexpr int TOPK_WARPS = 8;   // one token per warp, 8 tokens per block
 constexpr int KMAX = 64;
 
-// Top-k for one token per warp (warp_topk), then the raw scores of the chosen
-// experts normalised by their sum (a fixed butterfly order, so the result does
-// not depend on timing), and each block's per-expert selection counts.
+// Top-k for one token per warp (warp_topk_radix for 9 <= k <= 32, else
+// warp_topk), then the raw scores of the chosen experts normalised by their
+// sum (a fixed butterfly order, so the result does not depend on timing), and
+// each block's per-expert selection counts.
 //
 // nsplit = 0: r_in holds the router scores r [T, E].  nsplit > 0: r_in holds
 // nsplit fp32 partial slabs [nsplit, T, E] of the router logits (split-K
@@ -40,11 +41,19 @@ topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const floa
             int E, int k, int32_t *__restrict__ sel, float *__restrict__ p32, TO *__restrict__ p_out,
             int32_t *__restrict__ blockhist, int nb, float *__restrict__ cutoff)
 {
+    extern __shared__ __align__(16) uint8_t topk_scratch[];   // TOPK_SCRATCH_BYTES per warp when radix
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t t = (int64_t)blockIdx.x * TOPK_WARPS + warp;
     griddep_wait();
     griddep_launch_dependents();
     if (t >= T) return;
+    const bool radix = topk_radix(k);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(topk_scratch + warp * TOPK_SCRATCH_BYTES);
+    if (radix) {
+        reinterpret_cast<uint4 *>(hist)[lane] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4 *>(hist)[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
+        __syncwarp();
+    }
     float v[EPL];
     int ix[EPL];
 #pragma unroll
@@ -64,9 +73,12 @@ topk_kernel(const float *__restrict__ r_in, int nsplit, float *r_out, const floa
         }
         v[i] = e < E ? biased_key(r, bias[e]) : -INFINITY;
     }
-    int mine0, mine1;
+    int mine0, mine1 = 0;
     float cv;
-    warp_topk<EPL>(v, ix, k, E, lane, &mine0, &mine1, &cv);
+    if (radix)
+        warp_topk_radix<EPL>(v, k, E, lane, hist, &mine0, &cv);
+    else
+        warp_topk<EPL>(v, ix, k, E, lane, &mine0, &mine1, &cv);
     if (lane == 0) cutoff[t] = cv;
     const float *rr = nsplit ? r_out : r_in;
     if (nsplit) __syncwarp();               // r_out of this token, written by every lane, is visible
@@ -233,8 +245,8 @@ dispatch_kernel(const int32_t *__restrict__ sel, const float *__restrict__ p32, 
 // (deterministic), and r[t, e] = sigmoid of the sum.  The block then counts
 // itself done on a ticket; the last block to finish (all scores are written
 // and, by the writers' fences, visible) does the rest:
-//   top-k of each token (one warp per token, warp_topk), the Quantile-Balancing
-//   cutoff, p from the raw scores;
+//   top-k of each token (one warp per token, as in topk_kernel), the
+//   Quantile-Balancing cutoff, p from the raw scores;
 //   the stable counting sort of the T k slots by expert in shared memory: one
 //   bit word per expert marks the tokens that chose it, counts are popcounts,
 //   offsets and the m-tile prefix (tiles of bm rows) are block scans, and slot
@@ -259,6 +271,7 @@ route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, con
     __shared__ int s_sel[ROUTE_SMALL_MAX_T * KMAX];
     __shared__ float s_p[ROUTE_SMALL_MAX_T * KMAX];
     __shared__ int s_warp[RS_WARPS];
+    __shared__ __align__(16) uint8_t scratch[RS_WARPS][TOPK_SCRATCH_BYTES];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int e = blockIdx.x;
     griddep_wait();
@@ -320,6 +333,10 @@ route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, con
 
     // ---- the last block: top-k, p, cutoff (one warp per token)
     for (int i = threadIdx.x; i < E; i += blockDim.x) s_bits[i] = 0u;
+    const bool radix = topk_radix(k);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(scratch[warp]);
+    reinterpret_cast<uint4 *>(hist)[lane] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4 *>(hist)[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
     for (int t = warp; t < T; t += RS_WARPS) {
         float v[EPL];
@@ -332,9 +349,12 @@ route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, con
             rv[i] = ee < E ? __ldcg(r + (int64_t)t * E + ee) : 0.f;
             v[i] = ee < E ? biased_key(rv[i], bias[ee]) : -INFINITY;
         }
-        int mine0, mine1;
+        int mine0, mine1 = 0;
         float cv;
-        warp_topk<EPL>(v, ix, k, E, lane, &mine0, &mine1, &cv);
+        if (radix)
+            warp_topk_radix<EPL>(v, k, E, lane, hist, &mine0, &cv);
+        else
+            warp_topk<EPL>(v, ix, k, E, lane, &mine0, &mine1, &cv);
         if (lane == 0) cutoff[t] = cv;
         const float r0 = lane < k ? __ldcg(r + (int64_t)t * E + mine0) : 0.f;
         const float r1 = lane + 32 < k ? __ldcg(r + (int64_t)t * E + mine1) : 0.f;
@@ -458,8 +478,9 @@ cudaError_t run_topk(const float *r_in, int nsplit, float *r_out, const float *b
                      int32_t *sel, float *p32, void *p_out, int32_t *blockhist, int nb, float *cutoff, cudaStream_t s)
 {
     const unsigned nblk = (unsigned)((T + TOPK_WARPS - 1) / TOPK_WARPS);
-    return launch_pdl(topk_kernel<TO, EPL>, dim3(nblk), dim3(TOPK_WARPS * 32), 0, s, r_in, nsplit, r_out, bias, T, E,
-                      k, sel, p32, (TO *)p_out, blockhist, nb, cutoff);
+    const size_t smem = topk_radix(k) ? (size_t)TOPK_WARPS * TOPK_SCRATCH_BYTES : 0;
+    return launch_pdl(topk_kernel<TO, EPL>, dim3(nblk), dim3(TOPK_WARPS * 32), smem, s, r_in, nsplit, r_out, bias, T,
+                      E, k, sel, p32, (TO *)p_out, blockhist, nb, cutoff);
 }
 
 template <typename TO>
