@@ -688,7 +688,7 @@ static lmoe_status forward_body(lmoe_handle *h, const void *x, int64_t T, void *
     };
     auto st_permute = [&](cudaStream_t q) -> lmoe_status {
         if (gemv_routed) return LMOE_OK;   // the routed GEMVs read z through the slot -> token map
-        LMOE_CUDA(launch_permute_rows(c.standard ? x : z, perm_tok, Zp, S, c.l, (int)h->tb, q));
+        LMOE_CUDA(launch_permute_tokens(c.standard ? x : z, slot_of, Zp, T, c.k, c.l, (int)h->tb, q));
         return LMOE_OK;
     };
     auto st_gate_up = [&](cudaStream_t q) -> lmoe_status {

@@ -165,8 +165,10 @@ cudaError_t launch_scan(const int32_t *blockhist, int nb, int E, int32_t *counts
 cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t *base, const int32_t *counts,
                             int64_t T, int E, int k, int bm, int32_t *offsets, int32_t *tile_off, int32_t *slot_of,
                             int32_t *perm_tok, float *perm_w, cudaStream_t s);
-cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
-                                cudaStream_t s);
+// Zp[slot_of[t, j]] = z[t] for every token t and j < k (rows of l elements of
+// elem_bytes; l elem_bytes a multiple of 16, at most 8 KB).
+cudaError_t launch_permute_tokens(const void *z, const int32_t *slot_of, void *Zp, int64_t T, int k, int l,
+                                  int elem_bytes, cudaStream_t s);
 // Yp in the token dtype.
 // hs = NULL: u only (no RMSNorm; the standard-MoE form).
 cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t T, int l, int k, float eps,

@@ -9,6 +9,7 @@
 // columns [col0, col0 + l) of the final GEMM's A operand, right after the
 // shared experts' hidden columns, so that W_up n and both shared down
 // projections are one K-concatenated GEMM.
+#include "gemm_tc.cuh"
 #include "lmoe_internal.cuh"
 
 namespace lmoe {
@@ -50,9 +51,11 @@ __device__ __forceinline__ void store8(float *p, const float *v)
 // One block per token, one thread per 8 consecutive latent columns: the
 // thread loads its columns from the token's k slot rows (eight rows in flight
 // at a time), adds them in fp32 in slot order, and keeps u in registers for
-// the norm.
-template <typename TT>
-__global__ void __launch_bounds__(1024)
+// the norm.  DEEP (few tokens, blocks on a fraction of the SMs): a register
+// budget that keeps all eight bf16 rows in flight; otherwise the compiler's
+// smaller budget, which keeps more blocks resident.
+template <typename TT, bool DEEP>
+__global__ void __launch_bounds__(1024, DEEP ? 1 : 0)
 combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_of, int l, int k, float eps,
                     TT *__restrict__ u_out, TT *__restrict__ hs, int64_t ld_hs, int64_t col0)
 {
@@ -68,6 +71,21 @@ combine_norm_kernel(const TT *__restrict__ Yp, const int32_t *__restrict__ slot_
     float u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     if (active) {
         int j = 0;
+        if (DEEP && sizeof(TT) == 2) {
+            for (; j + 8 <= k; j += 8) {  // eight rows in flight as raw 16-byte vectors, added in slot order
+                uint4 raw[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    raw[q] = *reinterpret_cast<const uint4 *>(Yp + (int64_t)slots[j + q] * l + c0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float v[8];
+                    load8(reinterpret_cast<const bf16 *>(&raw[q]), v);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) u[i] += v[i];
+                }
+            }
+        }
         for (; j + 8 <= k; j += 8) {      // eight rows in flight, added in slot order
             float v[8][8];
 #pragma unroll
@@ -260,11 +278,13 @@ cudaError_t launch_combine_norm(const void *Yp, const int32_t *slot_of, int64_t 
     if (T == 0) return cudaSuccess;
     if (k > 64 || l % 8 || l > 8192 || ld_hs % 8 || col0 % 8) return cudaErrorInvalidValue;
     const int threads = ((l / 8 + 31) / 32) * 32;
-    if (tok_bf16)
-        return launch_pdl(combine_norm_kernel<bf16>, dim3((unsigned)T), dim3(threads), 0, s, (const bf16 *)Yp, slot_of,
-                          l, k, eps, (bf16 *)u_out, (bf16 *)hs, ld_hs, col0);
-    return launch_pdl(combine_norm_kernel<float>, dim3((unsigned)T), dim3(threads), 0, s, (const float *)Yp, slot_of, l,
-                      k, eps, (float *)u_out, (float *)hs, ld_hs, col0);
+    const int sms = tc_num_sms() > 0 ? tc_num_sms() : 148;
+#define LMOE_COMBINE(TT, DEEP)                                                                                   \
+    launch_pdl(combine_norm_kernel<TT, DEEP>, dim3((unsigned)T), dim3(threads), 0, s, (const TT *)Yp, slot_of, l, k, \
+               eps, (TT *)u_out, (TT *)hs, ld_hs, col0)
+    if (tok_bf16) return T < 2 * sms ? LMOE_COMBINE(bf16, true) : LMOE_COMBINE(bf16, false);
+    return T < 2 * sms ? LMOE_COMBINE(float, true) : LMOE_COMBINE(float, false);
+#undef LMOE_COMBINE
 }
 
 cudaError_t launch_pack_glu(const void *G, const void *U, void *P, int nE, int F, int K, int ib, int elem_bytes,

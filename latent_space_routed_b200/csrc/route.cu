@@ -17,6 +17,8 @@
 // Integer-only, hence bit-exact and deterministic.
 #include <float.h>
 
+#include <algorithm>
+
 #include "lmoe_internal.cuh"
 #include "topk.cuh"
 
@@ -433,42 +435,58 @@ route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, con
     if (threadIdx.x == 0) *ticket = 0;
 }
 
-// Zp[m, :] = z[perm_tok[m], :]: one warp per slot row, 16-byte vectors, up
-// to PERMUTE_U loads in flight per lane before their stores (with one, the
-// copy is latency bound well below the HBM rate).
-constexpr int PERMUTE_U = 4;
+// Zp[slot_of[t, j], :] = z[t, :] for j < k: G warps per token, warp g holding
+// the token's z row in registers (V 16-byte vectors per lane) and storing it
+// to the slot rows j = g, g + G, ...  With many tokens G = 1: z is read once
+// and few, long-lived warps stream the slot rows' writes (the HBM traffic);
+// with few tokens G grows up to k so that enough warps share the writes.
+template <int V>
 __global__ void __launch_bounds__(256)
-permute_rows_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ perm_tok, uint4 *__restrict__ Zp,
-                    int64_t S, int vec_per_row)
+permute_tokens_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ slot_of, uint4 *__restrict__ Zp,
+                      int64_t T, int k, int G, int vec_per_row)
 {
-    const int64_t m = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int64_t w = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     griddep_wait();
     griddep_launch_dependents();
-    if (m >= S) return;
+    const int64_t t = w / G;
+    const int g = (int)(w - t * G);
+    if (t >= T) return;
     const int lane = threadIdx.x & 31;
-    const uint4 *src = z + (int64_t)perm_tok[m] * vec_per_row;
-    uint4 *dst = Zp + m * vec_per_row;
-    for (int i0 = lane; i0 < vec_per_row; i0 += 32 * PERMUTE_U) {
-        uint4 v[PERMUTE_U];
+    uint4 v[V];
 #pragma unroll
-        for (int u = 0; u < PERMUTE_U; ++u)
-            if (i0 + 32 * u < vec_per_row) v[u] = src[i0 + 32 * u];
+    for (int u = 0; u < V; ++u)
+        if (lane + 32 * u < vec_per_row) v[u] = z[t * vec_per_row + lane + 32 * u];
+    const int s0 = lane < k ? slot_of[t * k + lane] : 0;
+    const int s1 = lane + 32 < k ? slot_of[t * k + lane + 32] : 0;
+    for (int j = g; j < k; j += G) {
+        const int slot = __shfl_sync(0xffffffffu, j < 32 ? s0 : s1, j & 31);
+        uint4 *dst = Zp + (int64_t)slot * vec_per_row;
 #pragma unroll
-        for (int u = 0; u < PERMUTE_U; ++u)
-            if (i0 + 32 * u < vec_per_row) dst[i0 + 32 * u] = v[u];
+        for (int u = 0; u < V; ++u)
+            if (lane + 32 * u < vec_per_row) dst[lane + 32 * u] = v[u];
     }
 }
 
 }  // namespace
 
-cudaError_t launch_permute_rows(const void *z, const int32_t *perm_tok, void *Zp, int64_t S, int l, int elem_bytes,
-                                cudaStream_t s)
+cudaError_t launch_permute_tokens(const void *z, const int32_t *slot_of, void *Zp, int64_t T, int k, int l,
+                                  int elem_bytes, cudaStream_t s)
 {
-    if (S == 0) return cudaSuccess;
-    if (((int64_t)l * elem_bytes) % 16) return cudaErrorInvalidValue;
+    if (T == 0) return cudaSuccess;
+    if (((int64_t)l * elem_bytes) % 16 || k > KMAX) return cudaErrorInvalidValue;
     const int vpr = (int)((int64_t)l * elem_bytes / 16);
-    return launch_pdl(permute_rows_kernel, dim3((unsigned)((S + 7) / 8)), dim3(256), 0, s, (const uint4 *)z, perm_tok,
-                      (uint4 *)Zp, S, vpr);
+    // warps per token: about 4096 warps in all, at most one per slot row
+    int G = (int)std::min<int64_t>((int64_t)k, std::max<int64_t>(1, 4096 / T));
+    const dim3 grid((unsigned)((T * G + 7) / 8));
+#define LMOE_PERMUTE(V) launch_pdl(permute_tokens_kernel<V>, grid, dim3(256), 0, s, (const uint4 *)z, slot_of, \
+                                   (uint4 *)Zp, T, k, G, vpr)
+    if (vpr <= 32) return LMOE_PERMUTE(1);
+    if (vpr <= 64) return LMOE_PERMUTE(2);
+    if (vpr <= 128) return LMOE_PERMUTE(4);
+    if (vpr <= 256) return LMOE_PERMUTE(8);
+    if (vpr <= 512) return LMOE_PERMUTE(16);
+#undef LMOE_PERMUTE
+    return cudaErrorInvalidValue;
 }
 
 namespace {
