@@ -998,13 +998,15 @@ cudaError_t run(int mode, const GemmArgs &g, int max_mtiles, int nterms, int64_t
 // LatentMoE", equations for r, T_k(x) and p_i), for E <= 256 experts.
 //
 // A cluster of KS >= 2 CTAs takes one 128-token tile: CTA `rank` runs the
-// k-blocks [rank, rank + 1) * NKB / KS of the three bf16 terms of the fp32
-// router weight (hi + mid + lo; with bf16 tokens every product is exact in
-// fp32) through tcgen05.mma into one fp32 TMEM accumulator of E columns.  Its
-// eight epilogue warps move the partial logits into its own shared memory (the
-// drained operand ring: 128 rows of E floats, each row's 16-byte chunks
-// swizzled by the row's low three bits so that the warps' row-per-lane stores
-// and the column-per-lane reads below hit distinct banks).  After a cluster
+// k-blocks [rank, rank + 1) * NKB / KS of x against the same k-blocks of the
+// three bf16 terms of the fp32 router weight (hi + mid + lo; with bf16 tokens
+// every product is exact in fp32): each ring stage holds one k-block of x and
+// of all three terms, so x is loaded once for the three, and tcgen05.mma adds
+// them into one fp32 TMEM accumulator of E columns.  Its eight epilogue warps
+// move the partial logits into its own shared memory (the drained operand
+// ring: 128 rows of E floats, each row's 16-byte chunks swizzled by the row's
+// low three bits so that the warps' row-per-lane stores and the
+// column-per-lane reads below hit distinct banks).  After a cluster
 // barrier each CTA owns 128 / KS tokens of the tile.  All its threads read the
 // KS partials of those rows, chunk by chunk, from the cluster's shared memory,
 // sum them in rank order (fixed order, deterministic), apply the sigmoid and
@@ -1064,8 +1066,7 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)(blockIdx.x % p.ks);
     const int64_t row0 = (int64_t)(blockIdx.x / p.ks) * 128;
-    const int nkb_total = 3 * p.nkb;
-    const int kb_begin = rank * nkb_total / p.ks, kb_end = (rank + 1) * nkb_total / p.ks;
+    const int kb_begin = rank * p.nkb / p.ks, kb_end = (rank + 1) * p.nkb / p.ks;   // k-blocks of x
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -1111,14 +1112,14 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     *(volatile int *)abort_flag = 1;
                     break;
                 }
-                const int kb = kb_begin + it;
-                const int term = kb / p.nkb, kk = (kb % p.nkb) * BK;
+                // one stage: a k-block of x and the same k-block of all three W_r terms
+                const int kk = (kb_begin + it) * BK;
                 const uint32_t sa = sbase + (uint32_t)s * p.stage_bytes;
-                mbar_expect_tx(full_bar(s), a_bytes + p.halves * bh_bytes);
+                mbar_expect_tx(full_bar(s), a_bytes + 3 * p.halves * bh_bytes);
                 tma_load_2d<1>(sa, &tmA, full_bar(s), kk, (int)row0);
-                for (int h = 0; h < p.halves; ++h)
-                    tma_load_2d<1>(sa + a_bytes + h * bh_bytes, &tmB, full_bar(s), kk,
-                                   term * p.E + h * p.n_half);
+                for (int th = 0; th < 3 * p.halves; ++th)   // term th / halves, column half th % halves
+                    tma_load_2d<1>(sa + a_bytes + th * bh_bytes, &tmB, full_bar(s), kk,
+                                   (th / p.halves) * p.E + (th % p.halves) * p.n_half);
                 drain_counts[pw] = it + 1;
                 s += NP;
                 if (s >= STAGES) {
@@ -1151,12 +1152,15 @@ router_topk_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     break;
                 }
                 const uint64_t da = desc0 + (uint64_t)(s * st16);
-                const uint32_t acc0 = kb > kb_begin ? 1u : 0u;   // each half's first MMA overwrites
-                for (int h = 0; h < p.halves; ++h) {
+                // the three terms of this k-block, term by term, into the same accumulator;
+                // each half's first MMA of the CTA's range overwrites
+                for (int th = 0; th < 3 * p.halves; ++th) {
+                    const int h = th % p.halves;
+                    const uint32_t acc0 = (kb > kb_begin || th >= p.halves) ? 1u : 0u;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
                         const uint64_t ad = da + (uint64_t)(2 * k);
-                        const uint64_t bd = da + (uint64_t)(a16 + h * bh16 + 2 * k);
+                        const uint64_t bd = da + (uint64_t)(a16 + th * bh16 + 2 * k);
                         asm volatile(
                             "{\n\t.reg .pred q;\n\t"
                             "setp.ne.b32 q, %4, 0;\n\t"
@@ -1355,7 +1359,7 @@ void rt_shape(int E, int *halves, int *n_half, int *stages, int *stage_bytes, in
 {
     *halves = E > 256 ? 2 : 1;
     *n_half = E > 256 ? 256 : E;
-    *stage_bytes = 128 * BK * 2 + *halves * *n_half * BK * 2;
+    *stage_bytes = 128 * BK * 2 + 3 * *halves * *n_half * BK * 2;   // x and the three W_r terms
     int st = (232448 - RT_SMEM_FIXED) / *stage_bytes;
     *stages = st > 6 ? 6 : st;
     int cols = 32;
@@ -1455,9 +1459,9 @@ int tc_router_topk_splits(int64_t T, int E, int d)
         return 0;
     const int sms = g_num_sms > 0 ? g_num_sms : 148;
     const int64_t tiles = (T + 127) / 128;
-    const int nkb_total = 3 * (d / BK);
+    const int nkb = d / BK;
     int ks = 1;
-    while (ks < RT_MAX_KS && tiles * ks * 2 <= sms && 2 * ks * 2 <= nkb_total) ks *= 2;
+    while (ks < RT_MAX_KS && tiles * ks * 2 <= sms && 2 * ks <= nkb) ks *= 2;   // >= 1 k-block of x per CTA
     // One CTA per tile leaves 128 tokens' top-k to its warps, one token after
     // another; measured on B200 (T = 16384, E = 256, k = 6) that phase is latency
     // bound (about 1100 instructions per token at 13 cycles each) and the router
