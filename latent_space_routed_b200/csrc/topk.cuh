@@ -118,8 +118,8 @@ __host__ __device__ __forceinline__ bool topk_radix(int k) { return k >= 9 && k 
 // place in the selection is the number of chosen pairs ahead of it on the
 // packed key (score key, then inverted index), so that lane j holds selection
 // j: the order warp_topk gives, because both order by score and then by lower
-// index.  The cutoff is the largest key below
-// the selection, or the chosen key itself when ties were left unselected.
+// index.  The cutoff is the largest key below the selection, or the chosen key
+// itself when ties were left unselected.
 template <int EPL>
 __device__ __forceinline__ void warp_topk_radix(const float (&v)[EPL], int k, int E, int lane, uint32_t *hist,
                                                 int *mine0, float *cut)
