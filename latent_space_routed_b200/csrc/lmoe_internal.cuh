@@ -166,7 +166,7 @@ cudaError_t launch_dispatch(const int32_t *sel, const float *p32, const int32_t 
                             int64_t T, int E, int k, int bm, int32_t *offsets, int32_t *tile_off, int32_t *slot_of,
                             int32_t *perm_tok, float *perm_w, cudaStream_t s);
 // Zp[slot_of[t, j]] = z[t] for every token t and j < k (rows of l elements of
-// elem_bytes; l elem_bytes a multiple of 16, at most 8 KB).
+// elem_bytes; l elem_bytes a multiple of 16).
 cudaError_t launch_permute_tokens(const void *z, const int32_t *slot_of, void *Zp, int64_t T, int k, int l,
                                   int elem_bytes, cudaStream_t s);
 // Yp in the token dtype.

@@ -436,10 +436,11 @@ route_small_kernel(const bf16 *__restrict__ x, const float *__restrict__ Wr, con
 }
 
 // Zp[slot_of[t, j], :] = z[t, :] for j < k: G warps per token, warp g holding
-// the token's z row in registers (V 16-byte vectors per lane) and storing it
-// to the slot rows j = g, g + G, ...  With many tokens G = 1: z is read once
-// and few, long-lived warps stream the slot rows' writes (the HBM traffic);
-// with few tokens G grows up to k so that enough warps share the writes.
+// the token's z row in registers (V 16-byte vectors per lane, longer rows in
+// pieces of 32 V vectors) and storing it to the slot rows j = g, g + G, ...
+// With many tokens G = 1: z is read once and few, long-lived warps stream the
+// slot rows' writes (the HBM traffic); with few tokens G grows up to k so that
+// enough warps share the writes.
 template <int V>
 __global__ void __launch_bounds__(256)
 permute_tokens_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ slot_of, uint4 *__restrict__ Zp,
@@ -452,18 +453,20 @@ permute_tokens_kernel(const uint4 *__restrict__ z, const int32_t *__restrict__ s
     const int g = (int)(w - t * G);
     if (t >= T) return;
     const int lane = threadIdx.x & 31;
-    uint4 v[V];
-#pragma unroll
-    for (int u = 0; u < V; ++u)
-        if (lane + 32 * u < vec_per_row) v[u] = z[t * vec_per_row + lane + 32 * u];
     const int s0 = lane < k ? slot_of[t * k + lane] : 0;
     const int s1 = lane + 32 < k ? slot_of[t * k + lane + 32] : 0;
-    for (int j = g; j < k; j += G) {
-        const int slot = __shfl_sync(0xffffffffu, j < 32 ? s0 : s1, j & 31);
-        uint4 *dst = Zp + (int64_t)slot * vec_per_row;
+    for (int base = 0; base < vec_per_row; base += 32 * V) {   // one pass for rows up to 512 V bytes
+        uint4 v[V];
 #pragma unroll
         for (int u = 0; u < V; ++u)
-            if (lane + 32 * u < vec_per_row) dst[lane + 32 * u] = v[u];
+            if (base + lane + 32 * u < vec_per_row) v[u] = z[t * vec_per_row + base + lane + 32 * u];
+        for (int j = g; j < k; j += G) {
+            const int slot = __shfl_sync(0xffffffffu, j < 32 ? s0 : s1, j & 31);
+            uint4 *dst = Zp + (int64_t)slot * vec_per_row + base;
+#pragma unroll
+            for (int u = 0; u < V; ++u)
+                if (base + lane + 32 * u < vec_per_row) dst[lane + 32 * u] = v[u];
+        }
     }
 }
 
@@ -484,9 +487,8 @@ cudaError_t launch_permute_tokens(const void *z, const int32_t *slot_of, void *Z
     if (vpr <= 64) return LMOE_PERMUTE(2);
     if (vpr <= 128) return LMOE_PERMUTE(4);
     if (vpr <= 256) return LMOE_PERMUTE(8);
-    if (vpr <= 512) return LMOE_PERMUTE(16);
+    return LMOE_PERMUTE(16);   // rows above 8 KB in pieces of 8 KB
 #undef LMOE_PERMUTE
-    return cudaErrorInvalidValue;
 }
 
 namespace {

@@ -165,6 +165,14 @@ def test_bf16_pair_tiles_edge_shapes(shape):
     assert errs["output"] <= TOL["bf16"]
 
 
+def test_bf16_latent_rows_above_8_kb():
+    """l = 4160 (8320-byte bf16 rows): the permute stores each z row to its
+    slot rows in two pieces; every row is compared."""
+    w = li.custom("wide_latent", 40, 4160, 4160, 128, 16, 4, 128, dtype="bf16", seed=46)
+    errs, _ = run_parity(w)
+    assert errs["output"] <= TOL["bf16"]
+
+
 @pytest.mark.parametrize("dtype,gemm", [("bf16", 0), ("bf16", 1), ("f32", 0)])
 def test_standard_moe_form(dtype, gemm):
     """config.standard: experts at the model width on x itself, no projections
